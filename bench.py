@@ -1,0 +1,498 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse MoE FFN layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral]
+    python bench.py --impl reference ...      # the CPU oracle, on the host cores
+
+A step is one pass of the whole layer (RMS statistic + router/top-k, dispatch,
+both grouped expert GEMMs, combine) over one batch of seeded synthetic tokens,
+through ``moe_layer_fwd``.  Inputs are resident in HBM when the timed region
+starts; they are larger than L2 (2.8 GB of expert weights, 134 MB of
+activations at the Mixtral shape), so no L2 flush is done between steps.
+Timing: W untimed steps, then K steps between CUDA events on the launching
+stream, with a barrier and a device synchronisation on both sides; the time is
+the maximum over ranks.  With N > 1 each rank runs an independent replica (the
+layer has no exchange step on one GPU), so ``value`` = N * T * K / time.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import moe_workloads as mw  # noqa: E402
+
+METRIC = "MoE layer fwd tokens/s & TFLOP/s, % of B200 bf16 peak / HBM roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 7  # route, dispatch count/scatter/permute, GEMM up, GEMM down, combine
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mixtral", choices=mw.WORKLOAD_ORDER)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's token count (profiling of smaller cases)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target seconds of oracle work for the CPU baseline sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def widths_of(w: mw.Workload):
+    out = []
+    for count, size in w.expert_sizes:
+        out += [-(-int(size) // 128) * 128] * int(count)
+    return out
+
+
+def workload_config(w: mw.Workload, world: int):
+    widths = widths_of(w)
+    return {
+        "workload": f"{w.name}: {w.description}",
+        "T": w.T, "d_model": w.d_model, "E": w.E, "k": w.k,
+        "d_ffn": widths[0] if len(set(widths)) == 1 else widths,
+        "capacity_factor": w.capacity_factor if w.capacity_factor > 0 else None,
+        "seed": w.seed,
+        "l2": "inputs larger than L2 (expert weights + activations); no flush between steps",
+        "parallelism": "single GPU" if world == 1 else f"{world} independent replicas (no exchange)",
+    }
+
+
+def cores_used() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        blas = [i["num_threads"] for i in info if i.get("user_api") == "blas"]
+        if blas:
+            return int(max(blas))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.samples = []
+        self.windows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.gpu_id],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [v.strip() for v in line.split(",")]))
+
+    def window(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        inside = [s for t, s in self.samples if any(a - 0.05 <= t <= b + 0.05 for a, b in self.windows)]
+        used = inside or [s for _, s in self.samples]
+        if not used:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return float("nan")
+        sm = [num(s[1]) for s in used if len(s) > 8]
+        smax = [num(s[2]) for s in used if len(s) > 8]
+        reasons = set()
+        for s in used:
+            for name, v in zip(self.NAMES, s[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(used),
+                "samples_in_timed_region": len(inside)}
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+    import sparse_mixture_experts_rms_b200 as moe
+    from sparse_mixture_experts_rms_b200 import build as moe_build
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    if rank == 0 or not os.path.exists(moe_build.LIB_PATH):
+        moe_build.build()
+    if world > 1:
+        dist.barrier()
+    moe._lib()
+
+    w = mw.WORKLOADS[args.workload]
+    if args.tokens > 0:
+        w = w.with_tokens(args.tokens, name=w.name)
+    widths = widths_of(w)
+    dev = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+    x_bits = mw.gen_x(w)
+    W1b, W3b, W2b = mw.gen_expert_weights(w, widths)
+    x, gamma, Wr = dev(x_bits), dev(mw.gen_gamma(w)), dev(mw.gen_router_weight(w))
+    b = mw.gen_router_bias(w)
+    bias = None if b is None else torch.from_numpy(b).cuda()
+    W1, W3, W2 = dev(W1b), dev(W3b), dev(W2b)
+    del W1b, W3b, W2b
+    cfg = moe.MoEConfig(T=w.T, d_model=w.d_model, E=w.E, k=w.k,
+                        ffn_offsets=moe.ffn_offsets_from_sizes(w.expert_sizes),
+                        capacity_factor=w.capacity_factor, eps=w.eps)
+    stream = torch.cuda.Stream()
+    ws = moe.alloc_workspace(cfg)
+    out = torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device="cuda")
+    counts = torch.zeros(w.E, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+
+    props = torch.cuda.get_device_properties(local)
+    uuid = str(getattr(props, "uuid", ""))
+    sampler = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or str(local)))
+    sampler.start()
+
+    def step():
+        moe.moe_layer_fwd(cfg, x, gamma, Wr, bias, W1, W3, W2, out, ws, counts=counts, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            step()
+    stream.synchronize()
+    code = moe.moe_get_device_error(ws, stream=stream, raise_on_error=False)
+    if code:
+        raise RuntimeError(f"device error word 0x{code:x} after warm-up")
+
+    # ---- main timed region: K fused layer steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    tw0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    tw1 = time.time()
+    barrier()
+    sampler.window(tw0, tw1)
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_step = ms_total / args.steps
+
+    # ---- per-stage breakdown: the same kernels through the staged calls
+    c = cfg
+    mk = max(moe.moe_max_kept(c), 1)
+    st = {
+        "idx": torch.empty((c.T, c.k), dtype=torch.int32, device="cuda"),
+        "gate": torch.empty((c.T, c.k), dtype=torch.float32, device="cuda"),
+        "r": torch.empty((c.T,), dtype=torch.float32, device="cuda"),
+        "counts": torch.empty((c.E,), dtype=torch.int32, device="cuda"),
+        "offsets": torch.empty((c.E + 1,), dtype=torch.int32, device="cuda"),
+        "perm": torch.empty((mk,), dtype=torch.int32, device="cuda"),
+        "inv_perm": torch.empty((c.T * c.k,), dtype=torch.int32, device="cuda"),
+        "x_perm": torch.empty((mk, c.d_model), dtype=torch.bfloat16, device="cuda"),
+        "y": torch.empty((mk, c.d_model), dtype=torch.bfloat16, device="cuda"),
+        "out": torch.empty((c.T, c.d_model), dtype=torch.bfloat16, device="cuda"),
+    }
+    stages = ["route", "dispatch", "gemm_up", "gemm_down", "combine"]
+
+    def staged(evs):
+        evs[0].record(stream)
+        moe.moe_route(c, x, gamma, Wr, bias, st["idx"], st["gate"], st["r"], None, ws, stream=stream)
+        evs[1].record(stream)
+        moe.moe_dispatch(c, st["idx"], x, gamma, st["counts"], st["offsets"], st["perm"], st["inv_perm"],
+                         st["x_perm"], ws, stream=stream)
+        evs[2].record(stream)
+        moe.moe_experts_up(c, st["x_perm"], st["r"], st["perm"], st["offsets"], W1, W3, ws, stream=stream)
+        evs[3].record(stream)
+        moe.moe_experts_down(c, st["gate"], st["perm"], st["offsets"], W2, st["y"], ws, stream=stream)
+        evs[4].record(stream)
+        moe.moe_combine(c, st["y"], st["inv_perm"], st["out"], stream=stream)
+        evs[5].record(stream)
+
+    for _ in range(2):
+        staged([torch.cuda.Event(enable_timing=True) for _ in range(6)])
+    torch.cuda.synchronize()
+    n_stage_steps = max(args.steps, 5)
+    all_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_stage_steps)]
+    tw0 = time.time()
+    for evs in all_evs:
+        staged(evs)
+    torch.cuda.synchronize()
+    sampler.window(tw0, time.time())
+    stage_ms = {s: sum(ev[i].elapsed_time(ev[i + 1]) for ev in all_evs) / n_stage_steps
+                for i, s in enumerate(stages)}
+    staged_step_ms = sum(stage_ms.values())
+
+    # ---- algorithmic work (kept rows from the device's own counts)
+    counts_h = st["counts"].cpu().numpy().astype(np.int64)
+    offs_h = st["offsets"].cpu().numpy().astype(np.int64)
+    kept = np.diff(offs_h)
+    d, E, T, k = w.d_model, w.E, w.T, w.k
+    nf = float(np.sum(kept * np.array(widths, dtype=np.int64)))
+    fl_router = 2.0 * T * d * E
+    fl_up = 4.0 * d * nf
+    fl_down = 2.0 * d * nf
+    F_alg = fl_router + fl_up + fl_down
+    n_kept = int(kept.sum())
+    w_bytes = float(sum(3 * d * f * 2 for f, n in zip(widths, kept) if n > 0))
+    B_alg = 2.0 * T * d * 2 + d * 2 + d * E * 2 + w_bytes + T * k * 8 + T * 4
+    peaks = load_peaks()
+    pk_tc = peaks["bf16_tflops_sustained"] * 1e12
+    pk_tc_burst = peaks["bf16_tflops"] * 1e12
+    pk_hbm = peaks["hbm_gbs"] * 1e9
+    t_roof = max(F_alg / pk_tc, B_alg / pk_hbm)
+    t_roof_burst = max(F_alg / pk_tc_burst, B_alg / pk_hbm)
+    t_step = ms_step * 1e-3
+
+    up_s = stage_ms["gemm_up"] * 1e-3
+    achieved_up = fl_up / up_s / 1e12
+    stage_report = {
+        "route": {"ms": stage_ms["route"], "GB/s": (T * d * 2 + d * E * 2 + T * (k * 8 + 4)) / (stage_ms["route"] * 1e-3) / 1e9},
+        "dispatch": {"ms": stage_ms["dispatch"], "GB/s": (2.0 * n_kept * d * 2 + T * k * 12) / (stage_ms["dispatch"] * 1e-3) / 1e9},
+        "gemm_up": {"ms": stage_ms["gemm_up"], "TFLOP/s": achieved_up},
+        "gemm_down": {"ms": stage_ms["gemm_down"], "TFLOP/s": fl_down / (stage_ms["gemm_down"] * 1e-3) / 1e12},
+        "combine": {"ms": stage_ms["combine"], "GB/s": (n_kept * d * 2 + T * d * 2 + T * k * 4) / (stage_ms["combine"] * 1e-3) / 1e9},
+    }
+
+    # ---- end to end through the public call, host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        x_h = x.cpu().pin_memory()
+        out_h = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+        x_d = torch.empty_like(x)
+
+        def e2e_step():
+            x_d.copy_(x_h, non_blocking=True)
+            moe.moe_layer_fwd(cfg, x_d, gamma, Wr, bias, W1, W3, W2, out, ws, stream=stream)
+            out_h.copy_(out, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        tw0 = time.time()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                e2e_step()
+            e1.record(stream)
+        e1.synchronize()
+        torch.cuda.synchronize()
+        sampler.window(tw0, time.time())
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+        e2e = {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(x_h.numel() * 2), "d2h_bytes_per_step": int(out_h.numel() * 2)}
+
+    clocks = sampler.stop()
+    code = moe.moe_get_device_error(ws, stream=stream, raise_on_error=False)
+
+    result = {
+        "metric": METRIC,
+        "value": world * T / t_step,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded Philox; random-init weights of the workload's shapes)",
+        "config": workload_config(w, world),
+        "tflops": F_alg / t_step / 1e12,
+        "layer_roofline": {
+            "flops": F_alg, "bytes": B_alg, "bound": "tensor" if F_alg / pk_tc >= B_alg / pk_hbm else "hbm",
+            "t_roof_ms": t_roof * 1e3, "frac": t_roof / t_step,
+            "frac_of_burst_peak": t_roof_burst / t_step,
+            "peaks": f"{peaks['source']}: bf16 {peaks['bf16_tflops_sustained']:.0f} TFLOP/s sustained "
+                     f"({peaks['bf16_tflops']:.0f} burst), HBM {peaks['hbm_gbs']:.0f} GB/s",
+        },
+        "roofline": {
+            "kernel": "grouped_gemm_kernel (up: x_perm x [W1|W3], SwiGLU epilogue)",
+            "bound": "tensor", "achieved": achieved_up, "peak": peaks["bf16_tflops_sustained"],
+            "unit": "TFLOP/s", "frac": achieved_up / peaks["bf16_tflops_sustained"],
+            "traffic": None,
+            "peak_note": f"{peaks['source']} sustained cuBLAS bf16 (kernel timed inside long steps)",
+            "flops_per_launch": fl_up,
+        },
+        "stages": stage_report,
+        "staged_ms_per_step": staged_step_ms,
+        "kept_rows": n_kept,
+        "counts": counts_h.tolist(),
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clocks,
+        "device_error": code,
+    }
+    if e2e is not None:
+        result["e2e"] = e2e
+    if world > 1:
+        dist.barrier()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, widths, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------- oracle legs
+class OracleRunner:
+    """The CPU oracle on host cores; weights widened to float64 once (untimed)."""
+
+    def __init__(self, w: mw.Workload, widths):
+        from oracle import moe_oracle as O
+        self.O = O
+        self.w = w
+        self.widths = widths
+        self.x_bits = mw.gen_x(w)
+        self.gamma = mw.gen_gamma(w)
+        self.Wr = mw.gen_router_weight(w)
+        self.bias = mw.gen_router_bias(w)
+        W1, W3, W2 = mw.gen_expert_weights(w, widths)
+        self.W1, self.W3, self.W2 = O.as_f64(W1), O.as_f64(W3), O.as_f64(W2)
+        del W1, W3, W2
+
+    def run(self, t0: int, n: int):
+        """The oracle layer on tokens [t0, t0+n) as one batch."""
+        sl = slice(t0, t0 + n)
+        return self.O.moe_layer(self.x_bits[sl], self.gamma, self.Wr, self.bias, self.W1, self.W3,
+                                self.W2, self.widths, self.w.k, self.w.eps, self.w.capacity_factor)
+
+
+def cpu_baseline(w: mw.Workload, widths, target_s: float):
+    r = OracleRunner(w, widths)
+    n0 = min(64, w.T)
+    t = time.time()
+    r.run(0, n0)
+    dt = time.time() - t
+    n = int(min(w.T, max(n0, n0 * target_s / max(dt, 1e-3))))
+    t = time.time()
+    r.run(0, n)
+    dt = time.time() - t
+    return {"value": n / dt, "unit": UNIT, "cores": cores_used(), "kind": "oracle",
+            "sample": f"tokens [0, {n}) of the {w.name} workload as one batch through the fp64 "
+                      f"numpy oracle (all steps; weights widened to fp64 once, untimed); {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = mw.WORKLOADS[args.workload]
+    if args.tokens > 0:
+        w = w.with_tokens(args.tokens, name=w.name)
+    widths = widths_of(w)
+    r = OracleRunner(w, widths)
+    # size each step so that warm-up + timed steps take about three minutes
+    n0 = min(16, w.T)
+    t = time.time()
+    r.run(0, n0)
+    per_tok = (time.time() - t) / n0
+    budget = 180.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(w.T, budget / max(per_tok, 1e-6))))
+    pos = 0
+    for _ in range(args.warmup):
+        r.run(pos % max(1, w.T - n + 1), n)
+        pos += n
+    t = time.time()
+    for _ in range(args.steps):
+        r.run(pos % max(1, w.T - n + 1), n)
+        pos += n
+    dt = time.time() - t
+    value = n * args.steps / dt
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded Philox; random-init weights of the workload's shapes)",
+        "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores_used(), "kind": "oracle",
+                         "sample": f"each step: {n} consecutive tokens of the {w.name} workload as one "
+                                   f"batch through the fp64 numpy oracle (weights widened once, untimed)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

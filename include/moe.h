@@ -1,0 +1,212 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse MoE FFN layer forward.
+ *
+ * The layer (forward only, one GPU):
+ *   RMS statistic  r_t = 1/sqrt(mean_i x_ti^2 + eps)
+ *   router         l_te = r_t * sum_i x_ti gamma_i Wr_ie + b_e   (fp32)
+ *   top-k gating   k largest l_te (ties -> lower e, slots largest first),
+ *                  gate_tj = softmax_e(l_t)[idx_tj]  (optionally renormalised)
+ *   dispatch       per-expert histogram, expert capacity, stable permutation
+ *                  grouping assignments a = t*k+j by expert, token order inside
+ *   experts        SwiGLU per expert with variable widths f_e:
+ *                  h = silu(r_t*(xg_t W1_e)) * (r_t*(xg_t W3_e)),  y = h W2_e,
+ *                  where xg_t = x_t * gamma
+ *   combine        out_t = sum over kept slots of gate_tj * y_(t,j)
+ *
+ * Sources of each step:
+ *  - CODA sparse-MoE thread (digg.com), RMSNorm paragraphs: the statistic r is
+ *    commuted across the GEMM that follows the norm and applied in that GEMM's
+ *    epilogue -- in the router right before the top-k, and in the first expert
+ *    linear, to which r travels with the dispatched token.
+ *  - Mixture of Experts glossary (inferensys.com): gating network, top-k and
+ *    Switch (top-1) routing, expert capacity
+ *    C = (T*k)/E * capacity_factor with excess tokens dropped, fused MoE
+ *    kernels combining routing, permutation and expert matmuls.
+ *  - nanoMOE variable-size-experts notes (hbfreed.com): expert widths as
+ *    multiples of 128, concatenated weights W1 [d, F], W2 [F, d] with
+ *    cumulative column offsets ("Weight Allocation", "Offset Calculation").
+ *  - OmniMoE summary (gist.science), section 2.2 "Expert-Centric Scheduling":
+ *    routing decisions grouped by expert, sorted by token inside a group,
+ *    executed as a grouped GEMM.
+ *
+ * Conventions (all entry points):
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller; the library
+ *    allocates nothing and keeps no state between calls.  Row-major layouts.
+ *    bf16 tensors are passed as moe_bf16_t (raw bf16 bit patterns).
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t, NULL = the
+ *    legacy default stream); the return value only reports argument checks and
+ *    launch errors.  Errors detected on the device (an expert id out of range,
+ *    a bounded wait that expired) are OR-ed into an error word in the
+ *    workspace; read it with moe_get_device_error().  No kernel traps.
+ *  - Arguments are validated before anything is launched; on error nothing is
+ *    enqueued.  bf16 matrices must be 16-byte aligned, fp32/int32 arrays
+ *    4-byte aligned, the workspace 256-byte aligned.
+ *  - Limits: 1 <= k <= E <= 64, d_model a positive multiple of 128, every
+ *    expert width a positive multiple of 128, T >= 0 (T = 0 is a no-op),
+ *    T*k < 2^31.  With T = 0 every call validates cfg and returns MOE_OK;
+ *    only counts/offsets outputs are written (zeros), other pointers may be NULL.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef uint16_t moe_bf16_t; /* raw bfloat16 bits */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* bad shape, null pointer, k > E, ...          */
+  MOE_ERR_ALIGNMENT = 2,   /* a pointer is not aligned as required         */
+  MOE_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required   */
+  MOE_ERR_UNSUPPORTED = 4, /* valid but outside this build's limits        */
+  MOE_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed            */
+  MOE_ERR_DEVICE = 6,      /* the device error word is non-zero            */
+  MOE_ERR_NO_DEVICE = 7    /* no usable sm_100 device                      */
+} moe_status_t;
+
+/* Bits of the device error word (moe_get_device_error). */
+#define MOE_DEVERR_EXPERT_ID 0x1u  /* an expert id outside [0, E) reached dispatch */
+#define MOE_DEVERR_TIMEOUT 0x2u    /* a bounded pipeline wait gave up             */
+#define MOE_DEVERR_TILE_TABLE 0x4u /* kept rows exceed the buffers they index     */
+
+typedef struct {
+  int32_t T;        /* tokens                                                */
+  int32_t d_model;  /* hidden size d                                         */
+  int32_t E;        /* experts                                               */
+  int32_t k;        /* experts per token                                     */
+  /* HOST array [E+1]: cumulative expert widths, ffn_offsets[0] = 0 and
+   * ffn_offsets[e+1] - ffn_offsets[e] = f_e (a multiple of 128).  Expert e
+   * owns columns [ffn_offsets[e], ffn_offsets[e+1]) of W1/W3 and the same rows
+   * of W2 (nanoMOE notes, "Offset Calculation").  Read during the call only. */
+  const int32_t* ffn_offsets;
+  float capacity_factor; /* <= 0: dropless; else C = floor((T*k)/E * cf)   */
+  float eps;             /* RMS epsilon, e.g. 1e-5                            */
+  int32_t renormalize;   /* 0: gate = softmax over all E; 1: renormalised
+                            over the k chosen experts                       */
+} moe_config_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+MOE_API const char* moe_status_string(moe_status_t status);
+
+/* Expert capacity C of `cfg` ((T*k)/E * capacity_factor rounded down, MoE
+ * glossary "Expert Capacity"), or -1 when dropless or cfg is invalid. */
+MOE_API int64_t moe_capacity(const moe_config_t* cfg);
+
+/* Maximum number of kept assignments: T*k when dropless, else min(T*k, E*C). */
+MOE_API int64_t moe_max_kept(const moe_config_t* cfg);
+
+/* Bytes of workspace every entry point below needs for `cfg` (0 if cfg is
+ * invalid).  One workspace of this size serves all calls; it holds the device
+ * error word, the dispatch scratch and, for moe_layer_fwd, every
+ * intermediate (routing, permutation, permuted activations, the SwiGLU
+ * activations H and the per-assignment expert outputs). */
+MOE_API size_t moe_workspace_size(const moe_config_t* cfg);
+
+/* Zero the workspace header (device error word).  Call once after allocating a
+ * workspace, before its first use.  Asynchronous on `stream`. */
+MOE_API moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, copy the device error word to *code and clear it.
+ * Returns MOE_ERR_DEVICE if the word was non-zero, MOE_OK otherwise. */
+MOE_API moe_status_t moe_get_device_error(void* ws, size_t ws_bytes, void* stream, uint32_t* code);
+
+/* Route: RMS statistic, router GEMM with the statistic applied after the GEMM
+ * and before the top-k (CODA thread), softmax and top-k gating (MoE glossary,
+ * "Top-k Gating" / "Switch Routing").
+ *   x        [T, d]   bf16   activations
+ *   gamma    [d]      bf16   RMSNorm weight
+ *   Wr       [d, E]   bf16   router weight
+ *   bias     [E]      fp32   router logit bias, or NULL for none
+ *   expert_idx [T, k] int32  out: chosen experts, largest logit first
+ *   gate     [T, k]   fp32   out: softmax(l_t) at the chosen experts
+ *   r        [T]      fp32   out: RMS statistic
+ *   logits   [T, E]   fp32   out (optional, NULL to skip): router logits
+ * Logits accumulate exact bf16*bf16 products in fp32. */
+MOE_API moe_status_t moe_route(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
+                       const moe_bf16_t* Wr, const float* bias, int32_t* expert_idx, float* gate,
+                       float* r, float* logits, void* ws, size_t ws_bytes, void* stream);
+
+/* Dispatch: histogram, capacity, expert-centric permutation (OmniMoE summary,
+ * "Expert-Centric Scheduling"; MoE glossary, "Expert Capacity"), and the
+ * permuted, gamma-scaled activations the expert GEMMs read.
+ *   expert_idx [T, k]   int32  in
+ *   x          [T, d]   bf16   in (activations, as given to moe_route)
+ *   gamma      [d]      bf16   in
+ *   counts     [E]      int32  out: assignments per expert (before capacity)
+ *   expert_offsets [E+1] int32 out: exclusive running sum of kept counts
+ *   perm       [T*k]    int32  out: perm[p], p < n_kept, is the assignment
+ *                              a = t*k+j kept at position p (grouped by
+ *                              expert, token order inside a group)
+ *   inv_perm   [T*k]    int32  out: position of assignment a, -1 if dropped
+ *   x_perm     [T*k, d] bf16   out: x_perm[p] = bf16(x_t * gamma), t = perm[p]/k
+ * The number of kept assignments is expert_offsets[E]; rows of perm/x_perm at
+ * and beyond it are left untouched. */
+MOE_API moe_status_t moe_dispatch(const moe_config_t* cfg, const int32_t* expert_idx, const moe_bf16_t* x,
+                          const moe_bf16_t* gamma, int32_t* counts, int32_t* expert_offsets,
+                          int32_t* perm, int32_t* inv_perm, moe_bf16_t* x_perm, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/* Experts: the two grouped GEMMs over the expert-centric order.
+ *   x_perm   [T*k, d] bf16   in (moe_dispatch)
+ *   r        [T]      fp32   in (moe_route): applied in GEMM 1's epilogue
+ *   gate     [T, k]   fp32   in (moe_route): applied in GEMM 2's epilogue
+ *   perm, expert_offsets     in (moe_dispatch)
+ *   W1, W3   [d, F]   bf16   expert e = columns ffn_offsets[e] .. [e+1]
+ *   W2       [F, d]   bf16   expert e = rows    ffn_offsets[e] .. [e+1]
+ *   y        [T*k, d] bf16   out: y[p] = bf16(gate_a * FFN_e(x_t)), a = perm[p],
+ *                            for p < expert_offsets[E] (expert-centric order)
+ * Uses the workspace for H (the SwiGLU activations). */
+MOE_API moe_status_t moe_experts_fwd(const moe_config_t* cfg, const moe_bf16_t* x_perm, const float* r,
+                             const float* gate, const int32_t* perm,
+                             const int32_t* expert_offsets, const moe_bf16_t* W1,
+                             const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* y, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* The two halves of moe_experts_fwd, for callers that schedule them apart.
+ * moe_experts_up runs GEMM 1 (x_perm x (W1 | W3), r and SwiGLU in the
+ * epilogue) and leaves H in the workspace; moe_experts_down runs GEMM 2
+ * (H x W2, gate in the epilogue) on that H and writes y.  Same arguments and
+ * layouts as moe_experts_fwd; the workspace must be the same between the two
+ * calls and must not be used by another call in between. */
+MOE_API moe_status_t moe_experts_up(const moe_config_t* cfg, const moe_bf16_t* x_perm, const float* r,
+                                    const int32_t* perm, const int32_t* expert_offsets,
+                                    const moe_bf16_t* W1, const moe_bf16_t* W3, void* ws,
+                                    size_t ws_bytes, void* stream);
+MOE_API moe_status_t moe_experts_down(const moe_config_t* cfg, const float* gate, const int32_t* perm,
+                                      const int32_t* expert_offsets, const moe_bf16_t* W2,
+                                      moe_bf16_t* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Combine: out_t = bf16(sum_j y[inv_perm[t*k+j]]) over kept slots, summed in
+ * fp32 in slot order j = 0..k-1; a token with every slot dropped gets 0.
+ *   y        [T*k, d] bf16   in (moe_experts_fwd)
+ *   inv_perm [T*k]    int32  in (moe_dispatch)
+ *   out      [T, d]   bf16   out */
+MOE_API moe_status_t moe_combine(const moe_config_t* cfg, const moe_bf16_t* y, const int32_t* inv_perm,
+                         moe_bf16_t* out, void* stream);
+
+/* The whole layer: route -> dispatch -> experts -> combine, on one stream,
+ * with no host synchronisation (the kept counts never leave the device).
+ *   out [T, d] bf16 out.  expert_idx/gate/r/counts: optional copies of the
+ *   routing results (NULL to skip), shapes as in moe_route / moe_dispatch. */
+MOE_API moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
+                           const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
+                           const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out,
+                           int32_t* expert_idx, float* gate, float* r, int32_t* counts, void* ws,
+                           size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -62,6 +62,14 @@ def widen_bf16(bits: np.ndarray) -> np.ndarray:
     return b.view(np.float32).astype(np.float64)
 
 
+def as_f64(a: np.ndarray) -> np.ndarray:
+    """Values of ``a`` as float64: bf16 bit patterns (uint16) are widened
+    exactly; float arrays (weights widened once by the caller) pass through."""
+    if a.dtype == np.uint16:
+        return widen_bf16(a)
+    return np.asarray(a, dtype=np.float64)
+
+
 # --------------------------------------------------------------------------
 # variable-width experts (nanoMOE variable-size-experts notes)
 # --------------------------------------------------------------------------
@@ -251,7 +259,8 @@ def experts_forward(x_bits: np.ndarray, gamma_bits: np.ndarray, r: np.ndarray,
 
     If ``tokens`` is given, only those tokens' assignments are computed (rows
     of the other tokens stay 0); ``x_bits`` then holds just those tokens' rows
-    in the same order.  Expert weight slices are widened one expert at a time.
+    in the same order.  Expert weight slices are widened one expert at a time
+    (or used as given when the caller passes them already as float64).
     """
     idx = np.asarray(idx, dtype=np.int64)
     T, k = idx.shape
@@ -276,9 +285,9 @@ def experts_forward(x_bits: np.ndarray, gamma_bits: np.ndarray, r: np.ndarray,
         rows = row_all[m]
         t_of = sel_a // k
         o0, o1 = int(offs[e]), int(offs[e + 1])
-        W1e = widen_bf16(W1_bits[:, o0:o1])
-        W3e = widen_bf16(W3_bits[:, o0:o1])
-        W2e = widen_bf16(W2_bits[o0:o1, :])
+        W1e = as_f64(W1_bits[:, o0:o1])
+        W3e = as_f64(W3_bits[:, o0:o1])
+        W2e = as_f64(W2_bits[o0:o1, :])
         y[sel_a] = expert_ffn(xg[rows], np.asarray(r, dtype=np.float64)[t_of], W1e, W3e, W2e)
     return y
 

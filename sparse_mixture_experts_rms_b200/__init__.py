@@ -1,0 +1,355 @@
+"""Python binding of ``libmoe_b200.so``: the B200 sparse MoE FFN layer forward.
+
+The functions here have the names of the C ABI in ``include/moe.h`` and only
+marshal arguments: they check torch tensors (device, dtype, shape,
+contiguity), pass raw pointers and the current CUDA stream, and raise
+``MoEError`` on a non-OK status.  Every step of the layer runs in the
+library's sm_100a kernels; there is no fallback path.  If the library has not
+been built, importing works but every call raises.
+
+Layer (forward only): RMS statistic -> router GEMM with the statistic applied
+before the top-k (CODA) -> softmax/top-k gating -> dispatch (histogram,
+capacity, expert-centric permutation) -> grouped SwiGLU expert GEMMs with
+variable widths, r applied after GEMM 1, gate after GEMM 2 -> combine.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_ALIGNMENT = 2
+MOE_ERR_WORKSPACE = 3
+MOE_ERR_UNSUPPORTED = 4
+MOE_ERR_CUDA = 5
+MOE_ERR_DEVICE = 6
+MOE_ERR_NO_DEVICE = 7
+
+MOE_DEVERR_EXPERT_ID = 0x1
+MOE_DEVERR_TIMEOUT = 0x2
+MOE_DEVERR_TILE_TABLE = 0x4
+
+EXPORTED = ["moe_status_string", "moe_capacity", "moe_max_kept", "moe_workspace_size",
+            "moe_workspace_init", "moe_get_device_error", "moe_route", "moe_dispatch",
+            "moe_experts_fwd", "moe_experts_up", "moe_experts_down", "moe_combine",
+            "moe_layer_fwd"]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str = "", code: int = 0):
+        self.status = status
+        self.code = code
+        msg = _status_text(status)
+        if what:
+            msg = f"{what}: {msg}"
+        if code:
+            msg += f" (device error word 0x{code:x})"
+        super().__init__(msg)
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d_model", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("ffn_offsets", ctypes.POINTER(ctypes.c_int32)),
+                ("capacity_factor", ctypes.c_float), ("eps", ctypes.c_float),
+                ("renormalize", ctypes.c_int32)]
+
+
+_lib_handle = None
+
+
+def library_available() -> bool:
+    return os.path.exists(LIB_PATH)
+
+
+def _lib():
+    global _lib_handle
+    if _lib_handle is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m sparse_mixture_experts_rms_b200.build` "
+                "(nvcc, sm_100a). There is no non-CUDA path.")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        cfgp = ctypes.POINTER(_Config)
+        lib.moe_status_string.restype = ctypes.c_char_p
+        lib.moe_status_string.argtypes = [ctypes.c_int]
+        lib.moe_capacity.restype = ctypes.c_int64
+        lib.moe_capacity.argtypes = [cfgp]
+        lib.moe_max_kept.restype = ctypes.c_int64
+        lib.moe_max_kept.argtypes = [cfgp]
+        lib.moe_workspace_size.restype = SZ
+        lib.moe_workspace_size.argtypes = [cfgp]
+        lib.moe_workspace_init.restype = ctypes.c_int
+        lib.moe_workspace_init.argtypes = [P, SZ, P]
+        lib.moe_get_device_error.restype = ctypes.c_int
+        lib.moe_get_device_error.argtypes = [P, SZ, P, ctypes.POINTER(ctypes.c_uint32)]
+        lib.moe_route.restype = ctypes.c_int
+        lib.moe_route.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_dispatch.restype = ctypes.c_int
+        lib.moe_dispatch.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_experts_fwd.restype = ctypes.c_int
+        lib.moe_experts_fwd.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_experts_up.restype = ctypes.c_int
+        lib.moe_experts_up.argtypes = [cfgp, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_experts_down.restype = ctypes.c_int
+        lib.moe_experts_down.argtypes = [cfgp, P, P, P, P, P, P, SZ, P]
+        lib.moe_combine.restype = ctypes.c_int
+        lib.moe_combine.argtypes = [cfgp, P, P, P, P]
+        lib.moe_layer_fwd.restype = ctypes.c_int
+        lib.moe_layer_fwd.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        _lib_handle = lib
+    return _lib_handle
+
+
+def _status_text(status: int) -> str:
+    try:
+        return _lib().moe_status_string(int(status)).decode()
+    except Exception:  # library missing: still describe the code
+        return f"status {status}"
+
+
+def ffn_offsets_from_sizes(expert_sizes: Sequence[Tuple[int, int]], block: int = 128) -> List[int]:
+    """Cumulative expert column offsets [E+1] from ``[(count, size), ...]``.
+
+    Each size is rounded up to a multiple of ``block`` and repeated ``count``
+    times; offsets are running sums of the widths (nanoMOE variable-size
+    experts notes, "Expert Size Computation" / "Offset Calculation").
+    """
+    offs = [0]
+    for count, size in expert_sizes:
+        w = -(-int(size) // block) * block
+        for _ in range(int(count)):
+            offs.append(offs[-1] + w)
+    return offs
+
+
+@dataclass
+class MoEConfig:
+    """Layer configuration (mirrors ``moe_config_t``)."""
+
+    T: int
+    d_model: int
+    E: int
+    k: int
+    ffn_offsets: List[int]
+    capacity_factor: float = 0.0
+    eps: float = 1e-5
+    renormalize: bool = False
+    _c: Optional[_Config] = field(default=None, repr=False, compare=False)
+    _offs: Optional[ctypes.Array] = field(default=None, repr=False, compare=False)
+
+    def c(self) -> _Config:
+        self._offs = (ctypes.c_int32 * len(self.ffn_offsets))(*[int(v) for v in self.ffn_offsets])
+        self._c = _Config(int(self.T), int(self.d_model), int(self.E), int(self.k),
+                          ctypes.cast(self._offs, ctypes.POINTER(ctypes.c_int32)),
+                          float(self.capacity_factor), float(self.eps), int(bool(self.renormalize)))
+        return self._c
+
+    @property
+    def F(self) -> int:
+        return int(self.ffn_offsets[-1])
+
+
+def _ptr(t: Optional[torch.Tensor], name: str, dtype=None, shape=None) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(0)
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(int(s.cuda_stream))
+
+
+def _check(status: int, what: str):
+    if status != MOE_OK:
+        raise MoEError(status, what)
+
+
+# ------------------------------------------------------------------ C ABI
+def moe_status_string(status: int) -> str:
+    return _lib().moe_status_string(int(status)).decode()
+
+
+def moe_capacity(cfg: MoEConfig) -> int:
+    return int(_lib().moe_capacity(ctypes.byref(cfg.c())))
+
+
+def moe_max_kept(cfg: MoEConfig) -> int:
+    return int(_lib().moe_max_kept(ctypes.byref(cfg.c())))
+
+
+def moe_workspace_size(cfg: MoEConfig) -> int:
+    return int(_lib().moe_workspace_size(ctypes.byref(cfg.c())))
+
+
+def alloc_workspace(cfg: MoEConfig, device=None, stream=None) -> torch.Tensor:
+    """A zero-initialised workspace of ``moe_workspace_size(cfg)`` bytes (torch-owned)."""
+    n = moe_workspace_size(cfg)
+    if n == 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    moe_workspace_init(ws, stream)
+    return ws
+
+
+def moe_workspace_init(ws: torch.Tensor, stream=None) -> None:
+    _check(_lib().moe_workspace_init(_ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)),
+           "moe_workspace_init")
+
+
+def moe_get_device_error(ws: torch.Tensor, stream=None, raise_on_error: bool = True) -> int:
+    code = ctypes.c_uint32(0)
+    st = _lib().moe_get_device_error(_ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream),
+                                     ctypes.byref(code))
+    if st == MOE_ERR_DEVICE:
+        if raise_on_error:
+            raise MoEError(st, "moe_get_device_error", int(code.value))
+        return int(code.value)
+    _check(st, "moe_get_device_error")
+    return int(code.value)
+
+
+def moe_route(cfg: MoEConfig, x, gamma, Wr, bias, expert_idx, gate, r, logits=None,
+              ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    T, d, E, k = cfg.T, cfg.d_model, cfg.E, cfg.k
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    st = _lib().moe_route(
+        ctypes.byref(cfg.c()), _ptr(x, "x", bf, (T, d)), _ptr(gamma, "gamma", bf, (d,)),
+        _ptr(Wr, "Wr", bf, (d, E)), _ptr(bias, "bias", f32, (E,)),
+        _ptr(expert_idx, "expert_idx", i32, (T, k)), _ptr(gate, "gate", f32, (T, k)),
+        _ptr(r, "r", f32, (T,)), _ptr(logits, "logits", f32, (T, E)),
+        _ptr(ws, "ws", torch.uint8), 0 if ws is None else ws.numel(), _stream(stream))
+    _check(st, "moe_route")
+
+
+def moe_dispatch(cfg: MoEConfig, expert_idx, x, gamma, counts, expert_offsets, perm, inv_perm,
+                 x_perm, ws: torch.Tensor, stream=None) -> None:
+    T, d, E, k = cfg.T, cfg.d_model, cfg.E, cfg.k
+    i32, bf = torch.int32, torch.bfloat16
+    if x_perm is not None and (x_perm.dim() != 2 or x_perm.shape[1] != d
+                               or x_perm.shape[0] < moe_max_kept(cfg)):
+        raise ValueError("x_perm must be [>= moe_max_kept(cfg), d]")
+    if perm is not None and perm.numel() < moe_max_kept(cfg):
+        raise ValueError("perm must hold >= moe_max_kept(cfg) entries")
+    st = _lib().moe_dispatch(
+        ctypes.byref(cfg.c()), _ptr(expert_idx, "expert_idx", i32, (T, k)), _ptr(x, "x", bf, (T, d)),
+        _ptr(gamma, "gamma", bf, (d,)), _ptr(counts, "counts", i32, (E,)),
+        _ptr(expert_offsets, "expert_offsets", i32, (E + 1,)), _ptr(perm, "perm", i32),
+        _ptr(inv_perm, "inv_perm", i32, (T * k,)), _ptr(x_perm, "x_perm", bf),
+        _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
+    _check(st, "moe_dispatch")
+
+
+def moe_experts_fwd(cfg: MoEConfig, x_perm, r, gate, perm, expert_offsets, W1, W3, W2, y,
+                    ws: torch.Tensor, stream=None) -> None:
+    T, d, E, k, F = cfg.T, cfg.d_model, cfg.E, cfg.k, cfg.F
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    mk = moe_max_kept(cfg)
+    for name, t in (("x_perm", x_perm), ("y", y)):
+        if t.dim() != 2 or t.shape[1] != d or t.shape[0] < mk:
+            raise ValueError(f"{name} must be [>= moe_max_kept(cfg), d]")
+    if perm.numel() < mk:
+        raise ValueError("perm must hold >= moe_max_kept(cfg) entries")
+    st = _lib().moe_experts_fwd(
+        ctypes.byref(cfg.c()), _ptr(x_perm, "x_perm", bf), _ptr(r, "r", f32, (T,)),
+        _ptr(gate, "gate", f32, (T, k)), _ptr(perm, "perm", i32),
+        _ptr(expert_offsets, "expert_offsets", i32, (E + 1,)), _ptr(W1, "W1", bf, (d, F)),
+        _ptr(W3, "W3", bf, (d, F)), _ptr(W2, "W2", bf, (F, d)), _ptr(y, "y", bf),
+        _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
+    _check(st, "moe_experts_fwd")
+
+
+def moe_experts_up(cfg: MoEConfig, x_perm, r, perm, expert_offsets, W1, W3, ws: torch.Tensor,
+                   stream=None) -> None:
+    T, d, E, F = cfg.T, cfg.d_model, cfg.E, cfg.F
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    mk = moe_max_kept(cfg)
+    if x_perm.dim() != 2 or x_perm.shape[1] != d or x_perm.shape[0] < mk:
+        raise ValueError("x_perm must be [>= moe_max_kept(cfg), d]")
+    if perm.numel() < mk:
+        raise ValueError("perm must hold >= moe_max_kept(cfg) entries")
+    st = _lib().moe_experts_up(
+        ctypes.byref(cfg.c()), _ptr(x_perm, "x_perm", bf), _ptr(r, "r", f32, (T,)),
+        _ptr(perm, "perm", i32), _ptr(expert_offsets, "expert_offsets", i32, (E + 1,)),
+        _ptr(W1, "W1", bf, (d, F)), _ptr(W3, "W3", bf, (d, F)),
+        _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
+    _check(st, "moe_experts_up")
+
+
+def moe_experts_down(cfg: MoEConfig, gate, perm, expert_offsets, W2, y, ws: torch.Tensor,
+                     stream=None) -> None:
+    T, d, E, k, F = cfg.T, cfg.d_model, cfg.E, cfg.k, cfg.F
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    mk = moe_max_kept(cfg)
+    if y.dim() != 2 or y.shape[1] != d or y.shape[0] < mk:
+        raise ValueError("y must be [>= moe_max_kept(cfg), d]")
+    if perm.numel() < mk:
+        raise ValueError("perm must hold >= moe_max_kept(cfg) entries")
+    st = _lib().moe_experts_down(
+        ctypes.byref(cfg.c()), _ptr(gate, "gate", f32, (T, k)), _ptr(perm, "perm", i32),
+        _ptr(expert_offsets, "expert_offsets", i32, (E + 1,)), _ptr(W2, "W2", bf, (F, d)),
+        _ptr(y, "y", bf), _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
+    _check(st, "moe_experts_down")
+
+
+def moe_combine(cfg: MoEConfig, y, inv_perm, out, stream=None) -> None:
+    T, d, k = cfg.T, cfg.d_model, cfg.k
+    if y.dim() != 2 or y.shape[1] != d:
+        raise ValueError("y must be [rows, d]")
+    st = _lib().moe_combine(ctypes.byref(cfg.c()), _ptr(y, "y", torch.bfloat16),
+                            _ptr(inv_perm, "inv_perm", torch.int32, (T * k,)),
+                            _ptr(out, "out", torch.bfloat16, (T, d)), _stream(stream))
+    _check(st, "moe_combine")
+
+
+def moe_layer_fwd(cfg: MoEConfig, x, gamma, Wr, bias, W1, W3, W2, out, ws: torch.Tensor,
+                  expert_idx=None, gate=None, r=None, counts=None, stream=None) -> None:
+    T, d, E, k, F = cfg.T, cfg.d_model, cfg.E, cfg.k, cfg.F
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    st = _lib().moe_layer_fwd(
+        ctypes.byref(cfg.c()), _ptr(x, "x", bf, (T, d)), _ptr(gamma, "gamma", bf, (d,)),
+        _ptr(Wr, "Wr", bf, (d, E)), _ptr(bias, "bias", f32, (E,)), _ptr(W1, "W1", bf, (d, F)),
+        _ptr(W3, "W3", bf, (d, F)), _ptr(W2, "W2", bf, (F, d)), _ptr(out, "out", bf, (T, d)),
+        _ptr(expert_idx, "expert_idx", i32, (T, k)), _ptr(gate, "gate", f32, (T, k)),
+        _ptr(r, "r", f32, (T,)), _ptr(counts, "counts", i32, (E,)),
+        _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
+    _check(st, "moe_layer_fwd")
+
+
+class MoELayer:
+    """Holds a layer's weights and workspace; ``forward(x)`` calls moe_layer_fwd."""
+
+    def __init__(self, cfg: MoEConfig, gamma, Wr, bias, W1, W3, W2):
+        self.cfg = cfg
+        self.gamma, self.Wr, self.bias = gamma, Wr, bias
+        self.W1, self.W3, self.W2 = W1, W3, W2
+        self.ws = alloc_workspace(cfg, device=gamma.device)
+
+    def forward(self, x, out=None, expert_idx=None, gate=None, r=None, counts=None, stream=None):
+        c = self.cfg
+        if out is None:
+            out = torch.empty((c.T, c.d_model), dtype=torch.bfloat16, device=x.device)
+        moe_layer_fwd(c, x, self.gamma, self.Wr, self.bias, self.W1, self.W3, self.W2, out, self.ws,
+                      expert_idx=expert_idx, gate=gate, r=r, counts=counts, stream=stream)
+        return out
+
+    __call__ = forward

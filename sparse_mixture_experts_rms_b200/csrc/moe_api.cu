@@ -1,0 +1,533 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: argument validation,
+// workspace layout, TMA descriptor encoding and launch sequencing on one
+// stream.  Allocates nothing; never synchronises except in
+// moe_get_device_error.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kHeaderBytes = 256;
+
+struct DeviceState {
+  bool ready = false;
+  bool ok = false;
+  int sms = 0;
+};
+
+std::mutex g_mutex;
+DeviceState g_dev[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+bool g_encode_tried = false;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Layout {
+  size_t err, tile_counts, r, idx, gate, counts, offsets, perm, inv_perm, x_perm, H, y, total;
+  int64_t max_kept;
+  int ldh;
+};
+
+int64_t capacity_of(const moe_config_t& c) {
+  if (!(c.capacity_factor > 0.0f)) return -1;
+  const double v = static_cast<double>(c.T) * c.k / c.E * static_cast<double>(c.capacity_factor);
+  const double tk = static_cast<double>(c.T) * c.k;
+  return static_cast<int64_t>(std::floor(v < tk ? v : tk));
+}
+
+int64_t max_kept_of(const moe_config_t& c) {
+  const int64_t tk = static_cast<int64_t>(c.T) * c.k;
+  const int64_t cap = capacity_of(c);
+  if (cap < 0) return tk;
+  const int64_t ec = cap * c.E;
+  return ec < tk ? ec : tk;
+}
+
+moe_status_t validate(const moe_config_t* c) {
+  if (c == nullptr) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->d_model <= 0 || c->E <= 0 || c->k <= 0 || c->k > c->E) return MOE_ERR_INVALID_ARG;
+  if (c->d_model % 128 != 0) return MOE_ERR_INVALID_ARG;
+  if (!std::isfinite(c->eps) || c->eps < 0.0f) return MOE_ERR_INVALID_ARG;
+  if (!std::isfinite(c->capacity_factor)) return MOE_ERR_INVALID_ARG;
+  if (c->ffn_offsets == nullptr) return MOE_ERR_INVALID_ARG;
+  if (c->E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(c->T) * c->k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  if (c->ffn_offsets[0] != 0) return MOE_ERR_INVALID_ARG;
+  for (int e = 0; e < c->E; ++e) {
+    const int64_t w = static_cast<int64_t>(c->ffn_offsets[e + 1]) - c->ffn_offsets[e];
+    if (w <= 0 || w % kBlockN != 0) return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+Layout layout_of(const moe_config_t& c) {
+  Layout L{};
+  size_t off = kHeaderBytes;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes > 0 ? bytes : 1, 1024);
+    return o;
+  };
+  const size_t tk = static_cast<size_t>(c.T) * c.k;
+  const size_t ntiles = (tk + kDispatchTile - 1) / kDispatchTile;
+  int fmax = 0;
+  for (int e = 0; e < c.E; ++e) {
+    const int w = c.ffn_offsets[e + 1] - c.ffn_offsets[e];
+    fmax = w > fmax ? w : fmax;
+  }
+  L.max_kept = max_kept_of(c);
+  L.ldh = fmax;
+  const size_t mk = static_cast<size_t>(L.max_kept);
+  L.err = 0;
+  L.tile_counts = take(ntiles * c.E * 4);
+  L.r = take(static_cast<size_t>(c.T) * 4);
+  L.idx = take(tk * 4);
+  L.gate = take(tk * 4);
+  L.counts = take(static_cast<size_t>(c.E) * 4);
+  L.offsets = take(static_cast<size_t>(c.E + 1) * 4);
+  L.perm = take(mk * 4);
+  L.inv_perm = take(tk * 4);
+  L.x_perm = take(mk * c.d_model * 2);
+  L.H = take(mk * static_cast<size_t>(fmax) * 2);
+  L.y = take(mk * c.d_model * 2);
+  L.total = off;
+  return L;
+}
+
+moe_status_t check_ws(const moe_config_t& c, void* ws, size_t ws_bytes, Layout* L) {
+  *L = layout_of(c);
+  if (ws == nullptr || ws_bytes < L->total) return MOE_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+moe_status_t device_ready(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    st.ready = true;
+    st.ok = false;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_NO_DEVICE;
+    }
+    if (prop.major != 10) return MOE_ERR_NO_DEVICE;
+    if (prepare_grouped_gemm() != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    if (!g_encode_tried) {
+      g_encode_tried = true;
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+              cudaSuccess &&
+          q == cudaDriverEntryPointSuccess)
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+      cudaGetLastError();
+    }
+    if (g_encode == nullptr) return MOE_ERR_CUDA;
+    st.sms = prop.multiProcessorCount;
+    st.ok = true;
+  }
+  if (!st.ok) return MOE_ERR_NO_DEVICE;
+  *sms = st.sms;
+  return MOE_OK;
+}
+
+// 2-D bf16 tensor map with 128-byte swizzle: `inner` contiguous elements per
+// row, `outer` rows, `row_elems` elements between rows; box inner x outer.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_elems,
+              uint32_t box_inner, uint32_t box_outer) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_elems * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+moe_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  cudaGetLastError();
+  return MOE_ERR_CUDA;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf16_t* gamma,
+                       const moe_bf16_t* Wr, const float* bias, int32_t* idx, float* gate, float* r,
+                       float* logits, cudaStream_t s) {
+  RouteArgs a{};
+  a.x = reinterpret_cast<const __nv_bfloat16*>(x);
+  a.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
+  a.Wr = reinterpret_cast<const __nv_bfloat16*>(Wr);
+  a.bias = bias;
+  a.idx = idx;
+  a.gate = gate;
+  a.r = r;
+  a.logits = logits;
+  a.T = c.T;
+  a.d = c.d_model;
+  a.E = c.E;
+  a.k = c.k;
+  a.eps = c.eps;
+  a.renormalize = c.renormalize ? 1 : 0;
+  return cuda_status(launch_route(a, s));
+}
+
+moe_status_t run_dispatch(const moe_config_t& c, const Layout& L, void* ws, const int32_t* idx,
+                          const moe_bf16_t* x, const moe_bf16_t* gamma, int32_t* counts,
+                          int32_t* offsets, int32_t* perm, int32_t* inv_perm, moe_bf16_t* x_perm,
+                          int sms, cudaStream_t s) {
+  DispatchArgs a{};
+  a.idx = idx;
+  a.x = reinterpret_cast<const __nv_bfloat16*>(x);
+  a.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
+  a.tile_counts = at<int32_t>(ws, L.tile_counts);
+  a.counts = counts;
+  a.offsets = offsets;
+  a.perm = perm;
+  a.inv_perm = inv_perm;
+  a.x_perm = reinterpret_cast<__nv_bfloat16*>(x_perm);
+  a.err = at<uint32_t>(ws, L.err);
+  a.T = c.T;
+  a.d = c.d_model;
+  a.E = c.E;
+  a.k = c.k;
+  const int64_t cap = capacity_of(c);
+  a.capacity = static_cast<int>(cap);
+  a.max_kept = static_cast<int>(L.max_kept);
+  if (c.T == 0) {
+    // nothing routed: offsets and counts are still defined
+    cudaError_t e = cudaMemsetAsync(offsets, 0, (c.E + 1) * sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, c.E * sizeof(int32_t), s);
+    return cuda_status(e);
+  }
+  return cuda_status(launch_dispatch(a, sms, s));
+}
+
+void fill_gemm_common(GemmArgs& g, const moe_config_t& c, const Layout& L, void* ws,
+                      const int32_t* perm, const int32_t* offsets) {
+  g.E = c.E;
+  g.k = c.k;
+  g.d = c.d_model;
+  g.rows = static_cast<int>(L.max_kept);
+  g.offsets = offsets;
+  g.perm = perm;
+  g.err = at<uint32_t>(ws, L.err);
+  for (int e = 0; e <= c.E; ++e) g.ffn.off[e] = c.ffn_offsets[e];
+}
+
+// GEMM 1: x_perm [rows, d] x (W1 | W3) [d, F] -> SwiGLU -> H [rows, ldh] (workspace)
+moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x_perm,
+                    const float* r, const int32_t* perm, const int32_t* offsets,
+                    const moe_bf16_t* W1, const moe_bf16_t* W3, int sms, cudaStream_t s) {
+  if (L.max_kept == 0) return MOE_OK;
+  const uint64_t rows = static_cast<uint64_t>(L.max_kept);
+  const uint64_t d = static_cast<uint64_t>(c.d_model);
+  const uint64_t F = static_cast<uint64_t>(c.ffn_offsets[c.E]);
+  GemmArgs g{};
+  fill_gemm_common(g, c, L, ws, perm, offsets);
+  CUtensorMap mA, mB0, mB1;
+  if (!make_map(&mA, x_perm, d, rows, d, 64, 128) || !make_map(&mB0, W1, F, d, F, 64, 64) ||
+      !make_map(&mB1, W3, F, d, F, 64, 64))
+    return MOE_ERR_CUDA;
+  g.up = 1;
+  g.bn = 2 * kBlockN;
+  g.scale = r;
+  g.out = at<__nv_bfloat16>(ws, L.H);
+  g.ld_out = L.ldh;
+  return cuda_status(launch_grouped_gemm(g, mA, mB0, mB1, sms, s));
+}
+
+// GEMM 2: H [rows, f_e] (workspace) x W2 [F, d] -> y [rows, d], gate in the epilogue
+moe_status_t run_down(const moe_config_t& c, const Layout& L, void* ws, const float* gate,
+                      const int32_t* perm, const int32_t* offsets, const moe_bf16_t* W2,
+                      moe_bf16_t* y, int sms, cudaStream_t s) {
+  if (L.max_kept == 0) return MOE_OK;
+  const uint64_t rows = static_cast<uint64_t>(L.max_kept);
+  const uint64_t d = static_cast<uint64_t>(c.d_model);
+  const uint64_t F = static_cast<uint64_t>(c.ffn_offsets[c.E]);
+  GemmArgs g{};
+  fill_gemm_common(g, c, L, ws, perm, offsets);
+  CUtensorMap mA, mB;
+  if (!make_map(&mA, at<void>(ws, L.H), static_cast<uint64_t>(L.ldh), rows,
+                static_cast<uint64_t>(L.ldh), 64, 128) ||
+      !make_map(&mB, W2, d, F, d, 64, 64))
+    return MOE_ERR_CUDA;
+  g.up = 0;
+  g.bn = (c.d_model % 256 == 0) ? 256 : 128;
+  g.scale = gate;
+  g.out = reinterpret_cast<__nv_bfloat16*>(y);
+  g.ld_out = c.d_model;
+  return cuda_status(launch_grouped_gemm(g, mA, mB, mB, sms, s));
+}
+
+moe_status_t run_experts(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x_perm,
+                         const float* r, const float* gate, const int32_t* perm,
+                         const int32_t* offsets, const moe_bf16_t* W1, const moe_bf16_t* W3,
+                         const moe_bf16_t* W2, moe_bf16_t* y, int sms, cudaStream_t s) {
+  moe_status_t st = run_up(c, L, ws, x_perm, r, perm, offsets, W1, W3, sms, s);
+  if (st != MOE_OK) return st;
+  return run_down(c, L, ws, gate, perm, offsets, W2, y, sms, s);
+}
+
+moe_status_t run_combine(const moe_config_t& c, const moe_bf16_t* y, const int32_t* inv_perm,
+                         moe_bf16_t* out, int sms, cudaStream_t s) {
+  CombineArgs a{};
+  a.y = reinterpret_cast<const __nv_bfloat16*>(y);
+  a.inv_perm = inv_perm;
+  a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.T = c.T;
+  a.d = c.d_model;
+  a.k = c.k;
+  return cuda_status(launch_combine(a, sms, s));
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+    case MOE_ERR_ALIGNMENT: return "MOE_ERR_ALIGNMENT: pointer not aligned as required";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing or too small";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: outside this build's limits";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call failed";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE: the device error word is set";
+    case MOE_ERR_NO_DEVICE: return "MOE_ERR_NO_DEVICE: no usable sm_100 device";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+int64_t moe_capacity(const moe_config_t* cfg) {
+  if (validate(cfg) != MOE_OK) return -1;
+  return capacity_of(*cfg);
+}
+
+int64_t moe_max_kept(const moe_config_t* cfg) {
+  if (validate(cfg) != MOE_OK) return -1;
+  return max_kept_of(*cfg);
+}
+
+size_t moe_workspace_size(const moe_config_t* cfg) {
+  if (validate(cfg) != MOE_OK) return 0;
+  return layout_of(*cfg).total;
+}
+
+moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes < kHeaderBytes) return MOE_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGNMENT;
+  int sms;
+  moe_status_t st = device_ready(&sms);
+  if (st != MOE_OK) return st;
+  return cuda_status(cudaMemsetAsync(ws, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_get_device_error(void* ws, size_t ws_bytes, void* stream, uint32_t* code) {
+  if (code == nullptr) return MOE_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < kHeaderBytes) return MOE_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGNMENT;
+  int sms;
+  moe_status_t st = device_ready(&sms);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(v), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e);
+  *code = v;
+  return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+moe_status_t moe_route(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
+                       const moe_bf16_t* Wr, const float* bias, int32_t* expert_idx, float* gate,
+                       float* r, float* logits, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  (void)ws;
+  (void)ws_bytes;
+  if (cfg->T == 0) return MOE_OK;  // no tokens: nothing to do (pointers may be null)
+  if (!x || !gamma || !Wr || !expert_idx || !gate || !r) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) ||
+      !aligned(expert_idx, 4) || !aligned(gate, 4) || !aligned(r, 4) || !aligned(logits, 4))
+    return MOE_ERR_ALIGNMENT;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  return run_route(*cfg, x, gamma, Wr, bias, expert_idx, gate, r, logits,
+                   static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_dispatch(const moe_config_t* cfg, const int32_t* expert_idx, const moe_bf16_t* x,
+                          const moe_bf16_t* gamma, int32_t* counts, int32_t* expert_offsets,
+                          int32_t* perm, int32_t* inv_perm, moe_bf16_t* x_perm, void* ws,
+                          size_t ws_bytes, void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) {  // no tokens: counts and offsets are zero, nothing else is touched
+    if (!counts || !expert_offsets) return MOE_ERR_INVALID_ARG;
+    if (!aligned(counts, 4) || !aligned(expert_offsets, 4)) return MOE_ERR_ALIGNMENT;
+    int sms;
+    if ((st = device_ready(&sms)) != MOE_OK) return st;
+    cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(expert_offsets, 0, (cfg->E + 1) * sizeof(int32_t), s0);
+    if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, cfg->E * sizeof(int32_t), s0);
+    return cuda_status(e);
+  }
+  if (!expert_idx || !x || !gamma || !counts || !expert_offsets || !perm || !inv_perm || !x_perm)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(expert_idx, 4) || !aligned(counts, 4) || !aligned(expert_offsets, 4) ||
+      !aligned(perm, 4) || !aligned(inv_perm, 4) || !aligned(x, 16) || !aligned(gamma, 16) ||
+      !aligned(x_perm, 16))
+    return MOE_ERR_ALIGNMENT;
+  Layout L;
+  if ((st = check_ws(*cfg, ws, ws_bytes, &L)) != MOE_OK) return st;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  return run_dispatch(*cfg, L, ws, expert_idx, x, gamma, counts, expert_offsets, perm, inv_perm,
+                      x_perm, sms, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_experts_fwd(const moe_config_t* cfg, const moe_bf16_t* x_perm, const float* r,
+                             const float* gate, const int32_t* perm,
+                             const int32_t* expert_offsets, const moe_bf16_t* W1,
+                             const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* y, void* ws,
+                             size_t ws_bytes, void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x_perm || !r || !gate || !perm || !expert_offsets || !W1 || !W3 || !W2 || !y)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x_perm, 16) || !aligned(W1, 16) || !aligned(W3, 16) || !aligned(W2, 16) ||
+      !aligned(y, 16) || !aligned(r, 4) || !aligned(gate, 4) || !aligned(perm, 4) ||
+      !aligned(expert_offsets, 4))
+    return MOE_ERR_ALIGNMENT;
+  Layout L;
+  if ((st = check_ws(*cfg, ws, ws_bytes, &L)) != MOE_OK) return st;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  return run_experts(*cfg, L, ws, x_perm, r, gate, perm, expert_offsets, W1, W3, W2, y, sms,
+                     static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_experts_up(const moe_config_t* cfg, const moe_bf16_t* x_perm, const float* r,
+                            const int32_t* perm, const int32_t* expert_offsets, const moe_bf16_t* W1,
+                            const moe_bf16_t* W3, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x_perm || !r || !perm || !expert_offsets || !W1 || !W3) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x_perm, 16) || !aligned(W1, 16) || !aligned(W3, 16) || !aligned(r, 4) ||
+      !aligned(perm, 4) || !aligned(expert_offsets, 4))
+    return MOE_ERR_ALIGNMENT;
+  Layout L;
+  if ((st = check_ws(*cfg, ws, ws_bytes, &L)) != MOE_OK) return st;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  return run_up(*cfg, L, ws, x_perm, r, perm, expert_offsets, W1, W3, sms,
+                static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_experts_down(const moe_config_t* cfg, const float* gate, const int32_t* perm,
+                              const int32_t* expert_offsets, const moe_bf16_t* W2, moe_bf16_t* y,
+                              void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!gate || !perm || !expert_offsets || !W2 || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned(W2, 16) || !aligned(y, 16) || !aligned(gate, 4) || !aligned(perm, 4) ||
+      !aligned(expert_offsets, 4))
+    return MOE_ERR_ALIGNMENT;
+  Layout L;
+  if ((st = check_ws(*cfg, ws, ws_bytes, &L)) != MOE_OK) return st;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  return run_down(*cfg, L, ws, gate, perm, expert_offsets, W2, y, sms,
+                  static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_combine(const moe_config_t* cfg, const moe_bf16_t* y, const int32_t* inv_perm,
+                         moe_bf16_t* out, void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!y || !inv_perm || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned(y, 16) || !aligned(out, 16) || !aligned(inv_perm, 4)) return MOE_ERR_ALIGNMENT;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  return run_combine(*cfg, y, inv_perm, out, sms, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
+                           const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
+                           const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out,
+                           int32_t* expert_idx, float* gate, float* r, int32_t* counts, void* ws,
+                           size_t ws_bytes, void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) {  // no tokens: only the optional counts are written (zeros)
+    if (counts == nullptr) return MOE_OK;
+    if (!aligned(counts, 4)) return MOE_ERR_ALIGNMENT;
+    int sms;
+    if ((st = device_ready(&sms)) != MOE_OK) return st;
+    return cuda_status(cudaMemsetAsync(counts, 0, cfg->E * sizeof(int32_t), static_cast<cudaStream_t>(stream)));
+  }
+  if (!x || !gamma || !Wr || !W1 || !W3 || !W2 || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) ||
+      !aligned(W1, 16) || !aligned(W3, 16) || !aligned(W2, 16) || !aligned(out, 16) ||
+      !aligned(expert_idx, 4) || !aligned(gate, 4) || !aligned(r, 4) || !aligned(counts, 4))
+    return MOE_ERR_ALIGNMENT;
+  Layout L;
+  if ((st = check_ws(*cfg, ws, ws_bytes, &L)) != MOE_OK) return st;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const moe_config_t& c = *cfg;
+  int32_t* idx_ = expert_idx ? expert_idx : at<int32_t>(ws, L.idx);
+  float* gate_ = gate ? gate : at<float>(ws, L.gate);
+  float* r_ = r ? r : at<float>(ws, L.r);
+  int32_t* counts_ = counts ? counts : at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+  moe_bf16_t* x_perm = at<moe_bf16_t>(ws, L.x_perm);
+  moe_bf16_t* y = at<moe_bf16_t>(ws, L.y);
+  if ((st = run_route(c, x, gamma, Wr, bias, idx_, gate_, r_, nullptr, s)) != MOE_OK) return st;
+  if ((st = run_dispatch(c, L, ws, idx_, x, gamma, counts_, offsets, perm, inv_perm, x_perm, sms, s)) != MOE_OK)
+    return st;
+  if ((st = run_experts(c, L, ws, x_perm, r_, gate_, perm, offsets, W1, W3, W2, y, sms, s)) != MOE_OK)
+    return st;
+  return run_combine(c, y, inv_perm, out, sms, s);
+}
+
+}  // extern "C"

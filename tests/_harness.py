@@ -1,0 +1,173 @@
+"""Helpers for the GPU parity tests: seeded inputs on the device, calls through
+the C ABI (staged or fused), and the comparisons against the CPU oracle."""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+import moe_workloads as mw
+import sparse_mixture_experts_rms_b200 as moe
+from oracle import moe_oracle as O
+
+# tolerances
+GATE_ATOL = 1e-5          # gates: absolute
+LOGIT_ATOL = 1e-5         # router logits: absolute (also the near-tie margin)
+TIE_MARGIN = 1e-5         # k-th vs (k+1)-th oracle fp32 logit
+ROW_REL = 2e-2            # per-token normwise relative error of the layer output
+MEAN_ABS = 1e-3           # mean absolute error of the layer output
+# The 1e-3 mean-absolute bound is stated for the five reference workloads,
+# whose outputs have mean magnitude 0.05-0.21.  bf16 quantisation error
+# (inputs x*gamma and H of the tensor-core GEMMs, stored outputs) grows in
+# proportion to the magnitude, so cases with larger outputs (k = E mixtures)
+# get the bound scaled by mean|out| / MAG_REF when that exceeds 1.
+MAG_REF = 0.25
+R_RTOL = 2e-6             # RMS statistic, relative
+
+
+def bits_to_dev(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def dev_to_bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def bf16_dev_to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+@dataclass
+class Problem:
+    w: mw.Workload
+    widths: list
+    x: np.ndarray
+    gamma: np.ndarray
+    Wr: np.ndarray
+    bias: Optional[np.ndarray]
+    W1: np.ndarray
+    W3: np.ndarray
+    W2: np.ndarray
+
+    @property
+    def cf32(self) -> float:
+        return float(np.float32(self.w.capacity_factor))
+
+
+def make_problem(w: mw.Workload) -> Problem:
+    widths = O.expert_widths(w.expert_sizes)
+    W1, W3, W2 = mw.gen_expert_weights(w, widths)
+    return Problem(w, widths, mw.gen_x(w), mw.gen_gamma(w), mw.gen_router_weight(w),
+                   mw.gen_router_bias(w), W1, W3, W2)
+
+
+def make_cfg(p: Problem, renormalize: bool = False) -> moe.MoEConfig:
+    w = p.w
+    return moe.MoEConfig(T=w.T, d_model=w.d_model, E=w.E, k=w.k,
+                         ffn_offsets=moe.ffn_offsets_from_sizes(w.expert_sizes),
+                         capacity_factor=w.capacity_factor, eps=w.eps, renormalize=renormalize)
+
+
+class Dev:
+    """The problem's tensors on the device plus a workspace."""
+
+    def __init__(self, p: Problem, cfg: moe.MoEConfig):
+        self.p, self.cfg = p, cfg
+        self.x = bits_to_dev(p.x)
+        self.gamma = bits_to_dev(p.gamma)
+        self.Wr = bits_to_dev(p.Wr)
+        self.bias = None if p.bias is None else torch.from_numpy(p.bias).cuda()
+        self.W1 = bits_to_dev(p.W1)
+        self.W3 = bits_to_dev(p.W3)
+        self.W2 = bits_to_dev(p.W2)
+        self.ws = moe.alloc_workspace(cfg)
+
+
+def run_staged(d: Dev) -> Dict[str, torch.Tensor]:
+    c = d.cfg
+    T, dm, E, k = c.T, c.d_model, c.E, c.k
+    mk = max(moe.moe_max_kept(c), 1)
+    o = {
+        "idx": torch.empty((T, k), dtype=torch.int32, device="cuda"),
+        "gate": torch.empty((T, k), dtype=torch.float32, device="cuda"),
+        "r": torch.empty((T,), dtype=torch.float32, device="cuda"),
+        "logits": torch.empty((T, E), dtype=torch.float32, device="cuda"),
+        "counts": torch.empty((E,), dtype=torch.int32, device="cuda"),
+        "offsets": torch.empty((E + 1,), dtype=torch.int32, device="cuda"),
+        "perm": torch.full((mk,), -7, dtype=torch.int32, device="cuda"),
+        "inv_perm": torch.empty((T * k,), dtype=torch.int32, device="cuda"),
+        "x_perm": torch.zeros((mk, dm), dtype=torch.bfloat16, device="cuda"),
+        "y": torch.zeros((mk, dm), dtype=torch.bfloat16, device="cuda"),
+        "out": torch.empty((T, dm), dtype=torch.bfloat16, device="cuda"),
+    }
+    moe.moe_route(c, d.x, d.gamma, d.Wr, d.bias, o["idx"], o["gate"], o["r"], o["logits"], d.ws)
+    moe.moe_dispatch(c, o["idx"], d.x, d.gamma, o["counts"], o["offsets"], o["perm"], o["inv_perm"],
+                     o["x_perm"], d.ws)
+    moe.moe_experts_fwd(c, o["x_perm"], o["r"], o["gate"], o["perm"], o["offsets"], d.W1, d.W3, d.W2,
+                        o["y"], d.ws)
+    moe.moe_combine(c, o["y"], o["inv_perm"], o["out"])
+    torch.cuda.synchronize()
+    return o
+
+
+def run_fused(d: Dev) -> Dict[str, torch.Tensor]:
+    c = d.cfg
+    o = {
+        "idx": torch.empty((c.T, c.k), dtype=torch.int32, device="cuda"),
+        "gate": torch.empty((c.T, c.k), dtype=torch.float32, device="cuda"),
+        "r": torch.empty((c.T,), dtype=torch.float32, device="cuda"),
+        "counts": torch.empty((c.E,), dtype=torch.int32, device="cuda"),
+        "out": torch.empty((c.T, c.d_model), dtype=torch.bfloat16, device="cuda"),
+    }
+    moe.moe_layer_fwd(c, d.x, d.gamma, d.Wr, d.bias, d.W1, d.W3, d.W2, o["out"], d.ws,
+                      expert_idx=o["idx"], gate=o["gate"], r=o["r"], counts=o["counts"])
+    torch.cuda.synchronize()
+    return o
+
+
+def oracle_route(p: Problem, renormalize: bool = False) -> Dict[str, np.ndarray]:
+    x = O.widen_bf16(p.x)
+    return O.route(x, O.widen_bf16(p.gamma), O.widen_bf16(p.Wr), p.bias, p.w.k, p.w.eps, renormalize)
+
+
+def check_route(p: Problem, R: Dict[str, np.ndarray], g_idx, g_gate, g_r, g_logits=None):
+    """idx bit-exact outside near ties; gates, r, logits within tolerance."""
+    k = p.w.k
+    margin = O.topk_margin(R["logits"], k)
+    ok_tok = margin >= TIE_MARGIN
+    np.testing.assert_allclose(g_r, R["r"], rtol=R_RTOL, atol=0)
+    if g_logits is not None:
+        np.testing.assert_allclose(g_logits, R["logits"].astype(np.float64), rtol=0, atol=LOGIT_ATOL)
+    bad = np.nonzero(ok_tok & np.any(g_idx != R["idx"], axis=1))[0]
+    assert bad.size == 0, f"{bad.size} tokens routed differently (margin >= {TIE_MARGIN}): {bad[:10]}"
+    np.testing.assert_allclose(g_gate[ok_tok], R["gate"][ok_tok], rtol=0, atol=GATE_ATOL)
+    return np.nonzero(~ok_tok)[0]
+
+
+def check_dispatch(g_idx: np.ndarray, E: int, C: Optional[int], o: Dict[str, np.ndarray]):
+    """Replay: the oracle's dispatch of the GPU's own routing, bit-exact."""
+    D = O.dispatch(g_idx, E, C)
+    assert np.array_equal(o["counts"], D["counts"])
+    assert np.array_equal(o["offsets"], D["offsets"])
+    n = D["n_kept"]
+    assert np.array_equal(o["perm"][:n], D["perm"])
+    assert np.array_equal(o["inv_perm"], D["inv_perm"])
+    return D
+
+
+def check_rows(g_out: np.ndarray, ref: np.ndarray, what: str = "out"):
+    """Per-row normwise relative error and mean absolute error."""
+    err = g_out - ref
+    nref = np.linalg.norm(ref, axis=1)
+    nerr = np.linalg.norm(err, axis=1)
+    zero = nref == 0
+    assert np.all(nerr[zero] == 0), f"{what}: rows that must be exactly zero are not"
+    rel = nerr[~zero] / nref[~zero]
+    worst = float(rel.max()) if rel.size else 0.0
+    mae = float(np.abs(err).mean()) if err.size else 0.0
+    bound = MEAN_ABS * max(1.0, float(np.abs(ref).mean()) / MAG_REF) if ref.size else MEAN_ABS
+    assert worst <= ROW_REL, f"{what}: max row relative error {worst:.3e} > {ROW_REL}"
+    assert mae <= bound, f"{what}: mean abs error {mae:.3e} > {bound:.3e}"
+    return worst, mae

@@ -1,0 +1,144 @@
+"""The C ABI library loads, exports every declared symbol, and validates its
+arguments on the host before touching a device (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import sparse_mixture_experts_rms_b200 as moe
+from sparse_mixture_experts_rms_b200 import build as moe_build
+from oracle import moe_oracle as O
+import moe_workloads as mw
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moe_build.build()
+    return moe._lib()
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)))
+
+
+def test_header_declares_every_binding_name():
+    assert _declared_symbols() == sorted(moe.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def _cfg(w: mw.Workload, **kw):
+    offs = moe.ffn_offsets_from_sizes(w.expert_sizes)
+    c = moe.MoEConfig(T=w.T, d_model=w.d_model, E=w.E, k=w.k, ffn_offsets=offs,
+                      capacity_factor=w.capacity_factor, eps=w.eps)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("name", mw.WORKLOAD_ORDER)
+def test_capacity_and_sizes_match_oracle(lib, name):
+    w = mw.WORKLOADS[name]
+    c = _cfg(w)
+    C = O.capacity(w.T, w.k, w.E, float(np.float32(w.capacity_factor)))
+    assert moe.moe_capacity(c) == (-1 if C is None else C)
+    mk = w.T * w.k if C is None else min(w.T * w.k, w.E * C)
+    assert moe.moe_max_kept(c) == mk
+    ws = moe.moe_workspace_size(c)
+    widths = O.expert_widths(w.expert_sizes)
+    assert c.ffn_offsets == O.expert_offsets(widths)
+    # at least the expert intermediates: x_perm, H (max width), y
+    assert ws >= mk * (2 * w.d_model + max(widths)) * 2
+
+
+def test_switch_capacity_is_320(lib):
+    assert moe.moe_capacity(_cfg(mw.WORKLOADS["switch_capacity"])) == 320
+
+
+def test_capacity_rounding_on_fp32_factor(lib):
+    w = mw.WORKLOADS["tiny"]
+    for cf in (0.3, 1.1, 1.25, 2.0, 0.01):
+        c = _cfg(w, capacity_factor=cf)
+        assert moe.moe_capacity(c) == O.capacity(w.T, w.k, w.E, float(np.float32(cf)))
+
+
+@pytest.mark.parametrize("bad", [
+    dict(k=0), dict(k=9), dict(E=0), dict(d_model=100), dict(d_model=0), dict(T=-1),
+    dict(eps=float("nan")), dict(eps=-1.0), dict(capacity_factor=float("inf")),
+])
+def test_invalid_config_rejected(lib, bad):
+    c = _cfg(mw.WORKLOADS["tiny"], **bad)
+    assert moe.moe_workspace_size(c) == 0
+    assert moe.moe_capacity(c) == -1
+
+
+def test_invalid_widths_rejected(lib):
+    base = mw.WORKLOADS["tiny"]
+    for offs in ([0, 256, 300, 512, 768, 1024, 1280, 1536, 1792],   # width 44
+                 [1, 257, 513, 769, 1025, 1281, 1537, 1793, 2049],  # offsets[0] != 0
+                 [0, 256, 256, 512, 768, 1024, 1280, 1536, 1792]):  # zero width
+        c = _cfg(base, ffn_offsets=offs)
+        assert moe.moe_workspace_size(c) == 0
+
+
+def test_too_many_experts_unsupported(lib):
+    c = moe.MoEConfig(T=16, d_model=128, E=65, k=2, ffn_offsets=[128 * i for i in range(66)])
+    assert moe.moe_workspace_size(c) == 0
+
+
+def _call_layer(lib, cfg, ptrs, ws_ptr, ws_bytes):
+    P = ctypes.c_void_p
+    return lib.moe_layer_fwd(ctypes.byref(cfg.c()), *[P(p) for p in ptrs], P(0), P(0), P(0), P(0),
+                             P(ws_ptr), ws_bytes, P(0))
+
+
+def test_layer_argument_errors_before_any_device_work(lib):
+    c = _cfg(mw.WORKLOADS["tiny"])
+    good = [4096 * (i + 1) for i in range(8)]   # fake, aligned, never dereferenced
+    wsz = moe.moe_workspace_size(c)
+    # null tensor
+    bad = list(good); bad[0] = 0
+    assert _call_layer(lib, c, bad, 1 << 20, wsz) == moe.MOE_ERR_INVALID_ARG
+    # misaligned bf16 matrix
+    bad = list(good); bad[4] += 8
+    assert _call_layer(lib, c, bad, 1 << 20, wsz) == moe.MOE_ERR_ALIGNMENT
+    # workspace too small / missing / misaligned
+    assert _call_layer(lib, c, good, 1 << 20, wsz - 1) == moe.MOE_ERR_WORKSPACE
+    assert _call_layer(lib, c, good, 0, wsz) == moe.MOE_ERR_WORKSPACE
+    assert _call_layer(lib, c, good, (1 << 20) + 16, wsz) == moe.MOE_ERR_ALIGNMENT
+    # k > E
+    ck = _cfg(mw.WORKLOADS["tiny"], k=9)
+    assert _call_layer(lib, ck, good, 1 << 20, wsz) == moe.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_device_reports_no_device(lib):
+    c = _cfg(mw.WORKLOADS["tiny"])
+    good = [4096 * (i + 1) for i in range(8)]
+    wsz = moe.moe_workspace_size(c)
+    assert _call_layer(lib, c, good, 1 << 20, wsz) == moe.MOE_ERR_NO_DEVICE
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert moe.moe_status_string(s).startswith("MOE_")
+    assert "UNKNOWN" in moe.moe_status_string(99)
+
+
+def test_product_does_not_import_oracle():
+    pkg = os.path.join(ROOT, "sparse_mixture_experts_rms_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in src.lower() or f == "__init__.py" and "oracle" not in src, f
+                assert "moe_workloads" not in src, f
