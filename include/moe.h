@@ -157,6 +157,34 @@ MOE_API moe_status_t moe_dispatch(const moe_config_t* cfg, const int32_t* expert
                           int32_t* perm, int32_t* inv_perm, moe_bf16_t* x_perm, void* ws,
                           size_t ws_bytes, void* stream);
 
+/* moe_dispatch for callers that cannot allocate device memory.
+ * (No counterpart in the pages: this is a deployment variant.)
+ * Some callers own no allocator: an inference engine that hands a plugin only
+ * its input and output buffers, a runtime that forbids cudaMalloc after start-up
+ * (it synchronises the device and can fail under memory pressure), or code that
+ * runs inside another library's memory pool.  Such callers cannot provide the
+ * workspace moe_dispatch needs for its per-tile count vectors, so this variant
+ * keeps that scratch in a fixed array inside the library (a file-scope
+ * __device__ array of 256 KiB + 256 B, held by every GPU that loads the
+ * library until the process exits).  It allocates nothing and takes no
+ * workspace; arguments and results are those of moe_dispatch.
+ *  - Limit: T*k <= 1048576 assignments (the array holds the count vectors of
+ *    1024 tiles of 1024 assignments for up to 64 experts); larger problems
+ *    return MOE_ERR_UNSUPPORTED before anything is enqueued.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any
+ *    stream capture.
+ *  - Every call on a device shares the one array, which keeps the last call's
+ *    contents; the call clears what must start at zero.  Calls that overlap on
+ *    the GPU (e.g. on two streams at once) race on the array: serialise them.
+ *  - The device error word also lives in the array and is not readable through
+ *    moe_get_device_error: an expert id outside [0, E) is dropped
+ *    (inv_perm = -1) and left out of counts, so sum(counts) < T*k reveals it. */
+MOE_API moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const int32_t* expert_idx,
+                                          const moe_bf16_t* x, const moe_bf16_t* gamma,
+                                          int32_t* counts, int32_t* expert_offsets, int32_t* perm,
+                                          int32_t* inv_perm, moe_bf16_t* x_perm, void* stream);
+
 /* Experts: the two grouped GEMMs over the expert-centric order.
  *   x_perm   [T*k, d] bf16   in (moe_dispatch)
  *   r        [T]      fp32   in (moe_route): applied in GEMM 1's epilogue

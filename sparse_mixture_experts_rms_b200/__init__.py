@@ -39,6 +39,7 @@ MOE_DEVERR_TILE_TABLE = 0x4
 
 EXPORTED = ["moe_status_string", "moe_capacity", "moe_max_kept", "moe_workspace_size",
             "moe_workspace_init", "moe_get_device_error", "moe_route", "moe_dispatch",
+            "moe_dispatch_noalloc",
             "moe_experts_fwd", "moe_experts_up", "moe_experts_down", "moe_combine",
             "moe_layer_fwd"]
 
@@ -95,6 +96,8 @@ def _lib():
         lib.moe_route.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, SZ, P]
         lib.moe_dispatch.restype = ctypes.c_int
         lib.moe_dispatch.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_dispatch_noalloc.restype = ctypes.c_int
+        lib.moe_dispatch_noalloc.argtypes = [cfgp, P, P, P, P, P, P, P, P, P]
         lib.moe_experts_fwd.restype = ctypes.c_int
         lib.moe_experts_fwd.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, SZ, P]
         lib.moe_experts_up.restype = ctypes.c_int
@@ -257,6 +260,25 @@ def moe_dispatch(cfg: MoEConfig, expert_idx, x, gamma, counts, expert_offsets, p
         _ptr(inv_perm, "inv_perm", i32, (T * k,)), _ptr(x_perm, "x_perm", bf),
         _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
     _check(st, "moe_dispatch")
+
+
+def moe_dispatch_noalloc(cfg: MoEConfig, expert_idx, x, gamma, counts, expert_offsets, perm,
+                         inv_perm, x_perm, stream=None) -> None:
+    """moe_dispatch without a workspace, for callers that cannot allocate device
+    memory: the scratch is a fixed array inside the library (T*k <= 2^20)."""
+    T, d, E, k = cfg.T, cfg.d_model, cfg.E, cfg.k
+    i32, bf = torch.int32, torch.bfloat16
+    if x_perm is not None and (x_perm.dim() != 2 or x_perm.shape[1] != d
+                               or x_perm.shape[0] < moe_max_kept(cfg)):
+        raise ValueError("x_perm must be [>= moe_max_kept(cfg), d]")
+    if perm is not None and perm.numel() < moe_max_kept(cfg):
+        raise ValueError("perm must hold >= moe_max_kept(cfg) entries")
+    st = _lib().moe_dispatch_noalloc(
+        ctypes.byref(cfg.c()), _ptr(expert_idx, "expert_idx", i32, (T, k)), _ptr(x, "x", bf, (T, d)),
+        _ptr(gamma, "gamma", bf, (d,)), _ptr(counts, "counts", i32, (E,)),
+        _ptr(expert_offsets, "expert_offsets", i32, (E + 1,)), _ptr(perm, "perm", i32),
+        _ptr(inv_perm, "inv_perm", i32, (T * k,)), _ptr(x_perm, "x_perm", bf), _stream(stream))
+    _check(st, "moe_dispatch_noalloc")
 
 
 def moe_experts_fwd(cfg: MoEConfig, x_perm, r, gate, perm, expert_offsets, W1, W3, W2, y,

@@ -307,6 +307,36 @@ moe_status_t run_combine(const moe_config_t& c, const moe_bf16_t* y, const int32
   return cuda_status(launch_combine(a, sms, s));
 }
 
+// ---- scratch of moe_dispatch_noalloc: a fixed device array instead of a workspace
+constexpr int64_t kNoallocMaxAssignments = int64_t(1) << 20;
+constexpr size_t kNoallocHeaderInts = 64;  // 256 B: the error word, then padding
+constexpr size_t kNoallocCountInts =
+    static_cast<size_t>(kNoallocMaxAssignments / kDispatchTile) * kMaxExperts;  // 256 KiB
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoallocHeaderInts + kNoallocCountInts];
+
+int32_t* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up once per
+// device; in host code the symbol itself is only a host-side stand-in).
+moe_status_t noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -416,6 +446,54 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const int32_t* expert_idx, co
   if ((st = device_ready(&sms)) != MOE_OK) return st;
   return run_dispatch(*cfg, L, ws, expert_idx, x, gamma, counts, expert_offsets, perm, inv_perm,
                       x_perm, sms, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const int32_t* expert_idx,
+                                  const moe_bf16_t* x, const moe_bf16_t* gamma, int32_t* counts,
+                                  int32_t* expert_offsets, int32_t* perm, int32_t* inv_perm,
+                                  moe_bf16_t* x_perm, void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  const int64_t tk = static_cast<int64_t>(cfg->T) * cfg->k;
+  if (tk > kNoallocMaxAssignments) return MOE_ERR_UNSUPPORTED;
+  if (!counts || !expert_offsets) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!expert_idx || !x || !gamma || !perm || !inv_perm || !x_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(expert_idx, 4) || !aligned(counts, 4) || !aligned(expert_offsets, 4) ||
+      !aligned(perm, 4) || !aligned(inv_perm, 4) || !aligned(x, 16) || !aligned(gamma, 16) ||
+      !aligned(x_perm, 16))
+    return MOE_ERR_ALIGNMENT;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  int32_t* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cfg->T == 0) {
+    cudaError_t e = cudaMemsetAsync(expert_offsets, 0, (cfg->E + 1) * sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, cfg->E * sizeof(int32_t), s);
+    return cuda_status(e);
+  }
+  // the error word must start at zero; the tile counts are fully rewritten
+  cudaError_t e = cudaMemsetAsync(scratch, 0, kNoallocHeaderInts * sizeof(int32_t), s);
+  if (e != cudaSuccess) return cuda_status(e);
+  DispatchArgs a{};
+  a.idx = expert_idx;
+  a.x = reinterpret_cast<const __nv_bfloat16*>(x);
+  a.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
+  a.tile_counts = scratch + kNoallocHeaderInts;
+  a.counts = counts;
+  a.offsets = expert_offsets;
+  a.perm = perm;
+  a.inv_perm = inv_perm;
+  a.x_perm = reinterpret_cast<__nv_bfloat16*>(x_perm);
+  a.err = reinterpret_cast<uint32_t*>(scratch);
+  a.T = cfg->T;
+  a.d = cfg->d_model;
+  a.E = cfg->E;
+  a.k = cfg->k;
+  a.capacity = static_cast<int>(capacity_of(*cfg));
+  a.max_kept = static_cast<int>(max_kept_of(*cfg));
+  return cuda_status(launch_dispatch(a, sms, s));
 }
 
 moe_status_t moe_experts_fwd(const moe_config_t* cfg, const moe_bf16_t* x_perm, const float* r,
