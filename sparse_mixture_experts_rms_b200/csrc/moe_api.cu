@@ -23,6 +23,7 @@ struct DeviceState {
   bool ready = false;
   bool ok = false;
   int sms = 0;
+  int gemm_grid = 0;
 };
 
 std::mutex g_mutex;
@@ -146,11 +147,20 @@ moe_status_t device_ready(int* sms) {
     }
     if (g_encode == nullptr) return MOE_ERR_CUDA;
     st.sms = prop.multiProcessorCount;
+    st.gemm_grid = grouped_gemm_max_grid(st.sms);
+    if (st.gemm_grid < 2) return MOE_ERR_CUDA;
     st.ok = true;
   }
   if (!st.ok) return MOE_ERR_NO_DEVICE;
   *sms = st.sms;
   return MOE_OK;
+}
+
+int gemm_grid_of_current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(g_mutex);
+  return g_dev[dev].gemm_grid;
 }
 
 // 2-D bf16 tensor map with 128-byte swizzle: `inner` contiguous elements per
@@ -260,7 +270,8 @@ moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_
   g.scale = r;
   g.out = at<__nv_bfloat16>(ws, L.H);
   g.ld_out = L.ldh;
-  return cuda_status(launch_grouped_gemm(g, mA, mB0, mB1, sms, s));
+  (void)sms;
+  return cuda_status(launch_grouped_gemm(g, mA, mB0, mB1, gemm_grid_of_current_device(), s));
 }
 
 // GEMM 2: H [rows, f_e] (workspace) x W2 [F, d] -> y [rows, d], gate in the epilogue
@@ -283,7 +294,8 @@ moe_status_t run_down(const moe_config_t& c, const Layout& L, void* ws, const fl
   g.scale = gate;
   g.out = reinterpret_cast<__nv_bfloat16*>(y);
   g.ld_out = c.d_model;
-  return cuda_status(launch_grouped_gemm(g, mA, mB, mB, sms, s));
+  (void)sms;
+  return cuda_status(launch_grouped_gemm(g, mA, mB, mB, gemm_grid_of_current_device(), s));
 }
 
 moe_status_t run_experts(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x_perm,

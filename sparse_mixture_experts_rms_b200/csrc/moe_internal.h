@@ -83,6 +83,9 @@ cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);
 
 // One-time per-device kernel attributes (dynamic shared memory opt-in).
 cudaError_t prepare_grouped_gemm();
+// Persistent grid of the grouped GEMM: an even number of CTAs (pairs), at most
+// the number of co-resident 2-CTA clusters times 2.
+int grouped_gemm_max_grid(int num_sms);
 size_t grouped_gemm_smem_bytes();
 
 }  // namespace moe
