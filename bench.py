@@ -39,7 +39,7 @@ import moe_workloads as mw  # noqa: E402
 METRIC = "MoE layer fwd tokens/s & TFLOP/s, % of B200 bf16 peak / HBM roofline"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 7  # route, dispatch count/scatter/permute, GEMM up, GEMM down, combine
+KERNELS_PER_STEP = 8  # router weights, route, dispatch count/scatter/permute, GEMM up, GEMM down, combine
 
 
 def parse_args():

@@ -132,7 +132,8 @@ MOE_API moe_status_t moe_get_device_error(void* ws, size_t ws_bytes, void* strea
  *   gate     [T, k]   fp32   out: softmax(l_t) at the chosen experts
  *   r        [T]      fp32   out: RMS statistic
  *   logits   [T, E]   fp32   out (optional, NULL to skip): router logits
- * Logits accumulate exact bf16*bf16 products in fp32. */
+ * Logits accumulate exact bf16*bf16 products in fp32.  The workspace (at least
+ * moe_workspace_size(cfg) bytes) holds gamma*Wr in fp32 and the error word. */
 MOE_API moe_status_t moe_route(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
                        const moe_bf16_t* Wr, const float* bias, int32_t* expert_idx, float* gate,
                        float* r, float* logits, void* ws, size_t ws_bytes, void* stream);

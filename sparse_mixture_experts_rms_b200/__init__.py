@@ -231,8 +231,8 @@ def moe_get_device_error(ws: torch.Tensor, stream=None, raise_on_error: bool = T
     return int(code.value)
 
 
-def moe_route(cfg: MoEConfig, x, gamma, Wr, bias, expert_idx, gate, r, logits=None,
-              ws: Optional[torch.Tensor] = None, stream=None) -> None:
+def moe_route(cfg: MoEConfig, x, gamma, Wr, bias, expert_idx, gate, r, logits,
+              ws: torch.Tensor, stream=None) -> None:
     T, d, E, k = cfg.T, cfg.d_model, cfg.E, cfg.k
     bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
     st = _lib().moe_route(
@@ -240,7 +240,7 @@ def moe_route(cfg: MoEConfig, x, gamma, Wr, bias, expert_idx, gate, r, logits=No
         _ptr(Wr, "Wr", bf, (d, E)), _ptr(bias, "bias", f32, (E,)),
         _ptr(expert_idx, "expert_idx", i32, (T, k)), _ptr(gate, "gate", f32, (T, k)),
         _ptr(r, "r", f32, (T,)), _ptr(logits, "logits", f32, (T, E)),
-        _ptr(ws, "ws", torch.uint8), 0 if ws is None else ws.numel(), _stream(stream))
+        _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
     _check(st, "moe_route")
 
 

@@ -36,7 +36,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct Layout {
-  size_t err, tile_counts, r, idx, gate, counts, offsets, perm, inv_perm, x_perm, H, y, total;
+  size_t err, rw, tile_counts, r, idx, gate, counts, offsets, perm, inv_perm, x_perm, H, y, total;
   int64_t max_kept;
   int ldh;
 };
@@ -92,6 +92,7 @@ Layout layout_of(const moe_config_t& c) {
   L.ldh = fmax;
   const size_t mk = static_cast<size_t>(L.max_kept);
   L.err = 0;
+  L.rw = take(static_cast<size_t>(c.d_model) * kRouterPadE * 4);
   L.tile_counts = take(ntiles * c.E * 4);
   L.r = take(static_cast<size_t>(c.T) * 4);
   L.idx = take(tk * 4);
@@ -189,8 +190,10 @@ T* at(void* ws, size_t off) {
 
 moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf16_t* gamma,
                        const moe_bf16_t* Wr, const float* bias, int32_t* idx, float* gate, float* r,
-                       float* logits, cudaStream_t s) {
+                       float* logits, uint32_t* err, float* wprime, cudaStream_t s) {
+  if (c.T == 0) return MOE_OK;
   RouteArgs a{};
+  a.wprime = wprime;
   a.x = reinterpret_cast<const __nv_bfloat16*>(x);
   a.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
   a.Wr = reinterpret_cast<const __nv_bfloat16*>(Wr);
@@ -199,13 +202,19 @@ moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf1
   a.gate = gate;
   a.r = r;
   a.logits = logits;
+  a.err = err;
   a.T = c.T;
   a.d = c.d_model;
   a.E = c.E;
   a.k = c.k;
   a.eps = c.eps;
   a.renormalize = c.renormalize ? 1 : 0;
-  return cuda_status(launch_route(a, s));
+  CUtensorMap xmap;
+  // x [T, d]: tiles of 64 tokens x 64 elements
+  if (!make_map(&xmap, x, static_cast<uint64_t>(c.d_model), static_cast<uint64_t>(c.T),
+                static_cast<uint64_t>(c.d_model), 64, 64))
+    return MOE_ERR_CUDA;
+  return cuda_status(launch_route(a, xmap, s));
 }
 
 moe_status_t run_dispatch(const moe_config_t& c, const Layout& L, void* ws, const int32_t* idx,
@@ -417,8 +426,6 @@ moe_status_t moe_route(const moe_config_t* cfg, const moe_bf16_t* x, const moe_b
                        float* r, float* logits, void* ws, size_t ws_bytes, void* stream) {
   moe_status_t st = validate(cfg);
   if (st != MOE_OK) return st;
-  (void)ws;
-  (void)ws_bytes;
   if (cfg->T == 0) return MOE_OK;  // no tokens: nothing to do (pointers may be null)
   if (!x || !gamma || !Wr || !expert_idx || !gate || !r) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) ||
@@ -426,8 +433,10 @@ moe_status_t moe_route(const moe_config_t* cfg, const moe_bf16_t* x, const moe_b
     return MOE_ERR_ALIGNMENT;
   int sms;
   if ((st = device_ready(&sms)) != MOE_OK) return st;
-  return run_route(*cfg, x, gamma, Wr, bias, expert_idx, gate, r, logits,
-                   static_cast<cudaStream_t>(stream));
+  Layout L;
+  if ((st = check_ws(*cfg, ws, ws_bytes, &L)) != MOE_OK) return st;
+  return run_route(*cfg, x, gamma, Wr, bias, expert_idx, gate, r, logits, at<uint32_t>(ws, L.err),
+                   at<float>(ws, L.rw), static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_dispatch(const moe_config_t* cfg, const int32_t* expert_idx, const moe_bf16_t* x,
@@ -612,7 +621,9 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x, const m
   int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
   moe_bf16_t* x_perm = at<moe_bf16_t>(ws, L.x_perm);
   moe_bf16_t* y = at<moe_bf16_t>(ws, L.y);
-  if ((st = run_route(c, x, gamma, Wr, bias, idx_, gate_, r_, nullptr, s)) != MOE_OK) return st;
+  if ((st = run_route(c, x, gamma, Wr, bias, idx_, gate_, r_, nullptr, at<uint32_t>(ws, L.err),
+                      at<float>(ws, L.rw), s)) != MOE_OK)
+    return st;
   if ((st = run_dispatch(c, L, ws, idx_, x, gamma, counts_, offsets, perm, inv_perm, x_perm, sms, s)) != MOE_OK)
     return st;
   if ((st = run_experts(c, L, ws, x_perm, r_, gate_, perm, offsets, W1, W3, W2, y, sms, s)) != MOE_OK)

@@ -13,6 +13,7 @@
 namespace moe {
 
 constexpr int kMaxExperts = 64;
+constexpr int kRouterPadE = 64;         // w' scratch is sized for the widest router variant
 constexpr int kBlockN = 128;            // expert width granule (and G1's N per projection)
 constexpr int kDispatchTile = 1024;     // assignments per dispatch CTA
 constexpr uint64_t kWaitTimeoutNs = 4000000000ull;  // bounded pipeline waits: 4 s
@@ -31,6 +32,8 @@ struct RouteArgs {
   float* gate;
   float* r;
   float* logits;      // may be null
+  uint32_t* err;      // device error word, may be null
+  float* wprime;      // [d, EP] fp32 scratch: gamma * Wr, zero-padded
   int T, d, E, k;
   float eps;
   int renormalize;
@@ -74,7 +77,7 @@ struct CombineArgs {
 };
 
 // Launchers (return the launch error, if any).
-cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA,
                                 const CUtensorMap& mapB0, const CUtensorMap& mapB1, int grid,

@@ -3,111 +3,250 @@
 // CODA sparse-MoE thread (digg.com), RMSNorm paragraphs: the router is a plain
 // GEMM right after the RMSNorm, and the scale by the statistic r commutes
 // across it, so it is applied in the GEMM's epilogue right before the top-k:
-//     l_te = r_t * sum_i x_ti * (gamma_i * Wr_ie) + b_e .
+//     l_te = r_t * sum_i x_ti * w'_ie + b_e ,   w'_ie = gamma_i * Wr_ie .
 // MoE glossary (inferensys.com), "Top-k Gating" / "Switch Routing": the k
 // largest router scores pick the experts; their softmax probabilities weight
 // the expert outputs.
 //
-// One thread owns one token.  The token's row streams through L1 in 16-byte
-// loads (the only pass over x); gamma*Wr is staged in shared memory in fp32
-// chunks of 128 rows.  gamma_i*Wr_ie (two bf16) is exact in fp32, and so is
-// x_ti times it, so the only rounding is the fp32 accumulation, done per
-// 128-element chunk and then across chunks.  Sum of squares likewise.
+// The contraction runs on the tensor cores (warp-level mma.sync m16n8k16,
+// bf16 in, fp32 out) without losing the exactness routing needs:
+//  - w' (two bf16 multiplied: 16 significant bits) is split exactly into
+//    w' = hi + lo with hi, lo bf16 (8 bits each), so x*w' = x*hi + x*lo and
+//    every product the tensor core forms is exact;
+//  - each 64-element chunk is accumulated by the MMAs from zero (4 k-steps),
+//    and the chunk partials are summed in fp64; r and l = r*acc + b are
+//    formed in fp64 and each logit is rounded once to fp32.
+// A near-tie between the k-th and (k+1)-th logit can therefore only flip when
+// the two fp32 logits differ by about one ulp.
+//
+// Layout: a CTA (4 warps) owns 64 tokens, a warp 16.  x streams through a ring
+// of stages, each a TMA tile [64 tokens x 64 elements] (128-byte swizzle;
+// ldmatrix reads it conflict-free) plus the chunk's B fragments of hi/lo
+// (precomputed once per call into the workspace, in the per-lane order the
+// MMA wants, and fetched with one bulk copy).  The sum of squares for r comes
+// from the same A fragments.  Logits meet in shared memory, where one thread
+// per token does the softmax and the top-k.
 #include "moe_internal.h"
+#include "ptx.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kRouteChunk = 128;
+constexpr int kTok = 64;                       // tokens per CTA
+constexpr int kWarps = kTok / 16;              // a warp owns 16 tokens (MMA rows)
+constexpr int kThreads = kWarps * 32;
+constexpr int kChunk = 64;                     // elements of d per stage (4 k-steps)
+constexpr int kTileBytes = kTok * kChunk * 2;  // 8 KB of x per stage
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+template <int EP>
+struct RouteCfg {
+  static constexpr int NT = EP / 8;                            // MMA n-tiles
+  static constexpr int kFragBytes = 4 * NT * 2 * 32 * 8;       // k-steps x tiles x {hi,lo} x lanes x 8 B
+  static constexpr int kStageBytes = kTileBytes + kFragBytes;  // a multiple of 1024
+  static constexpr int kRing = EP <= 16 ? 6 : (EP == 32 ? 5 : 4);
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kRing) * kStageBytes + 64;
+};
+
+__device__ __forceinline__ uint32_t bf16_bits_rn(float v) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h));
+}
+
+// B fragments of hi(w') and lo(w') for every (k-step, n-tile, lane):
+// b0 = {w'[k0][n], w'[k0+1][n]}, b1 = {w'[k0+8][n], w'[k0+9][n]},
+// k0 = 16*ks + 2*(lane%4), n = 8*nt + lane/4 (zero for n >= E).
+__global__ void router_weight_kernel(const RouteArgs a, int nt_count) {
+  const int ksteps = a.d / 16;
+  const int n = ksteps * nt_count * 2 * 32;
+  const uint16_t* gam = reinterpret_cast<const uint16_t*>(a.gamma);
+  const uint16_t* wr = reinterpret_cast<const uint16_t*>(a.Wr);
+  uint2* out = reinterpret_cast<uint2*>(a.wprime);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int lane = i % 32;
+    const int hl = (i / 32) % 2;
+    const int nt = (i / 64) % nt_count;
+    const int ks = i / (64 * nt_count);
+    const int col = nt * 8 + lane / 4;
+    const int k0 = ks * 16 + 2 * (lane % 4);
+    uint32_t h16[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    for (int j = 0; j < 4; ++j) {
+      const int kk = k0 + (j & 1) + (j >> 1) * 8;
+      float w = 0.f;
+      if (col < a.E) {
+        const float g = __uint_as_float(static_cast<uint32_t>(gam[kk]) << 16);
+        const float v = __uint_as_float(static_cast<uint32_t>(wr[static_cast<size_t>(kk) * a.E + col]) << 16);
+        w = g * v;  // exact
+      }
+      const uint32_t hi = bf16_bits_rn(w);
+      const float hif = __uint_as_float(hi << 16);
+      h16[j] = hl == 0 ? hi : bf16_bits_rn(w - hif);  // w - hi is exact and fits in bf16
+    }
+    out[i] = make_uint2(h16[0] | (h16[1] << 16), h16[2] | (h16[3] << 16));
   }
 }
 
-template <int EP, int TPB>
-__global__ void __launch_bounds__(TPB) route_kernel(const RouteArgs a) {
-  extern __shared__ __align__(16) float w_s[];  // [kRouteChunk][EP]
-  const int t = blockIdx.x * TPB + threadIdx.x;
-  const bool valid = t < a.T;
-  const uint4* xrow = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(valid ? t : 0) * a.d);
-  const uint16_t* gam = reinterpret_cast<const uint16_t*>(a.gamma);
-  const uint16_t* wr = reinterpret_cast<const uint16_t*>(a.Wr);
+template <int EP>
+__global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                         const RouteArgs a) {
+  using Cfg = RouteCfg<EP>;
+  constexpr int NT = Cfg::NT;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + Cfg::kRing * Cfg::kStageBytes);
+  int* abort_flag = reinterpret_cast<int*>(full + Cfg::kRing);
+  uint32_t* dummy_err = reinterpret_cast<uint32_t*>(abort_flag + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t0 = blockIdx.x * kTok;
+  uint32_t* err = a.err ? a.err : dummy_err;
+  const int nchunks = a.d / kChunk;
+  const uint8_t* frag_src = reinterpret_cast<const uint8_t*>(a.wprime);
 
-  float acc[EP];
-#pragma unroll
-  for (int e = 0; e < EP; ++e) acc[e] = 0.f;
-  float ss = 0.f;
+  auto issue = [&](int c, int s) {
+    uint8_t* st = ring + s * Cfg::kStageBytes;
+    mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
+    tma_load_2d(st, &xmap, &full[s], c * kChunk, t0);
+    bulk_load(st + kTileBytes, frag_src + static_cast<size_t>(c) * Cfg::kFragBytes, Cfg::kFragBytes, &full[s]);
+  };
 
-  for (int c0 = 0; c0 < a.d; c0 += kRouteChunk) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < kRouteChunk * EP; i += TPB) {
-      const int row = i / EP, e = i % EP;
-      float w = 0.f;
-      if (e < a.E) {
-        const float g = __uint_as_float(static_cast<uint32_t>(gam[c0 + row]) << 16);
-        const float v = __uint_as_float(static_cast<uint32_t>(wr[static_cast<size_t>(c0 + row) * a.E + e]) << 16);
-        w = g * v;  // exact: two 8-bit significands
-      }
-      w_s[i] = w;
-    }
-    __syncthreads();
-    float part[EP];
+  if (tid == 0) {
+    for (int s = 0; s < Cfg::kRing; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    *dummy_err = 0;
+    fence_mbar_init();
+    tma_prefetch_map(&xmap);
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int c = 0; c < Cfg::kRing && c < nchunks; ++c) issue(c, c);
+
+  // accumulators: this lane's C elements (rows g, g+8; columns 2t, 2t+1 of each n-tile)
+  double acc[NT][4];
 #pragma unroll
-    for (int e = 0; e < EP; ++e) part[e] = 0.f;
-    float ssp = 0.f;
-#pragma unroll 2
-    for (int i = 0; i < kRouteChunk; i += 8) {
-      float xv[8];
-      bf16x8_to_f32(__ldg(xrow + (c0 + i) / 8), xv);
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        ssp = fmaf(xv[j], xv[j], ssp);
-        const float4* wrow = reinterpret_cast<const float4*>(w_s + (i + j) * EP);
+    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0;
+  double ss_g = 0.0, ss_g8 = 0.0;
+  bool ok = true;
+
+  // ldmatrix row address of this lane: matrix m = lane/8 -> rows +8*(m&1), k piece +(m>>1)
+  const int lrow = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int lpiece = lane >> 4;
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int s = c % Cfg::kRing;
+    const uint32_t ph = (c / Cfg::kRing) & 1u;
+    if (ok) ok = mbar_wait(&full[s], ph, abort_flag, err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs);
+    if (ok) {
+      const uint8_t* st = ring + s * Cfg::kStageBytes;
+      const uint2* frag = reinterpret_cast<const uint2*>(st + kTileBytes);
+      const uint32_t tile = smem_addr(st);
+      float chi[NT][4], clo[NT][4];
 #pragma unroll
-        for (int q = 0; q < EP / 4; ++q) {
-          const float4 w = wrow[q];
-          part[4 * q + 0] = fmaf(xv[j], w.x, part[4 * q + 0]);
-          part[4 * q + 1] = fmaf(xv[j], w.y, part[4 * q + 1]);
-          part[4 * q + 2] = fmaf(xv[j], w.z, part[4 * q + 2]);
-          part[4 * q + 3] = fmaf(xv[j], w.w, part[4 * q + 3]);
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) chi[nt][i] = clo[nt][i] = 0.f;
+      float sg = 0.f, sg8 = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int piece = 2 * kk + lpiece;
+        uint32_t av[4];
+        ldmatrix_x4(tile + lrow * 128 + ((piece ^ (lrow & 7)) << 4), av);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float lo = __uint_as_float(av[i] << 16), hi = __uint_as_float(av[i] & 0xFFFF0000u);
+          if (i & 1) {
+            sg8 = fmaf(lo, lo, sg8);
+            sg8 = fmaf(hi, hi, sg8);
+          } else {
+            sg = fmaf(lo, lo, sg);
+            sg = fmaf(hi, hi, sg);
+          }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint2 bh = frag[((kk * NT + nt) * 2 + 0) * 32 + lane];
+          const uint2 bl = frag[((kk * NT + nt) * 2 + 1) * 32 + lane];
+          mma_bf16_16816(chi[nt], av, bh.x, bh.y);
+          mma_bf16_16816(clo[nt], av, bl.x, bl.y);
         }
       }
-    }
 #pragma unroll
-    for (int e = 0; e < EP; ++e) acc[e] += part[e];
-    ss += ssp;
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][i] += static_cast<double>(chi[nt][i]) + static_cast<double>(clo[nt][i]);
+      ss_g += static_cast<double>(sg);
+      ss_g8 += static_cast<double>(sg8);
+    }
+    // every warp is done with stage s; a wait that gave up anywhere stops the CTA
+    ok = __syncthreads_and(ok) != 0;
+    if (tid == 0 && ok && c + Cfg::kRing < nchunks) issue(c + Cfg::kRing, s);
   }
-  if (!valid) return;
+  if (!ok) {
+    // a stage never arrived: let the copies already issued land before exiting
+    if (tid == 0) {
+      volatile int no_abort = 0;
+      for (int c = (nchunks > Cfg::kRing ? nchunks - Cfg::kRing : 0); c < nchunks; ++c)
+        mbar_wait(&full[c % Cfg::kRing], (c / Cfg::kRing) & 1u, &no_abort, err, MOE_DEVERR_TIMEOUT,
+                  kWaitTimeoutNs);
+    }
+    return;
+  }
 
-  const float r = 1.0f / sqrtf(ss / static_cast<float>(a.d) + a.eps);
+  // sum of squares of rows g and g+8 over the quad's columns
+#pragma unroll
+  for (int m = 1; m <= 2; m <<= 1) {
+    ss_g += __shfl_xor_sync(0xFFFFFFFFu, ss_g, m);
+    ss_g8 += __shfl_xor_sync(0xFFFFFFFFu, ss_g8, m);
+  }
+  const int g = lane >> 2, tq = lane & 3;
+  const int row_g = warp * 16 + g, row_g8 = row_g + 8;
+  const double inv_d = 1.0 / static_cast<double>(a.d);
+  const double r_g = 1.0 / sqrt(ss_g * inv_d + static_cast<double>(a.eps));
+  const double r_g8 = 1.0 / sqrt(ss_g8 * inv_d + static_cast<double>(a.eps));
+
+  // logits of the CTA's 64 tokens meet in shared memory (the ring is idle now)
+  float* lg = reinterpret_cast<float*>(ring);
+  float* rr = lg + kTok * EP;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = nt * 8 + 2 * tq + (i & 1);
+      const int row = (i < 2) ? row_g : row_g8;
+      const double rv = (i < 2) ? r_g : r_g8;
+      const double b = (a.bias != nullptr && e < a.E) ? static_cast<double>(a.bias[e]) : 0.0;
+      lg[row * EP + e] = e < a.E ? static_cast<float>(fma(rv, acc[nt][i], b)) : -INFINITY;
+    }
+  }
+  if (tq == 0) {
+    rr[row_g] = static_cast<float>(r_g);
+    rr[row_g8] = static_cast<float>(r_g8);
+  }
+  __syncthreads();
+  if (tid >= kTok) return;
+  const int t = t0 + tid;
+  if (t >= a.T) return;
+
   float l[EP];
   float m = -INFINITY;
 #pragma unroll
   for (int e = 0; e < EP; ++e) {
-    if (e < a.E) {
-      l[e] = fmaf(r, acc[e], a.bias ? a.bias[e] : 0.f);
-      m = fmaxf(m, l[e]);
-    } else {
-      l[e] = -INFINITY;
-    }
+    l[e] = lg[tid * EP + e];
+    if (e < a.E) m = fmaxf(m, l[e]);
   }
-  float s = 0.f;
+  float sum = 0.f;
 #pragma unroll
   for (int e = 0; e < EP; ++e)
-    if (e < a.E) s += expf(l[e] - m);
-  const float inv_s = 1.0f / s;
+    if (e < a.E) sum += expf(l[e] - m);
+  const float inv_s = 1.0f / sum;
 
   if (a.logits) {
 #pragma unroll
     for (int e = 0; e < EP; ++e)
       if (e < a.E) a.logits[static_cast<size_t>(t) * a.E + e] = l[e];
   }
-  a.r[t] = r;
+  a.r[t] = rr[tid];
 
   // top-k: k rounds of a first-maximum scan (strict '>' keeps the lower index on ties)
   uint64_t used = 0;
@@ -125,10 +264,10 @@ __global__ void __launch_bounds__(TPB) route_kernel(const RouteArgs a) {
       }
     }
     used |= 1ull << bi;
-    const float g = expf(best - m) * inv_s;
+    const float gt = expf(best - m) * inv_s;
     a.idx[base + j] = bi;
-    a.gate[base + j] = g;
-    gsum += g;
+    a.gate[base + j] = gt;
+    gsum += gt;
   }
   if (a.renormalize) {
     const float inv = 1.0f / gsum;
@@ -136,22 +275,33 @@ __global__ void __launch_bounds__(TPB) route_kernel(const RouteArgs a) {
   }
 }
 
-template <int EP, int TPB>
-cudaError_t launch_route_t(const RouteArgs& a, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(kRouteChunk) * EP * sizeof(float);
-  const int grid = (a.T + TPB - 1) / TPB;
-  route_kernel<EP, TPB><<<grid, TPB, smem, s>>>(a);
+template <int EP>
+cudaError_t launch_route_t(const RouteArgs& a, const CUtensorMap& xmap, cudaStream_t s) {
+  const size_t smem = RouteCfg<EP>::kSmem;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(route_kernel<EP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  const int n = (a.d / 16) * RouteCfg<EP>::NT * 64;
+  router_weight_kernel<<<(n + 255) / 256, 256, 0, s>>>(a, RouteCfg<EP>::NT);
+  const int grid = (a.T + kTok - 1) / kTok;
+  route_kernel<EP><<<grid, kThreads, smem, s>>>(xmap, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
+cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
-  if (a.E <= 8) return launch_route_t<8, 64>(a, s);
-  if (a.E <= 16) return launch_route_t<16, 64>(a, s);
-  if (a.E <= 32) return launch_route_t<32, 64>(a, s);
-  return launch_route_t<64, 64>(a, s);
+  if (a.E <= 8) return launch_route_t<8>(a, xmap, s);
+  if (a.E <= 16) return launch_route_t<16>(a, xmap, s);
+  if (a.E <= 32) return launch_route_t<32>(a, xmap, s);
+  return launch_route_t<64>(a, xmap, s);
 }
 
 }  // namespace moe
