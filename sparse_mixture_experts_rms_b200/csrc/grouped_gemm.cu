@@ -215,7 +215,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int kblocks = a.up ? a.d / BK : (a.ffn.off[c.e + 1] - o_e) / BK;
         const uint32_t buf = tcount & 1u;
         const uint32_t aph = (tcount >> 1) & 1u;
-        if (!mbar_wait(&sh.tempty[buf], aph ^ 1u, abort_flag, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs)) {
+        // both CTAs' epilogues release the buffer (the peer's arrival is remote)
+        if (!mbar_wait(&sh.tempty[buf], aph ^ 1u, abort_flag, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs,
+                       true)) {
           ok = false;
           break;
         }

@@ -50,15 +50,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 // Wait for the phase of `bar` with the given parity to complete, giving up
 // after `timeout_ns` or as soon as *abort is set.  On a timeout it sets
 // *abort and ORs `err_bit` into *err.  Returns false if it gave up.
+// With `cluster` set, the wait acquires at cluster scope (for barriers that
+// receive arrivals released by another CTA of the cluster).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* err, uint32_t err_bit, uint64_t timeout_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+                                          uint32_t* err, uint32_t err_bit, uint64_t timeout_ns,
+                                          bool cluster = false) {
+  auto poll = [&]() { return cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (poll()) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (poll()) return true;
     if ((n & 63u) == 0) {
       if (*abort) return false;
       if (global_timer_ns() - t0 > timeout_ns) {
