@@ -162,6 +162,23 @@ class ClockSampler:
                 "samples_in_timed_region": len(inside)}
 
 
+# ----------------------------------------------------------------- ranks
+def max_over_ranks(v: float, world: int, device=None) -> float:
+    """Maximum of a per-rank value over all ranks (identity when world == 1)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, tokens_per_rank: int, steps: int, ms_total_max: float) -> float:
+    """Whole-job tokens/s of `world` independent replicas timed by the slowest rank."""
+    return world * tokens_per_rank * steps / (ms_total_max * 1e-3)
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local):
     import torch
@@ -213,12 +230,6 @@ def run_ours(args, rank, world, local):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
@@ -242,7 +253,7 @@ def run_ours(args, rank, world, local):
     tw1 = time.time()
     barrier()
     sampler.window(tw0, tw1)
-    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
     ms_step = ms_total / args.steps
 
     # ---- per-stage breakdown: the same kernels through the staged calls
@@ -349,8 +360,9 @@ def run_ours(args, rank, world, local):
         torch.cuda.synchronize()
         sampler.window(tw0, time.time())
         barrier()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
-        e2e = {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+        e2e_total = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
+        e2e_ms = e2e_total / args.steps
+        e2e = {"value": replica_throughput(world, T, args.steps, e2e_total), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": int(x_h.numel() * 2), "d2h_bytes_per_step": int(out_h.numel() * 2)}
 
     clocks = sampler.stop()
@@ -358,7 +370,7 @@ def run_ours(args, rank, world, local):
 
     result = {
         "metric": METRIC,
-        "value": world * T / t_step,
+        "value": replica_throughput(world, T, args.steps, ms_total),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
