@@ -305,6 +305,37 @@ def combine(y: np.ndarray, gate: np.ndarray, kept: np.ndarray) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# router metrics (MoE glossary, "Load Balancing" / "Auxiliary Loss")
+# --------------------------------------------------------------------------
+def router_stats(logits32: np.ndarray, counts: np.ndarray, n_kept: int, k: int) -> Dict[str, object]:
+    """Load-balance metrics of one routing pass, float64.
+
+    prob_mean[e] = (1/T) sum_t softmax(l_t)[e]  (the routing probability mass
+    each expert receives); the glossary's auxiliary loss is the squared
+    coefficient of variation of that distribution across experts,
+    cv2_prob = Var_e(prob_mean) / Mean_e(prob_mean)^2 (population variance);
+    the Switch-style form E * sum_e f_e * prob_mean_e with f_e = counts_e/(T*k)
+    is reported too, with cv2_load (the same CV^2 of the counts) and the
+    fraction of assignments dropped by the capacity limit.
+    """
+    p = softmax(logits32)
+    T, E = p.shape
+    prob_mean = p.mean(axis=0)
+    counts = np.asarray(counts, dtype=np.float64)
+    f = counts / float(T * k)
+
+    def cv2(v):
+        m = v.mean()
+        return float(((v - m) ** 2).mean() / (m * m)) if m != 0 else 0.0
+
+    return {"prob_mean": prob_mean,
+            "aux_loss": float(E * np.sum(f * prob_mean)),
+            "cv2_prob": cv2(prob_mean),
+            "cv2_load": cv2(counts),
+            "dropped_frac": float(1.0 - n_kept / float(T * k))}
+
+
+# --------------------------------------------------------------------------
 # the whole layer
 # --------------------------------------------------------------------------
 def moe_layer(x_bits, gamma_bits, Wr_bits, bias, W1_bits, W3_bits, W2_bits,

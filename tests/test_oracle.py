@@ -309,6 +309,44 @@ def test_sampled_tokens_equal_full_layer():
     np.testing.assert_allclose(out, R["out"][toks], rtol=1e-13, atol=1e-15)
 
 
+# ---------------------------------------------------------------- router metrics
+def test_router_stats_uniform_closed_form():
+    # equal logits: every expert gets probability 1/E; balanced counts
+    E, T, k = 8, 64, 2
+    lg = np.zeros((T, E), dtype=np.float32)
+    counts = np.full(E, T * k // E)
+    st = O.router_stats(lg, counts, n_kept=T * k, k=k)
+    np.testing.assert_allclose(st["prob_mean"], 1.0 / E, rtol=1e-15)
+    assert st["aux_loss"] == pytest.approx(1.0, rel=1e-15)
+    assert st["cv2_prob"] == pytest.approx(0.0, abs=1e-30) and st["cv2_load"] == 0.0
+    assert st["dropped_frac"] == 0.0
+
+
+def test_router_stats_one_hot_closed_form():
+    # one expert takes everything (huge logit): P -> e_j, f = e_j
+    E, T = 6, 50
+    lg = np.zeros((T, E), dtype=np.float32); lg[:, 2] = 200.0
+    counts = np.zeros(E, dtype=np.int64); counts[2] = T
+    st = O.router_stats(lg, counts, n_kept=10, k=1)
+    assert st["aux_loss"] == pytest.approx(E, rel=1e-12)
+    assert st["cv2_prob"] == pytest.approx(E - 1, rel=1e-12)      # CV^2 of a one-hot vector
+    assert st["cv2_load"] == pytest.approx(E - 1, rel=1e-12)
+    assert st["dropped_frac"] == pytest.approx(0.8)
+
+
+def test_router_stats_matches_torch_definitions():
+    rng = np.random.default_rng(8)
+    lg = (1.5 * rng.standard_normal((300, 10))).astype(np.float32)
+    idx = O.topk_experts(lg, 3)
+    counts = np.bincount(idx.reshape(-1), minlength=10)
+    st = O.router_stats(lg, counts, n_kept=900, k=3)
+    P = torch.softmax(_t(lg), dim=1).mean(0)
+    np.testing.assert_allclose(st["prob_mean"], P.numpy(), rtol=1e-13)
+    assert st["cv2_prob"] == pytest.approx(float(P.var(unbiased=False) / P.mean() ** 2), rel=1e-10)
+    assert st["aux_loss"] == pytest.approx(float(10 * (torch.from_numpy(counts / 900.0) * P).sum()), rel=1e-12)
+    assert np.isclose(st["prob_mean"].sum(), 1.0)
+
+
 # ---------------------------------------------------------------- generator
 def test_generator_is_seeded_and_sliceable():
     w = mw.WORKLOADS["tiny"]
