@@ -132,11 +132,29 @@ MOE_API moe_status_t moe_get_device_error(void* ws, size_t ws_bytes, void* strea
  *   gate     [T, k]   fp32   out: softmax(l_t) at the chosen experts
  *   r        [T]      fp32   out: RMS statistic
  *   logits   [T, E]   fp32   out (optional, NULL to skip): router logits
- * Logits accumulate exact bf16*bf16 products in fp32.  The workspace (at least
- * moe_workspace_size(cfg) bytes) holds gamma*Wr in fp32 and the error word. */
+ *   prob_mean [E]     fp32   out (optional, NULL to skip): mean softmax
+ *                            probability of each expert over the T tokens,
+ *                            reduced in the router's epilogue in a fixed order
+ *                            (deterministic); input of moe_router_stats
+ * Logits accumulate exact bf16*bf16 products; each is rounded once to fp32.
+ * The workspace (at least moe_workspace_size(cfg) bytes) holds gamma*Wr in
+ * tensor-core fragment order, the prob_mean partials and the error word. */
 MOE_API moe_status_t moe_route(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
                        const moe_bf16_t* Wr, const float* bias, int32_t* expert_idx, float* gate,
-                       float* r, float* logits, void* ws, size_t ws_bytes, void* stream);
+                       float* r, float* logits, float* prob_mean, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Router load-balance metrics (MoE glossary, "Load Balancing": an auxiliary
+ * loss on the spread of the routing probability across experts), computed on
+ * the device from moe_route's prob_mean and moe_dispatch's counts / offsets:
+ *   stats[0] = E * sum_e f_e * P_e   (Switch-style term, f_e = counts_e/(T*k))
+ *   stats[1] = CV^2 of P_e over experts (population variance / mean^2)
+ *   stats[2] = CV^2 of counts_e over experts
+ *   stats[3] = fraction of the T*k assignments dropped by the capacity limit
+ * stats [4] fp32 device output; asynchronous on `stream`. */
+MOE_API moe_status_t moe_router_stats(const moe_config_t* cfg, const float* prob_mean,
+                                      const int32_t* counts, const int32_t* expert_offsets,
+                                      float* stats, void* stream);
 
 /* Dispatch: histogram, capacity, expert-centric permutation (OmniMoE summary,
  * "Expert-Centric Scheduling"; MoE glossary, "Expert Capacity"), and the
@@ -226,13 +244,14 @@ MOE_API moe_status_t moe_combine(const moe_config_t* cfg, const moe_bf16_t* y, c
 
 /* The whole layer: route -> dispatch -> experts -> combine, on one stream,
  * with no host synchronisation (the kept counts never leave the device).
- *   out [T, d] bf16 out.  expert_idx/gate/r/counts: optional copies of the
- *   routing results (NULL to skip), shapes as in moe_route / moe_dispatch. */
+ *   out [T, d] bf16 out.  expert_idx/gate/r/counts/prob_mean: optional copies
+ *   of the routing results (NULL to skip), shapes as in moe_route /
+ *   moe_dispatch; stats [4]: optional router metrics (moe_router_stats). */
 MOE_API moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
                            const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
                            const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out,
-                           int32_t* expert_idx, float* gate, float* r, int32_t* counts, void* ws,
-                           size_t ws_bytes, void* stream);
+                           int32_t* expert_idx, float* gate, float* r, int32_t* counts,
+                           float* prob_mean, float* stats, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -41,7 +41,7 @@ EXPORTED = ["moe_status_string", "moe_capacity", "moe_max_kept", "moe_workspace_
             "moe_workspace_init", "moe_get_device_error", "moe_route", "moe_dispatch",
             "moe_dispatch_noalloc",
             "moe_experts_fwd", "moe_experts_up", "moe_experts_down", "moe_combine",
-            "moe_layer_fwd"]
+            "moe_layer_fwd", "moe_router_stats"]
 
 
 class MoEError(RuntimeError):
@@ -93,7 +93,9 @@ def _lib():
         lib.moe_get_device_error.restype = ctypes.c_int
         lib.moe_get_device_error.argtypes = [P, SZ, P, ctypes.POINTER(ctypes.c_uint32)]
         lib.moe_route.restype = ctypes.c_int
-        lib.moe_route.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_route.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_router_stats.restype = ctypes.c_int
+        lib.moe_router_stats.argtypes = [cfgp, P, P, P, P, P]
         lib.moe_dispatch.restype = ctypes.c_int
         lib.moe_dispatch.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, SZ, P]
         lib.moe_dispatch_noalloc.restype = ctypes.c_int
@@ -107,7 +109,7 @@ def _lib():
         lib.moe_combine.restype = ctypes.c_int
         lib.moe_combine.argtypes = [cfgp, P, P, P, P]
         lib.moe_layer_fwd.restype = ctypes.c_int
-        lib.moe_layer_fwd.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_layer_fwd.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         _lib_handle = lib
     return _lib_handle
 
@@ -232,7 +234,7 @@ def moe_get_device_error(ws: torch.Tensor, stream=None, raise_on_error: bool = T
 
 
 def moe_route(cfg: MoEConfig, x, gamma, Wr, bias, expert_idx, gate, r, logits,
-              ws: torch.Tensor, stream=None) -> None:
+              ws: torch.Tensor, prob_mean=None, stream=None) -> None:
     T, d, E, k = cfg.T, cfg.d_model, cfg.E, cfg.k
     bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
     st = _lib().moe_route(
@@ -240,8 +242,20 @@ def moe_route(cfg: MoEConfig, x, gamma, Wr, bias, expert_idx, gate, r, logits,
         _ptr(Wr, "Wr", bf, (d, E)), _ptr(bias, "bias", f32, (E,)),
         _ptr(expert_idx, "expert_idx", i32, (T, k)), _ptr(gate, "gate", f32, (T, k)),
         _ptr(r, "r", f32, (T,)), _ptr(logits, "logits", f32, (T, E)),
+        _ptr(prob_mean, "prob_mean", f32, (E,)),
         _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
     _check(st, "moe_route")
+
+
+def moe_router_stats(cfg: MoEConfig, prob_mean, counts, expert_offsets, stats, stream=None) -> None:
+    """stats[4] = {E*sum f_e*P_e, CV^2(P), CV^2(counts), dropped fraction} on the device."""
+    E = cfg.E
+    st = _lib().moe_router_stats(
+        ctypes.byref(cfg.c()), _ptr(prob_mean, "prob_mean", torch.float32, (E,)),
+        _ptr(counts, "counts", torch.int32, (E,)),
+        _ptr(expert_offsets, "expert_offsets", torch.int32, (E + 1,)),
+        _ptr(stats, "stats", torch.float32, (4,)), _stream(stream))
+    _check(st, "moe_router_stats")
 
 
 def moe_dispatch(cfg: MoEConfig, expert_idx, x, gamma, counts, expert_offsets, perm, inv_perm,
@@ -344,7 +358,8 @@ def moe_combine(cfg: MoEConfig, y, inv_perm, out, stream=None) -> None:
 
 
 def moe_layer_fwd(cfg: MoEConfig, x, gamma, Wr, bias, W1, W3, W2, out, ws: torch.Tensor,
-                  expert_idx=None, gate=None, r=None, counts=None, stream=None) -> None:
+                  expert_idx=None, gate=None, r=None, counts=None, prob_mean=None, stats=None,
+                  stream=None) -> None:
     T, d, E, k, F = cfg.T, cfg.d_model, cfg.E, cfg.k, cfg.F
     bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
     st = _lib().moe_layer_fwd(
@@ -353,6 +368,7 @@ def moe_layer_fwd(cfg: MoEConfig, x, gamma, Wr, bias, W1, W3, W2, out, ws: torch
         _ptr(W3, "W3", bf, (d, F)), _ptr(W2, "W2", bf, (F, d)), _ptr(out, "out", bf, (T, d)),
         _ptr(expert_idx, "expert_idx", i32, (T, k)), _ptr(gate, "gate", f32, (T, k)),
         _ptr(r, "r", f32, (T,)), _ptr(counts, "counts", i32, (E,)),
+        _ptr(prob_mean, "prob_mean", f32, (E,)), _ptr(stats, "stats", f32, (4,)),
         _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
     _check(st, "moe_layer_fwd")
 
@@ -366,12 +382,14 @@ class MoELayer:
         self.W1, self.W3, self.W2 = W1, W3, W2
         self.ws = alloc_workspace(cfg, device=gamma.device)
 
-    def forward(self, x, out=None, expert_idx=None, gate=None, r=None, counts=None, stream=None):
+    def forward(self, x, out=None, expert_idx=None, gate=None, r=None, counts=None, prob_mean=None,
+                stats=None, stream=None):
         c = self.cfg
         if out is None:
             out = torch.empty((c.T, c.d_model), dtype=torch.bfloat16, device=x.device)
         moe_layer_fwd(c, x, self.gamma, self.Wr, self.bias, self.W1, self.W3, self.W2, out, self.ws,
-                      expert_idx=expert_idx, gate=gate, r=r, counts=counts, stream=stream)
+                      expert_idx=expert_idx, gate=gate, r=r, counts=counts, prob_mean=prob_mean,
+                      stats=stats, stream=stream)
         return out
 
     __call__ = forward

@@ -36,7 +36,8 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct Layout {
-  size_t err, rw, tile_counts, r, idx, gate, counts, offsets, perm, inv_perm, x_perm, H, y, total;
+  size_t err, ticket, rw, prob_partial, prob_mean, tile_counts, r, idx, gate, counts, offsets, perm,
+      inv_perm, x_perm, H, y, total;
   int64_t max_kept;
   int ldh;
 };
@@ -92,7 +93,10 @@ Layout layout_of(const moe_config_t& c) {
   L.ldh = fmax;
   const size_t mk = static_cast<size_t>(L.max_kept);
   L.err = 0;
+  L.ticket = 4;  // second word of the header
   L.rw = take(static_cast<size_t>(c.d_model) * kRouterPadE * 4);
+  L.prob_partial = take(static_cast<size_t>((c.T + kRouteTok - 1) / kRouteTok) * c.E * 4);
+  L.prob_mean = take(static_cast<size_t>(c.E) * 4);
   L.tile_counts = take(ntiles * c.E * 4);
   L.r = take(static_cast<size_t>(c.T) * 4);
   L.idx = take(tk * 4);
@@ -190,10 +194,18 @@ T* at(void* ws, size_t off) {
 
 moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf16_t* gamma,
                        const moe_bf16_t* Wr, const float* bias, int32_t* idx, float* gate, float* r,
-                       float* logits, uint32_t* err, float* wprime, cudaStream_t s) {
+                       float* logits, float* prob_mean, const Layout& L, void* ws, cudaStream_t s) {
   if (c.T == 0) return MOE_OK;
   RouteArgs a{};
-  a.wprime = wprime;
+  a.wprime = at<float>(ws, L.rw);
+  a.err = at<uint32_t>(ws, L.err);
+  a.prob_mean = prob_mean;
+  a.prob_partial = at<float>(ws, L.prob_partial);
+  a.ticket = at<unsigned>(ws, L.ticket);
+  if (prob_mean != nullptr) {
+    cudaError_t e = cudaMemsetAsync(a.ticket, 0, sizeof(unsigned), s);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
   a.x = reinterpret_cast<const __nv_bfloat16*>(x);
   a.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
   a.Wr = reinterpret_cast<const __nv_bfloat16*>(Wr);
@@ -202,7 +214,6 @@ moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf1
   a.gate = gate;
   a.r = r;
   a.logits = logits;
-  a.err = err;
   a.T = c.T;
   a.d = c.d_model;
   a.E = c.E;
@@ -423,20 +434,22 @@ moe_status_t moe_get_device_error(void* ws, size_t ws_bytes, void* stream, uint3
 
 moe_status_t moe_route(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
                        const moe_bf16_t* Wr, const float* bias, int32_t* expert_idx, float* gate,
-                       float* r, float* logits, void* ws, size_t ws_bytes, void* stream) {
+                       float* r, float* logits, float* prob_mean, void* ws, size_t ws_bytes,
+                       void* stream) {
   moe_status_t st = validate(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;  // no tokens: nothing to do (pointers may be null)
   if (!x || !gamma || !Wr || !expert_idx || !gate || !r) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) ||
-      !aligned(expert_idx, 4) || !aligned(gate, 4) || !aligned(r, 4) || !aligned(logits, 4))
+      !aligned(expert_idx, 4) || !aligned(gate, 4) || !aligned(r, 4) || !aligned(logits, 4) ||
+      !aligned(prob_mean, 4))
     return MOE_ERR_ALIGNMENT;
   int sms;
   if ((st = device_ready(&sms)) != MOE_OK) return st;
   Layout L;
   if ((st = check_ws(*cfg, ws, ws_bytes, &L)) != MOE_OK) return st;
-  return run_route(*cfg, x, gamma, Wr, bias, expert_idx, gate, r, logits, at<uint32_t>(ws, L.err),
-                   at<float>(ws, L.rw), static_cast<cudaStream_t>(stream));
+  return run_route(*cfg, x, gamma, Wr, bias, expert_idx, gate, r, logits, prob_mean, L, ws,
+                   static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_dispatch(const moe_config_t* cfg, const int32_t* expert_idx, const moe_bf16_t* x,
@@ -590,8 +603,8 @@ moe_status_t moe_combine(const moe_config_t* cfg, const moe_bf16_t* y, const int
 moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
                            const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
                            const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out,
-                           int32_t* expert_idx, float* gate, float* r, int32_t* counts, void* ws,
-                           size_t ws_bytes, void* stream) {
+                           int32_t* expert_idx, float* gate, float* r, int32_t* counts,
+                           float* prob_mean, float* stats, void* ws, size_t ws_bytes, void* stream) {
   moe_status_t st = validate(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) {  // no tokens: only the optional counts are written (zeros)
@@ -601,6 +614,7 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x, const m
     if ((st = device_ready(&sms)) != MOE_OK) return st;
     return cuda_status(cudaMemsetAsync(counts, 0, cfg->E * sizeof(int32_t), static_cast<cudaStream_t>(stream)));
   }
+  if (!aligned(prob_mean, 4) || !aligned(stats, 4)) return MOE_ERR_ALIGNMENT;
   if (!x || !gamma || !Wr || !W1 || !W3 || !W2 || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) ||
       !aligned(W1, 16) || !aligned(W3, 16) || !aligned(W2, 16) || !aligned(out, 16) ||
@@ -621,14 +635,30 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x, const m
   int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
   moe_bf16_t* x_perm = at<moe_bf16_t>(ws, L.x_perm);
   moe_bf16_t* y = at<moe_bf16_t>(ws, L.y);
-  if ((st = run_route(c, x, gamma, Wr, bias, idx_, gate_, r_, nullptr, at<uint32_t>(ws, L.err),
-                      at<float>(ws, L.rw), s)) != MOE_OK)
-    return st;
+  float* pm = prob_mean ? prob_mean : (stats ? at<float>(ws, L.prob_mean) : nullptr);
+  if ((st = run_route(c, x, gamma, Wr, bias, idx_, gate_, r_, nullptr, pm, L, ws, s)) != MOE_OK) return st;
   if ((st = run_dispatch(c, L, ws, idx_, x, gamma, counts_, offsets, perm, inv_perm, x_perm, sms, s)) != MOE_OK)
     return st;
   if ((st = run_experts(c, L, ws, x_perm, r_, gate_, perm, offsets, W1, W3, W2, y, sms, s)) != MOE_OK)
     return st;
-  return run_combine(c, y, inv_perm, out, sms, s);
+  if ((st = run_combine(c, y, inv_perm, out, sms, s)) != MOE_OK) return st;
+  if (stats != nullptr)
+    return cuda_status(launch_router_stats(pm, counts_, offsets, stats, c.T, c.E, c.k, s));
+  return MOE_OK;
+}
+
+moe_status_t moe_router_stats(const moe_config_t* cfg, const float* prob_mean, const int32_t* counts,
+                              const int32_t* expert_offsets, float* stats, void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!prob_mean || !counts || !expert_offsets || !stats) return MOE_ERR_INVALID_ARG;
+  if (!aligned(prob_mean, 4) || !aligned(counts, 4) || !aligned(expert_offsets, 4) || !aligned(stats, 4))
+    return MOE_ERR_ALIGNMENT;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  return cuda_status(launch_router_stats(prob_mean, counts, expert_offsets, stats, cfg->T, cfg->E, cfg->k,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

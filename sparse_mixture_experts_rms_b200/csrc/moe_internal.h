@@ -34,6 +34,9 @@ struct RouteArgs {
   float* logits;      // may be null
   uint32_t* err;      // device error word, may be null
   float* wprime;      // [d, EP] fp32 scratch: gamma * Wr, zero-padded
+  float* prob_mean;     // [E] out: mean softmax probability per expert, may be null
+  float* prob_partial;  // scratch [gridDim, E]: per-CTA probability sums
+  unsigned* ticket;     // scratch: CTAs done (zeroed before the launch)
   int T, d, E, k;
   float eps;
   int renormalize;
@@ -83,6 +86,10 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA,
                                 const CUtensorMap& mapB0, const CUtensorMap& mapB1, int grid,
                                 cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);
+// stats[4] = {E*sum_e f_e*P_e, CV^2(P), CV^2(counts), dropped fraction}
+cudaError_t launch_router_stats(const float* prob_mean, const int32_t* counts, const int32_t* offsets,
+                                float* stats, int T, int E, int k, cudaStream_t s);
+constexpr int kRouteTok = 64;  // tokens per router CTA
 
 // One-time per-device kernel attributes (dynamic shared memory opt-in).
 cudaError_t prepare_grouped_gemm();

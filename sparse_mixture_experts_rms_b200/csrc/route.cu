@@ -32,7 +32,7 @@
 namespace moe {
 namespace {
 
-constexpr int kTok = 64;                       // tokens per CTA
+constexpr int kTok = kRouteTok;                // tokens per CTA
 constexpr int kWarps = kTok / 16;              // a warp owns 16 tokens (MMA rows)
 constexpr int kThreads = kWarps * 32;
 constexpr int kChunk = 64;                     // elements of d per stage (4 k-steps)
@@ -85,6 +85,10 @@ __global__ void router_weight_kernel(const RouteArgs a, int nt_count) {
     out[i] = make_uint2(h16[0] | (h16[1] << 16), h16[2] | (h16[3] << 16));
   }
 }
+
+template <int EP>
+__device__ __forceinline__ void route_token(const RouteArgs& a, float* lg, float rtok, int t,
+                                            bool keep_probs);
 
 template <int EP>
 __global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__ CUtensorMap xmap,
@@ -224,15 +228,45 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__
     rr[row_g8] = static_cast<float>(r_g8);
   }
   __syncthreads();
-  if (tid >= kTok) return;
   const int t = t0 + tid;
-  if (t >= a.T) return;
+  if (tid < kTok && t < a.T) route_token<EP>(a, lg + tid * EP, rr[tid], t, a.prob_mean != nullptr);
+  else if (tid < kTok && a.prob_mean != nullptr)
+    for (int e = 0; e < EP; ++e) lg[tid * EP + e] = 0.f;  // rows past T add nothing
+  if (a.prob_mean == nullptr) return;
 
+  // Router metric in the epilogue: this CTA's probability sums, then the last
+  // CTA to finish sums every CTA's partials in CTA order (deterministic).
+  __shared__ int is_last;
+  __syncthreads();
+  if (tid < a.E) {
+    float sum = 0.f;
+    for (int i = 0; i < kTok; ++i) sum += lg[i * EP + tid];
+    a.prob_partial[static_cast<size_t>(blockIdx.x) * a.E + tid] = sum;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) is_last = atomicAdd(a.ticket, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  if (tid < a.E) {
+    double sum = 0.0;
+    for (unsigned c = 0; c < gridDim.x; ++c)
+      sum += static_cast<double>(__ldcg(a.prob_partial + static_cast<size_t>(c) * a.E + tid));
+    a.prob_mean[tid] = static_cast<float>(sum / static_cast<double>(a.T));
+  }
+}
+
+// Softmax and top-k of one token from its fp32 logits (row of `lg`).  With
+// `keep_probs`, the row is overwritten with the token's softmax probabilities.
+template <int EP>
+__device__ __forceinline__ void route_token(const RouteArgs& a, float* lg, float rtok, int t,
+                                            bool keep_probs) {
   float l[EP];
   float m = -INFINITY;
 #pragma unroll
   for (int e = 0; e < EP; ++e) {
-    l[e] = lg[tid * EP + e];
+    l[e] = lg[e];
     if (e < a.E) m = fmaxf(m, l[e]);
   }
   float sum = 0.f;
@@ -246,7 +280,11 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__
     for (int e = 0; e < EP; ++e)
       if (e < a.E) a.logits[static_cast<size_t>(t) * a.E + e] = l[e];
   }
-  a.r[t] = rr[tid];
+  a.r[t] = rtok;
+  if (keep_probs) {
+#pragma unroll
+    for (int e = 0; e < EP; ++e) lg[e] = e < a.E ? expf(l[e] - m) * inv_s : 0.f;
+  }
 
   // top-k: k rounds of a first-maximum scan (strict '>' keeps the lower index on ties)
   uint64_t used = 0;
@@ -294,7 +332,48 @@ cudaError_t launch_route_t(const RouteArgs& a, const CUtensorMap& xmap, cudaStre
   return cudaGetLastError();
 }
 
+// Load-balance metrics from the router's prob_mean and the dispatch counts:
+// stats = {E * sum_e f_e * P_e, CV^2(P), CV^2(counts), dropped fraction},
+// f_e = counts_e / (T*k), CV^2 with the population variance, in fp64.
+__global__ void router_stats_kernel(const float* P, const int32_t* counts, const int32_t* offsets,
+                                    float* stats, int T, int E, int k) {
+  __shared__ double sp[kMaxExperts], sc[kMaxExperts];
+  const int e = threadIdx.x;
+  if (e < E) {
+    sp[e] = static_cast<double>(P[e]);
+    sc[e] = static_cast<double>(counts[e]);
+  }
+  __syncthreads();
+  if (e != 0) return;
+  const double tk = static_cast<double>(T) * k;
+  double aux = 0.0, mp = 0.0, mc = 0.0;
+  for (int i = 0; i < E; ++i) {
+    aux += (sc[i] / tk) * sp[i];
+    mp += sp[i];
+    mc += sc[i];
+  }
+  mp /= E;
+  mc /= E;
+  double vp = 0.0, vc = 0.0;
+  for (int i = 0; i < E; ++i) {
+    vp += (sp[i] - mp) * (sp[i] - mp);
+    vc += (sc[i] - mc) * (sc[i] - mc);
+  }
+  vp /= E;
+  vc /= E;
+  stats[0] = static_cast<float>(E * aux);
+  stats[1] = static_cast<float>(mp != 0.0 ? vp / (mp * mp) : 0.0);
+  stats[2] = static_cast<float>(mc != 0.0 ? vc / (mc * mc) : 0.0);
+  stats[3] = static_cast<float>(1.0 - static_cast<double>(offsets[E]) / tk);
+}
+
 }  // namespace
+
+cudaError_t launch_router_stats(const float* prob_mean, const int32_t* counts, const int32_t* offsets,
+                                float* stats, int T, int E, int k, cudaStream_t s) {
+  router_stats_kernel<<<1, kMaxExperts, 0, s>>>(prob_mean, counts, offsets, stats, T, E, k);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;

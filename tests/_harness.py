@@ -101,13 +101,17 @@ def run_staged(d: Dev) -> Dict[str, torch.Tensor]:
         "x_perm": torch.zeros((mk, dm), dtype=torch.bfloat16, device="cuda"),
         "y": torch.zeros((mk, dm), dtype=torch.bfloat16, device="cuda"),
         "out": torch.empty((T, dm), dtype=torch.bfloat16, device="cuda"),
+        "prob_mean": torch.empty((E,), dtype=torch.float32, device="cuda"),
+        "stats": torch.empty((4,), dtype=torch.float32, device="cuda"),
     }
-    moe.moe_route(c, d.x, d.gamma, d.Wr, d.bias, o["idx"], o["gate"], o["r"], o["logits"], d.ws)
+    moe.moe_route(c, d.x, d.gamma, d.Wr, d.bias, o["idx"], o["gate"], o["r"], o["logits"], d.ws,
+                  prob_mean=o["prob_mean"])
     moe.moe_dispatch(c, o["idx"], d.x, d.gamma, o["counts"], o["offsets"], o["perm"], o["inv_perm"],
                      o["x_perm"], d.ws)
     moe.moe_experts_fwd(c, o["x_perm"], o["r"], o["gate"], o["perm"], o["offsets"], d.W1, d.W3, d.W2,
                         o["y"], d.ws)
     moe.moe_combine(c, o["y"], o["inv_perm"], o["out"])
+    moe.moe_router_stats(c, o["prob_mean"], o["counts"], o["offsets"], o["stats"])
     torch.cuda.synchronize()
     return o
 
@@ -120,9 +124,11 @@ def run_fused(d: Dev) -> Dict[str, torch.Tensor]:
         "r": torch.empty((c.T,), dtype=torch.float32, device="cuda"),
         "counts": torch.empty((c.E,), dtype=torch.int32, device="cuda"),
         "out": torch.empty((c.T, c.d_model), dtype=torch.bfloat16, device="cuda"),
+        "stats": torch.empty((4,), dtype=torch.float32, device="cuda"),
     }
     moe.moe_layer_fwd(c, d.x, d.gamma, d.Wr, d.bias, d.W1, d.W3, d.W2, o["out"], d.ws,
-                      expert_idx=o["idx"], gate=o["gate"], r=o["r"], counts=o["counts"])
+                      expert_idx=o["idx"], gate=o["gate"], r=o["r"], counts=o["counts"],
+                      stats=o["stats"])
     torch.cuda.synchronize()
     return o
 
@@ -144,6 +150,19 @@ def check_route(p: Problem, R: Dict[str, np.ndarray], g_idx, g_gate, g_r, g_logi
     assert bad.size == 0, f"{bad.size} tokens routed differently (margin >= {TIE_MARGIN}): {bad[:10]}"
     np.testing.assert_allclose(g_gate[ok_tok], R["gate"][ok_tok], rtol=0, atol=GATE_ATOL)
     return np.nonzero(~ok_tok)[0]
+
+
+STATS_RTOL = 1e-5         # router metrics (fp32 probabilities, fp64 reductions)
+
+
+def check_stats(R: Dict[str, np.ndarray], counts: np.ndarray, n_kept: int, k: int,
+                g_prob_mean: Optional[np.ndarray], g_stats: np.ndarray):
+    """Router metrics against the oracle on the same routing (the GPU's counts)."""
+    S = O.router_stats(R["logits"], counts, n_kept, k)
+    if g_prob_mean is not None:
+        np.testing.assert_allclose(g_prob_mean, S["prob_mean"], rtol=STATS_RTOL, atol=1e-7)
+    exp = np.array([S["aux_loss"], S["cv2_prob"], S["cv2_load"], S["dropped_frac"]])
+    np.testing.assert_allclose(g_stats, exp, rtol=STATS_RTOL, atol=1e-6)
 
 
 def check_dispatch(g_idx: np.ndarray, E: int, C: Optional[int], o: Dict[str, np.ndarray]):

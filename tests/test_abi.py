@@ -98,7 +98,7 @@ def test_too_many_experts_unsupported(lib):
 def _call_layer(lib, cfg, ptrs, ws_ptr, ws_bytes):
     P = ctypes.c_void_p
     return lib.moe_layer_fwd(ctypes.byref(cfg.c()), *[P(p) for p in ptrs], P(0), P(0), P(0), P(0),
-                             P(ws_ptr), ws_bytes, P(0))
+                             P(0), P(0), P(ws_ptr), ws_bytes, P(0))
 
 
 def test_layer_argument_errors_before_any_device_work(lib):

@@ -78,10 +78,12 @@ def _full_check(p: H.Problem, renormalize=False, fused_too=True):
         H.check_rows(H.bf16_dev_to_f64(o["y"][:n]), exp_y, "y")
     out_ref = O.combine(y, gate_o, D["kept"])
     H.check_rows(H.bf16_dev_to_f64(o["out"]), out_ref, "out")
+    H.check_stats(R, g["counts"], n, p.w.k, g["prob_mean"], g["stats"])
     if fused_too:
         f = H.run_fused(d)
         assert torch.equal(f["out"], o["out"]), "fused layer differs from the staged calls"
         assert torch.equal(f["idx"], o["idx"]) and torch.equal(f["counts"], o["counts"])
+        assert torch.equal(f["stats"], o["stats"]), "fused router metrics differ from the staged ones"
         assert moe.moe_get_device_error(d.ws, raise_on_error=False) == 0
     return o, R, D
 
@@ -125,6 +127,7 @@ def test_layer_full_size_sampled(name):
     C = O.capacity(w.T, w.k, w.E, p.cf32)
     D = O.dispatch(g_idx, w.E, C)
     assert np.array_equal(o["counts"].cpu().numpy(), D["counts"])
+    H.check_stats(R, D["counts"], D["n_kept"], w.k, None, o["stats"].cpu().numpy())
     toks = mw.sample_tokens(w, 192)
     gate_o = O.gates(R["logits"], g_idx)
     ref = O.moe_layer_tokens(p.x[toks], toks, p.gamma, p.W1, p.W3, p.W2, p.widths,
