@@ -39,6 +39,25 @@ import moe_workloads as mw  # noqa: E402
 METRIC = "MoE layer fwd tokens/s & TFLOP/s, % of B200 bf16 peak / HBM roofline"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) per launch of the up GEMM on the default
+# workload, from one ncu capture at full size (dram__bytes_read.sum +
+# dram__bytes_write.sum, a 1-pass metric; summary and command in
+# profiles/grouped_gemm_traffic_mixtral_T16384.md).  Reported only while the
+# kernel sources still hash to `digest`; after any change it is null until
+# re-measured.
+MEASURED_TRAFFIC = {"workload": "mixtral", "T": 16384, "digest": "b1e688244d6e7377",
+                    "bytes": 4.92e9 + 0.931e9}   # dram read + write of the up launch
+
+
+def kernel_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("grouped_gemm.cu", "ptx.cuh"):
+        with open(os.path.join(ROOT, "sparse_mixture_experts_rms_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 KERNELS_PER_STEP = 8  # router weights, route, dispatch count/scatter/permute, GEMM up, GEMM down, combine
 
 
@@ -394,7 +413,13 @@ def run_ours(args, rank, world, local):
             "kernel": "grouped_gemm_kernel (up: x_perm x [W1|W3], SwiGLU epilogue)",
             "bound": "tensor", "achieved": achieved_up, "peak": peaks["bf16_tflops_sustained"],
             "unit": "TFLOP/s", "frac": achieved_up / peaks["bf16_tflops_sustained"],
-            "traffic": None,
+            "traffic": (MEASURED_TRAFFIC["bytes"]
+                        if (MEASURED_TRAFFIC["digest"] == kernel_digest()
+                            and w.name == MEASURED_TRAFFIC["workload"] and w.T == MEASURED_TRAFFIC["T"])
+                        else None),
+            # W1|W3 of the experts that received rows + x_perm read + H written
+            "traffic_algorithmic": (float(sum(2 * d * f * 2 for f, n in zip(widths, kept) if n > 0))
+                                    + n_kept * d * 2.0 + nf * 2.0),
             "peak_note": f"{peaks['source']} sustained cuBLAS bf16 (kernel timed inside long steps)",
             "flops_per_launch": fl_up,
         },

@@ -28,10 +28,11 @@
 // MMA commit arrives on both CTAs' "empty" and "accumulator full" barriers;
 // both CTAs' epilogues arrive on the leader's "accumulator empty" barrier.
 //
-// Tiles: expert e contributes ceil(n_e/256) * (N_e/BN) pair tiles, enumerated
-// M-fastest on the device from the kept-row offsets (no host sync), so pairs
-// running together share a weight column block in L2.  Persistent pairs
-// stride through the list.
+// Tiles: expert e contributes ceil(n_e/256) * (N_e/BN) pair tiles, listed on
+// the device from the kept-row offsets (no host sync) in raster groups of
+// M tiles whose A rows fit a 48 MB L2 budget (M fastest inside a group), so
+// pairs running together share A rows and weight column blocks in L2.
+// Persistent pairs stride through the list.
 //
 // Warp roles (192 threads per CTA): warp 0 = TMA producer, warp 1 = MMA issuer
 // (leader only) and TMEM owner, warps 2..5 = epilogue (TMEM -> registers ->
@@ -57,6 +58,7 @@ constexpr int kTmemCols = 512;
 constexpr int kAccCols = 256;                 // columns per accumulator buffer
 constexpr int kAtomBytes = BK * 64 * 2;       // one 64(n) x 64(k) B box: 8 KB
 constexpr int kEpiWarps = 4;
+constexpr long long kL2GroupBudget = 48ll << 20;  // A bytes of one raster group
 
 struct __align__(8) GemmShared {
   uint64_t full[kStages];    // leader: both CTAs' loads of a stage landed
@@ -69,6 +71,8 @@ struct __align__(8) GemmShared {
   int total_tiles;
   int tile_start[kMaxExperts + 1];
   int m_tiles[kMaxExperts];
+  int n_tiles[kMaxExperts];
+  int group_m[kMaxExperts];  // m tiles per raster group (see decode_tile)
   int seg[kMaxExperts + 1];
 };
 
@@ -78,12 +82,20 @@ struct TileCoord {
   int e, nt, mt;
 };
 
+// Tiles of expert e are rastered in groups of group_m[e] M tiles: inside a
+// group, M is fastest and N next, so the pairs running together share the
+// group's A rows (kept in L2) and a few B column blocks.  group_m is chosen so
+// that a group's A rows fit an L2 budget; when the whole expert fits, the
+// order is plain M-fastest.
 __device__ __forceinline__ TileCoord decode_tile(const GemmShared& sh, int E, int tile) {
   int e = 0;
   while (e + 1 < E && tile >= sh.tile_start[e + 1]) ++e;
   const int local = tile - sh.tile_start[e];
-  const int mt_count = sh.m_tiles[e];
-  return TileCoord{e, local / mt_count, local % mt_count};
+  const int mt_count = sh.m_tiles[e], nt_count = sh.n_tiles[e], gm = sh.group_m[e];
+  const int g = local / (gm * nt_count);
+  const int rem = local - g * gm * nt_count;
+  const int gm_g = min(gm, mt_count - g * gm);  // the last group may be short
+  return TileCoord{e, rem / gm_g, g * gm + rem % gm_g};
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -136,7 +148,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int ncols = a.up ? (a.ffn.off[tid + 1] - a.ffn.off[tid]) : a.d;
     const int nt = a.up ? ncols / kBlockN : ncols / a.bn;
     const int mt = (rows + BM - 1) / BM;
+    // A bytes of one M tile: 256 rows x the reduction length (d up, f_e down)
+    const long long a_rows_bytes =
+        static_cast<long long>(BM) * (a.up ? a.d : (a.ffn.off[tid + 1] - a.ffn.off[tid])) * 2;
+    int gm = static_cast<int>(kL2GroupBudget / (a_rows_bytes > 0 ? a_rows_bytes : 1));
+    gm = gm < 1 ? 1 : gm;
     sh.m_tiles[tid] = mt > 0 ? mt : 1;
+    sh.n_tiles[tid] = nt > 0 ? nt : 1;
+    sh.group_m[tid] = gm < sh.m_tiles[tid] ? gm : sh.m_tiles[tid];
     sh.tile_start[tid + 1] = mt * nt;  // count for now
   }
   __syncthreads();
