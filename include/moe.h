@@ -253,6 +253,76 @@ MOE_API moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x,
                            int32_t* expert_idx, float* gate, float* r, int32_t* counts,
                            float* prob_mean, float* stats, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- training: forward that saves what the backward reads, and the backward
+ *
+ * CODA sparse-MoE thread (digg.com): the RMSNorm backward is fused into the
+ * backward of the linears that read the normalised token (the router and the
+ * first expert linear), which needs each token's statistic r; r is therefore
+ * saved by the forward and read by the backward's epilogues.  The gradient is
+ * the derivative of the forward above (routing ids and capacity drops carry
+ * none; the router receives gradient through the gates).
+ *
+ * The training workspace (size from moe_train_workspace_size) holds the device
+ * error word (so moe_get_device_error works on it), r, the routing, the fp32
+ * logits, the expert-centric permutation with every expert's row segment
+ * padded to a multiple of 64 rows (padding rows are zero), x_perm, the
+ * pre-activations U = r*(x*gamma)W1_e and V = r*(x*gamma)W3_e, H, and the
+ * ungated expert outputs, plus the backward's scratch.  One workspace serves
+ * one forward/backward pair: moe_layer_bwd reads what the last
+ * moe_layer_fwd_train on the same workspace saved, with the same cfg and
+ * inputs.  Limits beyond the forward's: none. */
+
+/* Bytes of training workspace for `cfg` (0 if cfg is invalid). */
+MOE_API size_t moe_train_workspace_size(const moe_config_t* cfg);
+
+/* The layer forward of moe_layer_fwd (same arguments, same out to the bit),
+ * saving the backward's inputs in the training workspace `tws`. */
+MOE_API moe_status_t moe_layer_fwd_train(const moe_config_t* cfg, const moe_bf16_t* x,
+                                         const moe_bf16_t* gamma, const moe_bf16_t* Wr,
+                                         const float* bias, const moe_bf16_t* W1, const moe_bf16_t* W3,
+                                         const moe_bf16_t* W2, moe_bf16_t* out, void* tws,
+                                         size_t tws_bytes, void* stream);
+
+/* Gradients of L = <dout, out> for the forward last run on `tws`:
+ *   dout   [T, d] bf16 in
+ *   dx     [T, d] fp32 out        dgamma [d]    fp32 out
+ *   dWr    [d, E] fp32 out        dbias  [E]    fp32 out (written even when
+ *                                                the forward had no bias)
+ *   dW1, dW3 [d, F] fp32 out      dW2    [F, d] fp32 out
+ * Every output is overwritten (experts that received no rows get zero weight
+ * gradients).  x, gamma, Wr, bias, W1, W3, W2 are the forward's inputs.
+ * Pointers: 16-byte aligned except bias/dbias/dgamma (4).  Asynchronous on
+ * `stream`; errors as for moe_layer_fwd. */
+MOE_API moe_status_t moe_layer_bwd(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
+                                   const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
+                                   const moe_bf16_t* W3, const moe_bf16_t* W2, const moe_bf16_t* dout,
+                                   float* dx, float* dgamma, float* dWr, float* dbias, float* dW1,
+                                   float* dW3, float* dW2, void* tws, size_t tws_bytes, void* stream);
+
+/* Saved tensors of the training workspace, for inspection (device pointers
+ * into `tws`, valid while it lives; NULL and MOE_ERR_INVALID_ARG for an
+ * unknown id).  Rows of the permuted tensors: moe_train_rows(cfg). */
+typedef enum {
+  MOE_SAVED_R = 0,        /* [T] fp32                                        */
+  MOE_SAVED_IDX = 1,      /* [T, k] int32                                    */
+  MOE_SAVED_GATE = 2,     /* [T, k] fp32                                     */
+  MOE_SAVED_LOGITS = 3,   /* [T, E] fp32                                     */
+  MOE_SAVED_OFFSETS = 4,  /* [E+1] int32, padded row segments                */
+  MOE_SAVED_PERM = 5,     /* [rows] int32, -1 at padding                     */
+  MOE_SAVED_INV_PERM = 6, /* [T*k] int32, -1 when dropped                    */
+  MOE_SAVED_U = 7,        /* [rows, f_max] bf16                              */
+  MOE_SAVED_V = 8,        /* [rows, f_max] bf16                              */
+  MOE_SAVED_H = 9,        /* [rows, f_max] bf16                              */
+  MOE_SAVED_Y = 10,       /* [rows, d] bf16, ungated expert outputs          */
+  MOE_SAVED_DGATE = 11,   /* [T*k] fp32 (after moe_layer_bwd; kept slots)    */
+  MOE_SAVED_DR = 12,      /* [T] fp32 dL/dr (after moe_layer_bwd)            */
+  MOE_SAVED_COUNTS = 13   /* [E] int32 routed assignments per expert         */
+} moe_saved_t;
+MOE_API moe_status_t moe_train_saved(const moe_config_t* cfg, void* tws, size_t tws_bytes,
+                                     int32_t which, void** ptr);
+/* Rows of the padded permuted buffers: max kept + E * 63. */
+MOE_API int64_t moe_train_rows(const moe_config_t* cfg);
+
 #ifdef __cplusplus
 }
 #endif

@@ -41,7 +41,12 @@ EXPORTED = ["moe_status_string", "moe_capacity", "moe_max_kept", "moe_workspace_
             "moe_workspace_init", "moe_get_device_error", "moe_route", "moe_dispatch",
             "moe_dispatch_noalloc",
             "moe_experts_fwd", "moe_experts_up", "moe_experts_down", "moe_combine",
-            "moe_layer_fwd", "moe_router_stats"]
+            "moe_layer_fwd", "moe_router_stats", "moe_train_workspace_size", "moe_train_rows",
+            "moe_train_saved", "moe_layer_fwd_train", "moe_layer_bwd"]
+
+# ids of moe_train_saved
+MOE_SAVED = {"r": 0, "idx": 1, "gate": 2, "logits": 3, "offsets": 4, "perm": 5, "inv_perm": 6,
+             "U": 7, "V": 8, "H": 9, "y": 10, "dgate": 11, "dr": 12, "counts": 13}
 
 
 class MoEError(RuntimeError):
@@ -110,6 +115,16 @@ def _lib():
         lib.moe_combine.argtypes = [cfgp, P, P, P, P]
         lib.moe_layer_fwd.restype = ctypes.c_int
         lib.moe_layer_fwd.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_train_workspace_size.restype = SZ
+        lib.moe_train_workspace_size.argtypes = [cfgp]
+        lib.moe_train_rows.restype = ctypes.c_int64
+        lib.moe_train_rows.argtypes = [cfgp]
+        lib.moe_train_saved.restype = ctypes.c_int
+        lib.moe_train_saved.argtypes = [cfgp, P, SZ, ctypes.c_int32, ctypes.POINTER(ctypes.c_void_p)]
+        lib.moe_layer_fwd_train.restype = ctypes.c_int
+        lib.moe_layer_fwd_train.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_layer_bwd.restype = ctypes.c_int
+        lib.moe_layer_bwd.argtypes = [cfgp] + [P] * 15 + [P, SZ, P]
         _lib_handle = lib
     return _lib_handle
 
@@ -371,6 +386,80 @@ def moe_layer_fwd(cfg: MoEConfig, x, gamma, Wr, bias, W1, W3, W2, out, ws: torch
         _ptr(prob_mean, "prob_mean", f32, (E,)), _ptr(stats, "stats", f32, (4,)),
         _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
     _check(st, "moe_layer_fwd")
+
+
+# ------------------------------------------------------------------ training
+def moe_train_workspace_size(cfg: MoEConfig) -> int:
+    return int(_lib().moe_train_workspace_size(ctypes.byref(cfg.c())))
+
+
+def moe_train_rows(cfg: MoEConfig) -> int:
+    return int(_lib().moe_train_rows(ctypes.byref(cfg.c())))
+
+
+def alloc_train_workspace(cfg: MoEConfig, device=None, stream=None) -> torch.Tensor:
+    """A training workspace of ``moe_train_workspace_size(cfg)`` bytes (torch-owned)."""
+    n = moe_train_workspace_size(cfg)
+    if n == 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_train_workspace_size")
+    tws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    moe_workspace_init(tws, stream)
+    return tws
+
+
+def moe_train_saved(cfg: MoEConfig, tws: torch.Tensor, name: str) -> int:
+    """Device address of a saved tensor inside the training workspace."""
+    out = ctypes.c_void_p(0)
+    st = _lib().moe_train_saved(ctypes.byref(cfg.c()), _ptr(tws, "tws", torch.uint8), tws.numel(),
+                                MOE_SAVED[name], ctypes.byref(out))
+    _check(st, "moe_train_saved")
+    return int(out.value)
+
+
+def train_saved_view(cfg: MoEConfig, tws: torch.Tensor, name: str) -> torch.Tensor:
+    """A view of a saved tensor (shares the workspace's memory)."""
+    T, d, E, k = cfg.T, cfg.d_model, cfg.E, cfg.k
+    rows = moe_train_rows(cfg)
+    fmax = max(b - a for a, b in zip(cfg.ffn_offsets[:-1], cfg.ffn_offsets[1:]))
+    spec = {"r": (torch.float32, (T,)), "idx": (torch.int32, (T, k)), "gate": (torch.float32, (T, k)),
+            "logits": (torch.float32, (T, E)), "offsets": (torch.int32, (E + 1,)),
+            "perm": (torch.int32, (rows,)), "inv_perm": (torch.int32, (T * k,)),
+            "U": (torch.bfloat16, (rows, fmax)), "V": (torch.bfloat16, (rows, fmax)),
+            "H": (torch.bfloat16, (rows, fmax)), "y": (torch.bfloat16, (rows, d)),
+            "dgate": (torch.float32, (T * k,)), "dr": (torch.float32, (T,)),
+            "counts": (torch.int32, (E,))}[name]
+    dtype, shape = spec
+    off = moe_train_saved(cfg, tws, name) - tws.data_ptr()
+    n = 1
+    for v in shape:
+        n *= v
+    return tws[off:off + n * torch.empty(0, dtype=dtype).element_size()].view(dtype).view(shape)
+
+
+def moe_layer_fwd_train(cfg: MoEConfig, x, gamma, Wr, bias, W1, W3, W2, out, tws: torch.Tensor,
+                        stream=None) -> None:
+    T, d, E, F = cfg.T, cfg.d_model, cfg.E, cfg.F
+    bf, f32 = torch.bfloat16, torch.float32
+    st = _lib().moe_layer_fwd_train(
+        ctypes.byref(cfg.c()), _ptr(x, "x", bf, (T, d)), _ptr(gamma, "gamma", bf, (d,)),
+        _ptr(Wr, "Wr", bf, (d, E)), _ptr(bias, "bias", f32, (E,)), _ptr(W1, "W1", bf, (d, F)),
+        _ptr(W3, "W3", bf, (d, F)), _ptr(W2, "W2", bf, (F, d)), _ptr(out, "out", bf, (T, d)),
+        _ptr(tws, "tws", torch.uint8), tws.numel(), _stream(stream))
+    _check(st, "moe_layer_fwd_train")
+
+
+def moe_layer_bwd(cfg: MoEConfig, x, gamma, Wr, bias, W1, W3, W2, dout, dx, dgamma, dWr, dbias,
+                  dW1, dW3, dW2, tws: torch.Tensor, stream=None) -> None:
+    T, d, E, F = cfg.T, cfg.d_model, cfg.E, cfg.F
+    bf, f32 = torch.bfloat16, torch.float32
+    st = _lib().moe_layer_bwd(
+        ctypes.byref(cfg.c()), _ptr(x, "x", bf, (T, d)), _ptr(gamma, "gamma", bf, (d,)),
+        _ptr(Wr, "Wr", bf, (d, E)), _ptr(bias, "bias", f32, (E,)), _ptr(W1, "W1", bf, (d, F)),
+        _ptr(W3, "W3", bf, (d, F)), _ptr(W2, "W2", bf, (F, d)), _ptr(dout, "dout", bf, (T, d)),
+        _ptr(dx, "dx", f32, (T, d)), _ptr(dgamma, "dgamma", f32, (d,)), _ptr(dWr, "dWr", f32, (d, E)),
+        _ptr(dbias, "dbias", f32, (E,)), _ptr(dW1, "dW1", f32, (d, F)), _ptr(dW3, "dW3", f32, (d, F)),
+        _ptr(dW2, "dW2", f32, (F, d)), _ptr(tws, "tws", torch.uint8), tws.numel(), _stream(stream))
+    _check(st, "moe_layer_bwd")
 
 
 class MoELayer:

@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libmoe_b200.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 
-SOURCES = ["moe_api.cu", "route.cu", "dispatch.cu", "grouped_gemm.cu", "combine.cu"]
+SOURCES = ["moe_api.cu", "route.cu", "dispatch.cu", "grouped_gemm.cu", "combine.cu", "backward.cu"]
 HEADERS = ["moe_internal.h", "ptx.cuh"]
 
 NVCC_FLAGS = [

@@ -55,7 +55,8 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_count_kernel(const Disp
 __global__ void __launch_bounds__(kDispThreads) dispatch_scatter_kernel(const DispatchArgs a,
                                                                         int ntiles) {
   __shared__ int before[kMaxExperts];   // assignments to e in tiles < this one
-  __shared__ int offs[kMaxExperts + 1];  // kept-row offsets
+  __shared__ int offs[kMaxExperts + 1];  // row-segment offsets (kept rows + padding)
+  __shared__ int kept[kMaxExperts];      // kept rows per expert
   __shared__ int run[kMaxExperts];       // running count inside this tile
   __shared__ int wcnt[kDispWarps][kMaxExperts];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -71,7 +72,9 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_scatter_kernel(const Di
     }
     before[tid] = b;
     run[tid] = 0;
-    offs[tid + 1] = (cap < 0) ? tot : min(tot, cap);
+    const int align = a.row_align > 1 ? a.row_align : 1;
+    kept[tid] = (cap < 0) ? tot : min(tot, cap);
+    offs[tid + 1] = (kept[tid] + align - 1) / align * align;
     if (blockIdx.x == 0) a.counts[tid] = tot;
   }
   for (int i = tid; i < kDispWarps * kMaxExperts; i += kDispThreads) (&wcnt[0][0])[i] = 0;
@@ -82,8 +85,13 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_scatter_kernel(const Di
     if (offs[E] > a.max_kept) atomicOr(a.err, MOE_DEVERR_TILE_TABLE);
   }
   __syncthreads();
-  if (blockIdx.x == 0)
+  if (blockIdx.x == 0) {
     for (int e = tid; e <= E; e += kDispThreads) a.offsets[e] = offs[e];
+    // padding rows of the training layout (fewer than row_align per expert)
+    for (int e = 0; e < E; ++e)
+      for (int i = offs[e] + kept[e] + tid; i < offs[e + 1] && i < a.max_kept; i += kDispThreads)
+        a.perm[i] = -1;
+  }
 
   const int n = a.T * a.k;
   const int base = blockIdx.x * kDispatchTile;
@@ -122,7 +130,8 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_scatter_kernel(const Di
   }
 }
 
-// x_perm[p] = bf16(x[perm[p]/k] * gamma) for p < offsets[E].
+// x_perm[p] = bf16(x[perm[p]/k] * gamma) for p < offsets[E]; zero rows where
+// perm[p] = -1 (padding).
 __global__ void __launch_bounds__(256) permute_rows_kernel(const DispatchArgs a) {
   const int n_kept = min(a.offsets[a.E], a.max_kept);
   const int lane = threadIdx.x & 31;
@@ -130,7 +139,13 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const DispatchArgs a)
   const int chunks = a.d / 8;
   const uint4* g4 = reinterpret_cast<const uint4*>(a.gamma);
   for (int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; p < n_kept; p += warps) {
-    const int t = a.perm[p] / a.k;
+    const int asg = a.perm[p];
+    if (asg < 0) {
+      uint4* dst = reinterpret_cast<uint4*>(a.x_perm + static_cast<size_t>(p) * a.d);
+      for (int c = lane; c < chunks; c += 32) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const int t = asg / a.k;
     const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d);
     uint4* dst = reinterpret_cast<uint4*>(a.x_perm + static_cast<size_t>(p) * a.d);
     for (int c = lane; c < chunks; c += 32) {

@@ -1,7 +1,7 @@
-// grouped_gemm.cu -- the expert FFN as two persistent grouped GEMMs on the
-// 5th-generation tensor cores: 2-CTA (cta_group::2) tcgen05.mma with fp32
-// accumulators in TMEM, operands staged by TMA into 128-byte-swizzled shared
-// memory.
+// grouped_gemm.cu -- the expert FFN's contractions, forward and backward, as
+// persistent grouped GEMMs on the 5th-generation tensor cores: 2-CTA
+// (cta_group::2) tcgen05.mma with fp32 accumulators in TMEM, operands staged
+// by TMA into 128-byte-swizzled shared memory.
 //
 // OmniMoE summary (gist.science), section 2.2 "Expert-Centric Scheduling":
 // with the rows grouped by expert, each expert's weight block is loaded once
@@ -11,28 +11,39 @@
 // through cumulative offsets; the work decomposition uses running sums of
 // per-expert tile counts, never index * size ("Critical Bug Fix").
 // CODA sparse-MoE thread (digg.com): the RMS statistic r of each token is
-// applied in the epilogue of the first expert GEMM.
+// applied in the epilogue of the first expert GEMM, and the RMSNorm backward
+// is fused into that linear's backward, which is why r travels with the token.
 //
-//   up   (GEMM 1): for the kept rows p of expert e (t = perm[p] / k),
-//        H[p, n] = bf16( silu(r_t * acc1[p, n]) * (r_t * acc3[p, n]) ),
-//        acc1 = x_perm[p] . W1[:, o_e + n], acc3 = x_perm[p] . W3[:, o_e + n].
-//        One 256 x 256 x 16 pair MMA covers 128 columns of W1 and the same 128
-//        columns of W3, so both SwiGLU inputs of a row sit in one accumulator.
-//   down (GEMM 2): y[p, n] = bf16( gate[perm[p]] * (H[p, :f_e] . W2[o_e + :, n]) ).
+// Modes (p = kept row of expert e, t = perm[p] / k; -1 in perm marks a
+// padding row, whose outputs are zero):
+//   up     H[p, n] = bf16( silu(r_t * acc1) * (r_t * acc3) ), acc1 = x_perm[p] . W1[:, o_e+n],
+//          acc3 = x_perm[p] . W3[:, o_e+n].  One 256 x 256 x 16 pair MMA covers 128 columns
+//          of W1 and the same 128 of W3.  Training also stores U = r*acc1, V = r*acc3.
+//   down   y[p, n] = bf16( gate[perm[p]] * (H[p, :f_e] . W2[o_e + :, n]) ); training also
+//          stores the ungated bf16(acc).
+//   bwd_h  G = dY[p] . W2[o_e + n, :]  (dY = gate * dout of the row's token), then
+//          du = G * v * silu'(u), dv = G * silu(u) from the saved U, V, and
+//          dS = bf16(r_t du), dS3 = bf16(r_t dv), plus the dr partial sum_n (du u + dv v) / r_t
+//          of this N tile.
+//   bwd_x  dX[p, c] = dS[p] . W1[c, o_e + :] + dS3[p] . W3[c, o_e + :]   (fp32 out)
+//   wgrad_x dW1[c, o_e+n] = sum_p x_perm[p, c] dS[p, n], dW3 likewise with dS3 (fp32 out)
+//   wgrad_h dW2[o_e+m, c] = sum_p H[p, m] dY[p, c]                          (fp32 out)
+// The weight-gradient modes reduce over an expert's rows, so their K range is
+// the expert's row segment; the training layout pads every segment to a
+// multiple of 64 rows with zero rows so that K blocks never cross segments.
 //
 // CTA pairs (clusters of 2): a pair owns a 256-row x BN tile.  Each CTA loads
-// its own 128 rows of A and its half of the BN columns of B (so B crosses L2
-// once per pair, not once per CTA); the leader CTA issues the pair MMA, which
-// reads both CTAs' shared memory and writes each CTA's 128 rows of D into that
-// CTA's TMEM.  Both CTAs' loads complete on the leader's "full" barrier; the
-// MMA commit arrives on both CTAs' "empty" and "accumulator full" barriers;
-// both CTAs' epilogues arrive on the leader's "accumulator empty" barrier.
+// its own 128 rows (M) of A and half of the BN columns of B; the leader CTA
+// issues the pair MMA, which reads both CTAs' shared memory and writes each
+// CTA's 128 rows of D into that CTA's TMEM.  Both CTAs' loads complete on the
+// leader's "full" barrier; the MMA commit arrives on both CTAs' "empty" and
+// "accumulator full" barriers; both CTAs' epilogues arrive on the leader's
+// "accumulator empty" barrier.
 //
-// Tiles: expert e contributes ceil(n_e/256) * (N_e/BN) pair tiles, listed on
-// the device from the kept-row offsets (no host sync) in raster groups of
-// M tiles whose A rows fit a 48 MB L2 budget (M fastest inside a group), so
-// pairs running together share A rows and weight column blocks in L2.
-// Persistent pairs stride through the list.
+// Tiles: expert e contributes ceil(M_e/256) * (N_e/BN) pair tiles, listed on
+// the device from the row offsets (no host sync) in raster groups of M tiles
+// whose A bytes fit a 48 MB L2 budget (M fastest inside a group).  Persistent
+// pairs stride through the list.
 //
 // Warp roles (192 threads per CTA): warp 0 = TMA producer, warp 1 = MMA issuer
 // (leader only) and TMEM owner, warps 2..5 = epilogue (TMEM -> registers ->
@@ -56,7 +67,7 @@ constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = 256;                 // columns per accumulator buffer
-constexpr int kAtomBytes = BK * 64 * 2;       // one 64(n) x 64(k) B box: 8 KB
+constexpr int kAtomBytes = BK * 64 * 2;       // one 64(mn) x 64(k) MN-major box: 8 KB
 constexpr int kEpiWarps = 4;
 constexpr long long kL2GroupBudget = 48ll << 20;  // A bytes of one raster group
 
@@ -68,10 +79,12 @@ struct __align__(8) GemmShared {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
+  int bad_segment;
   int total_tiles;
   int tile_start[kMaxExperts + 1];
   int m_tiles[kMaxExperts];
   int n_tiles[kMaxExperts];
+  int k_blocks[kMaxExperts];
   int group_m[kMaxExperts];  // m tiles per raster group (see decode_tile)
   int seg[kMaxExperts + 1];
 };
@@ -103,12 +116,276 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
 
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_t (&o)[16]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) d4[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+}
+
+__device__ __forceinline__ void store_zero_bf16(__nv_bfloat16* dst) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) d4[j] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+__device__ __forceinline__ void store_row_f32(float* dst, const uint32_t (&u)[32], bool zero) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    d4[j] = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                 : make_float4(__uint_as_float(u[4 * j]), __uint_as_float(u[4 * j + 1]),
+                               __uint_as_float(u[4 * j + 2]), __uint_as_float(u[4 * j + 3]));
+}
+
+template <int MODE>
+struct Traits {
+  static constexpr bool a_mn = (MODE == kGemmWgradX || MODE == kGemmWgradH);
+  static constexpr bool b_mn = (MODE == kGemmUp || MODE == kGemmDown || MODE == kGemmWgradX ||
+                                MODE == kGemmWgradH);
+  static constexpr bool row_tiles = !a_mn;  // M runs over an expert's rows
+};
+
+// Extent of the tile space of expert e: M extent (rows of D), N tiles, K blocks.
+template <int MODE>
+__device__ __forceinline__ void geometry(int rows, int f, int d, int bn, int& mext, int& nt, int& kb) {
+  if (MODE == kGemmUp) {
+    mext = rows; nt = f / kBlockN; kb = d / BK;
+  } else if (MODE == kGemmDown) {
+    mext = rows; nt = d / bn; kb = f / BK;
+  } else if (MODE == kGemmBwdH) {
+    mext = rows; nt = f / bn; kb = d / BK;
+  } else if (MODE == kGemmBwdX) {
+    mext = rows; nt = d / bn; kb = 2 * f / BK;
+  } else if (MODE == kGemmWgradX) {
+    mext = d; nt = 2 * f / bn; kb = rows / BK;
+  } else {  // kGemmWgradH
+    mext = f; nt = d / bn; kb = rows / BK;
+  }
+}
+
+struct Maps {
+  const CUtensorMap* a0;
+  const CUtensorMap* a1;
+  const CUtensorMap* b0;
+  const CUtensorMap* b1;
+};
+
+// TMA loads of K block kb of tile c into one stage (this CTA's half).
+// Every x coordinate is a multiple of 64 elements (128 B).
+template <int MODE>
+__device__ __forceinline__ void issue_loads(const Maps& m, const TileCoord& c, int kb, uint8_t* sA,
+                                            uint8_t* sB, uint32_t bar, int seg_e, int o_e, int f,
+                                            uint32_t rank, int bn) {
+  const int half_bn = bn / 2;
+  if (Traits<MODE>::row_tiles) {
+    const int row0 = seg_e + c.mt * BM + static_cast<int>(rank) * BM_CTA;
+    if (MODE == kGemmUp) {
+      // leader: 128 columns of W1; peer: the same 128 columns of W3 (MN-major)
+      tma_load_2d_pair(sA, m.a0, bar, kb * BK, row0);
+      const CUtensorMap* mB = rank == 0 ? m.b0 : m.b1;
+      const int n0 = o_e + c.nt * kBlockN;
+      tma_load_2d_pair(sB, mB, bar, n0, kb * BK);
+      tma_load_2d_pair(sB + kAtomBytes, mB, bar, n0 + 64, kb * BK);
+    } else if (MODE == kGemmDown) {
+      tma_load_2d_pair(sA, m.a0, bar, kb * BK, row0);
+      const int n0 = c.nt * bn + static_cast<int>(rank) * half_bn;
+      for (int j = 0; j < half_bn / 64; ++j)
+        tma_load_2d_pair(sB + j * kAtomBytes, m.b0, bar, n0 + j * 64, o_e + kb * BK);
+    } else if (MODE == kGemmBwdH) {
+      // B = rows o_e + n of W2 [F, d], K-major (box 64 k x half_bn rows)
+      tma_load_2d_pair(sA, m.a0, bar, kb * BK, row0);
+      tma_load_2d_pair(sB, m.b0, bar, kb * BK, o_e + c.nt * bn + static_cast<int>(rank) * half_bn);
+    } else {  // kGemmBwdX: K runs over f_e columns of dS (x W1^T), then of dS3 (x W3^T)
+      const int kf = f / BK;
+      const bool second = kb >= kf;
+      const int kk = second ? kb - kf : kb;
+      tma_load_2d_pair(sA, second ? m.a1 : m.a0, bar, kk * BK, row0);
+      tma_load_2d_pair(sB, second ? m.b1 : m.b0, bar, o_e + kk * BK,
+                       c.nt * bn + static_cast<int>(rank) * half_bn);
+    }
+  } else {
+    // weight gradients: A^T and B both MN-major, K = rows seg_e + kb*64 ...
+    const int m0 = c.mt * BM + static_cast<int>(rank) * BM_CTA;
+    const int k0 = seg_e + kb * BK;
+    tma_load_2d_pair(sA, m.a0, bar, m0, k0);
+    tma_load_2d_pair(sA + kAtomBytes, m.a0, bar, m0 + 64, k0);
+    int n0 = c.nt * bn + static_cast<int>(rank) * half_bn;
+    const CUtensorMap* mB = m.b0;
+    if (MODE == kGemmWgradX && n0 >= f) {  // dW3 half of the [dW1 | dW3] N range
+      n0 -= f;
+      mB = m.b1;
+    }
+    for (int j = 0; j < half_bn / 64; ++j) tma_load_2d_pair(sB + j * kAtomBytes, mB, bar, n0 + j * 64, k0);
+  }
+}
+
+// ---- epilogues: one thread per accumulator row (TMEM lane), 32 columns per load
+template <int MODE>
+__device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShared& sh, const TileCoord& c,
+                                              uint32_t taddr, int row_in_cta, uint32_t rank) {
+  const int p = sh.seg[c.e] + c.mt * BM + static_cast<int>(rank) * BM_CTA + row_in_cta;
+  const bool valid = p < sh.seg[c.e + 1];
+  const int asg = valid ? a.perm[p] : -1;
+  const bool pad = valid && asg < 0;  // padding row of the training layout: zeros out
+  const size_t prow = static_cast<size_t>(valid ? p : 0);
+  if (MODE == kGemmUp) {
+    const float scale = asg >= 0 ? a.scale[asg / a.k] : 0.f;
+    const size_t off = prow * a.ld_out + c.nt * kBlockN;
+#pragma unroll 1
+    for (int cc = 0; cc < kBlockN; cc += 32) {
+      uint32_t u[32], v[32];
+      tmem_ld_32x32b_x32(taddr + cc, u);
+      tmem_ld_32x32b_x32(taddr + kBlockN + cc, v);
+      tmem_ld_wait();
+      if (!valid) continue;
+      if (pad) {
+        store_zero_bf16(a.out + off + cc);
+        if (a.out_u != nullptr) {
+          store_zero_bf16(a.out_u + off + cc);
+          store_zero_bf16(a.out_v + off + cc);
+        }
+        continue;
+      }
+      uint32_t o[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float h0 = silu(scale * __uint_as_float(u[2 * j])) * (scale * __uint_as_float(v[2 * j]));
+        const float h1 = silu(scale * __uint_as_float(u[2 * j + 1])) * (scale * __uint_as_float(v[2 * j + 1]));
+        o[j] = pack_bf16(h0, h1);
+      }
+      store_row_bf16(a.out + off + cc, o);
+      if (a.out_u != nullptr) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          o[j] = pack_bf16(scale * __uint_as_float(u[2 * j]), scale * __uint_as_float(u[2 * j + 1]));
+        store_row_bf16(a.out_u + off + cc, o);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          o[j] = pack_bf16(scale * __uint_as_float(v[2 * j]), scale * __uint_as_float(v[2 * j + 1]));
+        store_row_bf16(a.out_v + off + cc, o);
+      }
+    }
+  } else if (MODE == kGemmDown) {
+    const float scale = asg >= 0 ? a.scale[asg] : 0.f;
+    const size_t off = prow * a.ld_out + c.nt * a.bn;
+#pragma unroll 1
+    for (int cc = 0; cc < a.bn; cc += 32) {
+      uint32_t u[32];
+      tmem_ld_32x32b_x32(taddr + cc, u);
+      tmem_ld_wait();
+      if (!valid) continue;
+      if (pad) {
+        store_zero_bf16(a.out + off + cc);
+        if (a.out_yu != nullptr) store_zero_bf16(a.out_yu + off + cc);
+        continue;
+      }
+      uint32_t o[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        o[j] = pack_bf16(scale * __uint_as_float(u[2 * j]), scale * __uint_as_float(u[2 * j + 1]));
+      store_row_bf16(a.out + off + cc, o);
+      if (a.out_yu != nullptr) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) o[j] = pack_bf16(__uint_as_float(u[2 * j]), __uint_as_float(u[2 * j + 1]));
+        store_row_bf16(a.out_yu + off + cc, o);
+      }
+    }
+  } else if (MODE == kGemmBwdH) {
+    const float r = asg >= 0 ? a.scale[asg / a.k] : 0.f;
+    const size_t off = prow * a.ld_out + c.nt * a.bn;
+    float dr = 0.f;
+#pragma unroll 1
+    for (int cc = 0; cc < a.bn; cc += 32) {
+      uint32_t g[32];
+      tmem_ld_32x32b_x32(taddr + cc, g);
+      tmem_ld_wait();
+      if (!valid) continue;
+      if (pad) {
+        store_zero_bf16(a.out_ds + off + cc);
+        store_zero_bf16(a.out_ds3 + off + cc);
+        continue;
+      }
+      uint32_t uw[16], vw[16];
+      const uint4* u4 = reinterpret_cast<const uint4*>(a.in_u + off + cc);
+      const uint4* v4 = reinterpret_cast<const uint4*>(a.in_v + off + cc);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 x = u4[j], y = v4[j];
+        uw[4 * j] = x.x; uw[4 * j + 1] = x.y; uw[4 * j + 2] = x.z; uw[4 * j + 3] = x.w;
+        vw[4 * j] = y.x; vw[4 * j + 1] = y.y; vw[4 * j + 2] = y.z; vw[4 * j + 3] = y.w;
+      }
+      uint32_t o1[16], o3[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        float du[2], dv[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float uu = h ? bf16_hi(uw[j]) : bf16_lo(uw[j]);
+          const float vv = h ? bf16_hi(vw[j]) : bf16_lo(vw[j]);
+          const float gg = __uint_as_float(g[2 * j + h]);
+          const float sg = 1.0f / (1.0f + __expf(-uu));
+          du[h] = gg * vv * (sg * (1.0f + uu * (1.0f - sg)));
+          dv[h] = gg * (uu * sg);
+          dr += du[h] * uu + dv[h] * vv;
+        }
+        o1[j] = pack_bf16(r * du[0], r * du[1]);
+        o3[j] = pack_bf16(r * dv[0], r * dv[1]);
+      }
+      store_row_bf16(a.out_ds + off + cc, o1);
+      store_row_bf16(a.out_ds3 + off + cc, o3);
+    }
+    if (valid) a.drp[prow * a.ld_drp + c.nt] = pad ? 0.f : dr / r;
+  } else {  // kGemmBwdX
+    float* dst = a.out_f0 + prow * a.ld_f + c.nt * a.bn;
+#pragma unroll 1
+    for (int cc = 0; cc < a.bn; cc += 32) {
+      uint32_t u[32];
+      tmem_ld_32x32b_x32(taddr + cc, u);
+      tmem_ld_wait();
+      if (valid) store_row_f32(dst + cc, u, pad);
+    }
+  }
+}
+
+// Weight gradients: the accumulator row is an output row of dW (a column of
+// x_perm or H); an expert with no rows gets zeros.
+template <int MODE>
+__device__ __forceinline__ void epilogue_wgrad(const GemmArgs& a, const GemmShared& sh, const TileCoord& c,
+                                               uint32_t taddr, int row_in_cta, uint32_t rank) {
+  const int o_e = a.ffn.off[c.e];
+  const int f = a.ffn.off[c.e + 1] - o_e;
+  const int m = c.mt * BM + static_cast<int>(rank) * BM_CTA + row_in_cta;
+  const bool zero = sh.k_blocks[c.e] == 0;
+  const bool valid = m < (MODE == kGemmWgradX ? a.d : f);
+#pragma unroll 1
+  for (int cc = 0; cc < a.bn; cc += 32) {
+    uint32_t u[32];
+    if (!zero) {
+      tmem_ld_32x32b_x32(taddr + cc, u);
+      tmem_ld_wait();
+    }
+    if (!valid) continue;
+    const int n = c.nt * a.bn + cc;
+    float* dst;
+    if (MODE == kGemmWgradX)
+      dst = (n < f ? a.out_f0 + static_cast<size_t>(m) * a.ld_f + o_e + n
+                   : a.out_f1 + static_cast<size_t>(m) * a.ld_f + o_e + (n - f));
+    else
+      dst = a.out_f0 + static_cast<size_t>(o_e + m) * a.ld_f + n;
+    store_row_f32(dst, u, zero);
+  }
+}
+
+template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
-                        const __grid_constant__ CUtensorMap mapB0,
-                        const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ GemmArgs a) {
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
+                        const __grid_constant__ CUtensorMap mapB0, const __grid_constant__ CUtensorMap mapB1,
+                        const __grid_constant__ GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   GemmShared& sh = *reinterpret_cast<GemmShared*>(smem + kStages * kStageBytes);
@@ -130,12 +407,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     mbar_init(&sh.drain, 1);
     sh.abort_flag = 0;
+    sh.bad_segment = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_map(&mapA);
+    tma_prefetch_map(&mapA0);
     tma_prefetch_map(&mapB0);
-    tma_prefetch_map(&mapB1);
+    if (MODE == kGemmBwdX) tma_prefetch_map(&mapA1);
+    if (MODE == kGemmUp || MODE == kGemmBwdX || MODE == kGemmWgradX) tma_prefetch_map(&mapB1);
   }
   if (warp == 1) {
     tmem_alloc_pair(&sh.tmem_base, kTmemCols);
@@ -145,25 +424,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (tid < E) {
     const int rows = sh.seg[tid + 1] - sh.seg[tid];
-    const int ncols = a.up ? (a.ffn.off[tid + 1] - a.ffn.off[tid]) : a.d;
-    const int nt = a.up ? ncols / kBlockN : ncols / a.bn;
-    const int mt = (rows + BM - 1) / BM;
-    // A bytes of one M tile: 256 rows x the reduction length (d up, f_e down)
-    const long long a_rows_bytes =
-        static_cast<long long>(BM) * (a.up ? a.d : (a.ffn.off[tid + 1] - a.ffn.off[tid])) * 2;
+    const int f = a.ffn.off[tid + 1] - a.ffn.off[tid];
+    int mext, nt, kb;
+    geometry<MODE>(rows, f, a.d, a.bn, mext, nt, kb);
+    // K of the weight gradients is a row segment: it must be whole K blocks
+    if (!Traits<MODE>::row_tiles && (rows < 0 || rows % BK != 0)) sh.bad_segment = 1;
+    const int mt = (mext + BM - 1) / BM;
+    const long long a_rows_bytes = static_cast<long long>(BM) * kb * BK * 2;
     int gm = static_cast<int>(kL2GroupBudget / (a_rows_bytes > 0 ? a_rows_bytes : 1));
     gm = gm < 1 ? 1 : gm;
     sh.m_tiles[tid] = mt > 0 ? mt : 1;
     sh.n_tiles[tid] = nt > 0 ? nt : 1;
+    sh.k_blocks[tid] = kb;
     sh.group_m[tid] = gm < sh.m_tiles[tid] ? gm : sh.m_tiles[tid];
-    sh.tile_start[tid + 1] = mt * nt;  // count for now
+    sh.tile_start[tid + 1] = (mt > 0 && nt > 0) ? mt * nt : 0;  // count for now
   }
   __syncthreads();
   if (tid == 0) {
     sh.tile_start[0] = 0;
     for (int e = 0; e < E; ++e) sh.tile_start[e + 1] += sh.tile_start[e];
     sh.total_tiles = sh.tile_start[E];
-    if (sh.seg[E] > a.rows) {  // more kept rows than the buffers hold: do nothing
+    if (sh.seg[E] > a.rows || sh.bad_segment) {  // rows the buffers do not hold: do nothing
       if (rank == 0) atomicOr(a.err, MOE_DEVERR_TILE_TABLE);
       sh.total_tiles = 0;
     }
@@ -174,20 +455,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = sh.tmem_base;
   const int total = sh.total_tiles;
   volatile int* abort_flag = &sh.abort_flag;
-  const int half_bn = a.bn / 2;
+  const Maps maps{&mapA0, &mapA1, &mapB0, &mapB1};
 
   if (warp == 0) {
     // ================= TMA producer (one lane per CTA)
     if (lane == 0) {
       const uint32_t full_leader0 = map_to_cta(smem_addr(&sh.full[0]), 0);
-      const uint32_t tx_pair = 2u * (kABytes + static_cast<uint32_t>(half_bn) * BK * 2u);
+      const uint32_t tx_pair = 2u * (kABytes + static_cast<uint32_t>(a.bn / 2) * BK * 2u);
       uint32_t it = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < total; tile += npairs) {
         const TileCoord c = decode_tile(sh, E, tile);
-        const int row0 = sh.seg[c.e] + c.mt * BM + static_cast<int>(rank) * BM_CTA;
         const int o_e = a.ffn.off[c.e];
-        const int kblocks = a.up ? a.d / BK : (a.ffn.off[c.e + 1] - o_e) / BK;
+        const int f = a.ffn.off[c.e + 1] - o_e;
+        const int kblocks = sh.k_blocks[c.e];
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1u;
@@ -196,21 +477,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* sA = smem + s * kStageBytes;
-          uint8_t* sB = sA + kABytes;
           const uint32_t bar = full_leader0 + static_cast<uint32_t>(s) * 8u;
           if (rank == 0) mbar_arrive_expect_tx(&sh.full[s], tx_pair);
-          tma_load_2d_pair(sA, &mapA, bar, kb * BK, row0);
-          if (a.up) {
-            // leader: 128 columns of W1; peer: the same 128 columns of W3
-            const CUtensorMap* mB = rank == 0 ? &mapB0 : &mapB1;
-            const int n0 = o_e + c.nt * kBlockN;
-            tma_load_2d_pair(sB, mB, bar, n0, kb * BK);
-            tma_load_2d_pair(sB + kAtomBytes, mB, bar, n0 + 64, kb * BK);
-          } else {
-            const int n0 = c.nt * a.bn + static_cast<int>(rank) * half_bn;
-            for (int j = 0; j < half_bn / 64; ++j)
-              tma_load_2d_pair(sB + j * kAtomBytes, &mapB0, bar, n0 + j * 64, o_e + kb * BK);
-          }
+          issue_loads<MODE>(maps, c, kb, sA, sA + kABytes, bar, sh.seg[c.e], o_e, f, rank, a.bn);
         }
       }
       // Drain: the last stages issued are released by the MMA (normally already
@@ -225,13 +494,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ================= MMA issuer (leader CTA, one lane)
     if (rank == 0 && lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16(BM, a.bn, 1);
+      const uint32_t idesc = umma_idesc_bf16(BM, a.bn, Traits<MODE>::b_mn ? 1u : 0u, Traits<MODE>::a_mn ? 1u : 0u);
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < total; tile += npairs, ++tcount) {
         const TileCoord c = decode_tile(sh, E, tile);
-        const int o_e = a.ffn.off[c.e];
-        const int kblocks = a.up ? a.d / BK : (a.ffn.off[c.e + 1] - o_e) / BK;
+        const int kblocks = sh.k_blocks[c.e];
         const uint32_t buf = tcount & 1u;
         const uint32_t aph = (tcount >> 1) & 1u;
         // both CTAs' epilogues release the buffer (the peer's arrival is remote)
@@ -254,8 +522,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t aB = aA + kABytes;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(aA + kk * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(aB + kk * 2048, kAtomBytes, 1024);
+            const uint64_t adesc = Traits<MODE>::a_mn ? smem_desc_sw128(aA + kk * 2048, kAtomBytes, 1024)
+                                                      : smem_desc_sw128(aA + kk * 32, 16, 1024);
+            const uint64_t bdesc = Traits<MODE>::b_mn ? smem_desc_sw128(aB + kk * 2048, kAtomBytes, 1024)
+                                                      : smem_desc_sw128(aB + kk * 32, 16, 1024);
             umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit_pair_mc(&sh.empty[s], 0x3);  // frees the stage in both CTAs
@@ -283,53 +553,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       tc_fence_after();
-      const int p = sh.seg[c.e] + c.mt * BM + static_cast<int>(rank) * BM_CTA + row_in_cta;
-      const bool valid = p < sh.seg[c.e + 1];
-      float scale = 0.f;
-      if (valid) {
-        const int asg = a.perm[p];
-        scale = a.up ? a.scale[asg / a.k] : a.scale[asg];
-      }
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kAccCols;
-      if (a.up) {
-        __nv_bfloat16* dst = a.out + static_cast<size_t>(valid ? p : 0) * a.ld_out + c.nt * kBlockN;
-#pragma unroll 1
-        for (int cc = 0; cc < kBlockN; cc += 32) {
-          uint32_t u[32], v[32];
-          tmem_ld_32x32b_x32(taddr + cc, u);
-          tmem_ld_32x32b_x32(taddr + kBlockN + cc, v);
-          tmem_ld_wait();
-          if (valid) {
-            uint32_t o[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float h0 = silu(scale * __uint_as_float(u[2 * j])) * (scale * __uint_as_float(v[2 * j]));
-              const float h1 = silu(scale * __uint_as_float(u[2 * j + 1])) * (scale * __uint_as_float(v[2 * j + 1]));
-              o[j] = pack_bf16(h0, h1);
-            }
-            uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) d4[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-          }
-        }
-      } else {
-        __nv_bfloat16* dst = a.out + static_cast<size_t>(valid ? p : 0) * a.ld_out + c.nt * a.bn;
-#pragma unroll 1
-        for (int cc = 0; cc < a.bn; cc += 32) {
-          uint32_t u[32];
-          tmem_ld_32x32b_x32(taddr + cc, u);
-          tmem_ld_wait();
-          if (valid) {
-            uint32_t o[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              o[j] = pack_bf16(scale * __uint_as_float(u[2 * j]), scale * __uint_as_float(u[2 * j + 1]));
-            uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) d4[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-          }
-        }
-      }
+      if (Traits<MODE>::row_tiles)
+        epilogue_rows<MODE>(a, sh, c, taddr, row_in_cta, rank);
+      else
+        epilogue_wgrad<MODE>(a, sh, c, taddr, row_in_cta, rank);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + buf * 8u);
@@ -343,22 +571,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
 }
 
+template <int MODE>
+cudaError_t set_smem_attr() {
+  return cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(kSmemBytes));
+}
+
 }  // namespace
 
 size_t grouped_gemm_smem_bytes() { return kSmemBytes; }
 
 cudaError_t prepare_grouped_gemm() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(kSmemBytes));
+  cudaError_t e = set_smem_attr<kGemmUp>();
+  if (e == cudaSuccess) e = set_smem_attr<kGemmDown>();
+  if (e == cudaSuccess) e = set_smem_attr<kGemmBwdH>();
+  if (e == cudaSuccess) e = set_smem_attr<kGemmBwdX>();
+  if (e == cudaSuccess) e = set_smem_attr<kGemmWgradX>();
+  if (e == cudaSuccess) e = set_smem_attr<kGemmWgradH>();
+  return e;
 }
 
+// All modes share the launch shape (192 threads, the same shared memory), so
+// the co-resident cluster count of one instantiation holds for all.
 int grouped_gemm_max_grid(int num_sms) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel, &cfg) != cudaSuccess || clusters <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<kGemmUp>, &cfg) != cudaSuccess ||
+      clusters <= 0) {
     cudaGetLastError();
     return num_sms & ~1;
   }
@@ -366,9 +608,32 @@ int grouped_gemm_max_grid(int num_sms) {
   return grid < (num_sms & ~1) ? grid : (num_sms & ~1);
 }
 
-cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB0,
-                                const CUtensorMap& mapB1, int grid, cudaStream_t s) {
-  grouped_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(mapA, mapB0, mapB1, a);
+cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA0, const CUtensorMap& mapA1,
+                                const CUtensorMap& mapB0, const CUtensorMap& mapB1, int grid,
+                                cudaStream_t s) {
+  if (a.bn != 128 && a.bn != 256) return cudaErrorInvalidValue;
+  switch (a.mode) {
+    case kGemmUp:
+      grouped_gemm_kernel<kGemmUp><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, a);
+      break;
+    case kGemmDown:
+      grouped_gemm_kernel<kGemmDown><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, a);
+      break;
+    case kGemmBwdH:
+      grouped_gemm_kernel<kGemmBwdH><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, a);
+      break;
+    case kGemmBwdX:
+      grouped_gemm_kernel<kGemmBwdX><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, a);
+      break;
+    case kGemmWgradX:
+      grouped_gemm_kernel<kGemmWgradX><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, a);
+      break;
+    case kGemmWgradH:
+      grouped_gemm_kernel<kGemmWgradH><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, a);
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

@@ -56,18 +56,42 @@ struct DispatchArgs {
   int T, d, E, k;
   int capacity;             // -1: dropless
   int max_kept;             // rows of x_perm
+  int row_align;            // 1: dense segments; 64: each expert's segment padded
+                            // to a multiple of 64 rows (perm = -1, x_perm = 0 there)
+};
+
+// Modes of the grouped GEMM (one kernel template, one instantiation each).
+enum GemmMode : int {
+  kGemmUp = 0,      // x_perm x (W1|W3) -> SwiGLU -> H            (forward GEMM 1)
+  kGemmDown = 1,    // H x W2 -> gate * y                         (forward GEMM 2)
+  kGemmBwdH = 2,    // dY x W2^T -> SwiGLU/statistic backward -> dS, dS3, dr partials
+  kGemmBwdX = 3,    // [dS | dS3] x [W1 | W3]^T -> dX per kept row (fp32)
+  kGemmWgradX = 4,  // x_perm^T x [dS | dS3] -> dW1 | dW3 (fp32), K = expert rows
+  kGemmWgradH = 5,  // H^T x dY -> dW2 (fp32), K = expert rows
 };
 
 struct GemmArgs {
-  int up;                   // 1: x_perm x (W1|W3) -> SwiGLU -> H; 0: H x W2 -> y
+  int mode;
   int E, k, d;
-  int bn;                   // N tile: 256 for up (128 of W1 + 128 of W3); 128/256 for down
-  int rows;                 // rows of the A operand buffer (max kept)
-  const int32_t* offsets;   // [E+1] kept-row offsets (device)
-  const int32_t* perm;      // [max_kept]
-  const float* scale;       // up: r [T] (indexed by token); down: gate [T*k] (by assignment)
+  int bn;                   // N tile of the pair MMA: 128 or 256
+  int rows;                 // rows of the permuted buffers
+  const int32_t* offsets;   // [E+1] row-segment offsets (device)
+  const int32_t* perm;      // [rows]; -1 marks a padding row
+  const float* scale;       // up, bwd_h: r [T] (by token); down: gate [T*k] (by assignment)
   __nv_bfloat16* out;       // up: H [rows, ld_out]; down: y [rows, d]
-  int ld_out;
+  int ld_out;               // row stride of H-shaped buffers (max expert width)
+  __nv_bfloat16* out_u;     // up, training: U = r*(x W1) [rows, ld_out] (may be null)
+  __nv_bfloat16* out_v;     // up, training: V = r*(x W3)
+  __nv_bfloat16* out_yu;    // down, training: ungated y [rows, d] (may be null)
+  const __nv_bfloat16* in_u;  // bwd_h: U, V saved by the forward
+  const __nv_bfloat16* in_v;
+  __nv_bfloat16* out_ds;    // bwd_h: dS = r*du, dS3 = r*dv [rows, ld_out]
+  __nv_bfloat16* out_ds3;
+  float* drp;               // bwd_h: [rows, ld_drp] per-N-tile partials of dr
+  int ld_drp;
+  float* out_f0;            // bwd_x: dX [rows, d]; wgrad_x: dW1 [d, F]; wgrad_h: dW2 [F, d]
+  float* out_f1;            // wgrad_x: dW3 [d, F]
+  int ld_f;
   uint32_t* err;
   ExpertTable ffn;
 };
@@ -79,10 +103,56 @@ struct CombineArgs {
   int T, d, k;
 };
 
+// Backward elementwise / reduction stages (backward.cu).
+struct BwdArgs {
+  int T, d, E, k, renormalize;
+  int rows;                       // rows of the padded permuted buffers
+  const __nv_bfloat16* x;         // [T, d]
+  const __nv_bfloat16* gamma;     // [d]
+  const __nv_bfloat16* Wr;        // [d, E]
+  const float* bias;              // [E] or null
+  const __nv_bfloat16* dout;      // [T, d] upstream gradient
+  const float* r;                 // [T] saved statistic
+  const int32_t* idx;             // [T, k] saved routing
+  const float* gate;              // [T, k]
+  const float* logits;            // [T, E] saved fp32 logits (bias included)
+  const int32_t* offsets;         // [E+1] padded row segments
+  const int32_t* perm;            // [rows], -1 = padding
+  const int32_t* inv_perm;        // [T*k], -1 = dropped
+  const __nv_bfloat16* yu;        // [rows, d] saved ungated expert outputs
+  __nv_bfloat16* dY;              // [rows, d] out: gate * dout of the row's token
+  float* dgate;                   // [T*k] out: <dout_t, y_a> (kept slots only)
+  const float* drp;               // [rows, ld_drp] dr partials of the bwd_h GEMM
+  int ld_drp, bn_h;               // bn_h: N tile of that GEMM (partials per row = f_e / bn_h)
+  const float* dXp;               // [rows, d] expert part of d(x*gamma) per kept row
+  float* rdl;                     // [T, E] out: r_t * dl_t
+  float* dr;                      // [T] out: dL/dr_t
+  float* dbias_part;              // [route_blocks, E]
+  int route_blocks;
+  float* dx;                      // [T, d] out
+  float* dgamma_part;             // [chunks, d]
+  float* dWr_part;                // [chunks, d, E]
+  int chunks, chunk_tokens;
+  float* dgamma;                  // [d] out
+  float* dWr;                     // [d, E] out
+  float* dbias;                   // [E] out
+  uint32_t* err;
+  ExpertTable ffn;
+};
+
+cudaError_t launch_bwd_gather(const BwdArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_bwd_route(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_norm(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_reduce(const BwdArgs& a, cudaStream_t s);
+constexpr int kBwdRouteTokens = 64;   // tokens per bwd_route CTA (8 warps x 8)
+constexpr int kBwdNormCols = 128;     // columns per bwd_norm CTA
+
 // Launchers (return the launch error, if any).
 cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchArgs& a, int num_sms, cudaStream_t s);
-cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA,
+// mapA1 is the second A operand (bwd_x: dS3); mapB1 the second B operand
+// (up: W3; bwd_x: W3; wgrad_x: dS3).  Unused maps may repeat another.
+cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA0, const CUtensorMap& mapA1,
                                 const CUtensorMap& mapB0, const CUtensorMap& mapB1, int grid,
                                 cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);

@@ -303,11 +303,11 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate, bf16 A and
 // B, A K-major, B MN-major (b_mn_major = 1) or K-major (0), shape M x N.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(uint32_t M, uint32_t N,
-                                                       uint32_t b_mn_major) {
+                                                       uint32_t b_mn_major, uint32_t a_mn_major = 0) {
   return (1u << 4)                  // D format: f32
          | (1u << 7)                // A format: bf16
          | (1u << 10)               // B format: bf16
-         | (0u << 15)               // A major: K
+         | (a_mn_major << 15)       // A major
          | (b_mn_major << 16)       // B major
          | ((N >> 3) << 17)         // N / 8
          | ((M >> 4) << 24);        // M / 16

@@ -150,3 +150,47 @@ def test_noalloc_dispatch_rejects_oversize_before_device_work(lib):
     P = ctypes.c_void_p
     st = lib.moe_dispatch_noalloc(ctypes.byref(c.c()), *[P(4096 * (i + 1)) for i in range(8)], P(0))
     assert st == moe.MOE_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("name", mw.WORKLOAD_ORDER)
+def test_training_sizes_and_saved_tensors(lib, name):
+    """The training layout pads every expert segment to 64 rows and holds the
+    saved tensors inside the workspace; both are host-side arithmetic."""
+    w = mw.WORKLOADS[name]
+    c = _cfg(w)
+    rows = moe.moe_train_rows(c)
+    assert rows == moe.moe_max_kept(c) + w.E * 63
+    n = moe.moe_train_workspace_size(c)
+    fmax = max(O.expert_widths(w.expert_sizes))
+    # U, V, H, dS, dS3 (bf16) + y, dY (bf16) + dX (fp32) per padded row
+    assert n >= rows * (5 * fmax * 2 + 2 * w.d_model * 2 + w.d_model * 4)
+    base = 1 << 20
+    seen = []
+    for sid in range(14):
+        out = ctypes.c_void_p(0)
+        assert lib.moe_train_saved(ctypes.byref(c.c()), ctypes.c_void_p(base), n, sid, ctypes.byref(out)) == 0
+        assert base <= out.value < base + n
+        seen.append(out.value)
+    assert len(set(seen)) == 14
+    out = ctypes.c_void_p(0)
+    assert lib.moe_train_saved(ctypes.byref(c.c()), ctypes.c_void_p(base), n, 99, ctypes.byref(out)) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_train_saved(ctypes.byref(c.c()), ctypes.c_void_p(base), n - 1, 0, ctypes.byref(out)) == \
+        moe.MOE_ERR_WORKSPACE
+
+
+def test_backward_rejects_bad_arguments_before_device_work(lib):
+    c = _cfg(mw.WORKLOADS["tiny"])
+    P = ctypes.c_void_p
+    ok = [P(1 << 20)] * 15   # x .. dW2
+    n = moe.moe_train_workspace_size(c)
+    # a missing weight-gradient output
+    args = list(ok)
+    args[12] = P(0)         # dW1
+    assert lib.moe_layer_bwd(ctypes.byref(c.c()), *args, P(1 << 20), n, P(0)) == moe.MOE_ERR_INVALID_ARG
+    # a misaligned dW2
+    args = list(ok)
+    args[14] = P((1 << 20) + 4)   # dW2
+    assert lib.moe_layer_bwd(ctypes.byref(c.c()), *args, P(1 << 20), n, P(0)) == moe.MOE_ERR_ALIGNMENT
+    # a workspace one byte short
+    assert lib.moe_layer_bwd(ctypes.byref(c.c()), *ok, P(1 << 20), n - 1, P(0)) == moe.MOE_ERR_WORKSPACE

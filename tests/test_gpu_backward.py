@@ -1,0 +1,115 @@
+"""GPU parity of the layer backward (training forward + moe_layer_bwd) against
+the float64 backward oracle, on the GPU's own routing (replayed into the
+oracle, whose routing parity the forward tests establish).
+
+Tolerance: every gradient tensor within 2e-2 normwise relative error
+(||gpu - ref|| / ||ref||), the same bar as the forward's per-token output.
+The GPU path rounds x*gamma, U, V, H, gate*dout, dS and dS3 to bf16 (each
+2^-9 relative) and accumulates in fp32; the measured errors are printed.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_workloads as mw
+import sparse_mixture_experts_rms_b200 as moe
+from oracle import moe_oracle as O
+from oracle import moe_oracle_bwd as B
+from tests import _harness as H
+
+pytestmark = pytest.mark.gpu
+GRAD_REL = 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from sparse_mixture_experts_rms_b200 import build
+    build.build()
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def _upstream(T, d, seed=7):
+    g = np.random.default_rng(seed).standard_normal((T, d)).astype(np.float32)
+    return mw.f32_to_bf16_bits(g)
+
+
+def _rel(a, b):
+    n = float(np.linalg.norm(b))
+    return float(np.linalg.norm(a - b)) / (n if n > 0 else 1.0)
+
+
+def run_case(w, renormalize=False, bias_override=None):
+    p = H.make_problem(w)
+    if bias_override is not None:
+        p.bias = np.asarray(bias_override, dtype=np.float32)
+    cfg = H.make_cfg(p, renormalize=renormalize)
+    d = H.Dev(p, cfg)
+    T, dm, E, F = cfg.T, cfg.d_model, cfg.E, cfg.F
+    tws = moe.alloc_train_workspace(cfg)
+    out = torch.empty((T, dm), dtype=torch.bfloat16, device="cuda")
+    moe.moe_layer_fwd_train(cfg, d.x, d.gamma, d.Wr, d.bias, d.W1, d.W3, d.W2, out, tws)
+    ref_out = torch.empty_like(out)
+    moe.moe_layer_fwd(cfg, d.x, d.gamma, d.Wr, d.bias, d.W1, d.W3, d.W2, ref_out, d.ws)
+    g_bits = _upstream(T, dm)
+    dout = H.bits_to_dev(g_bits)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    G = {"dx": torch.full((T, dm), float("nan"), **f32), "dgamma": torch.full((dm,), float("nan"), **f32),
+         "dWr": torch.full((dm, E), float("nan"), **f32), "dbias": torch.full((E,), float("nan"), **f32),
+         "dW1": torch.full((dm, F), float("nan"), **f32), "dW3": torch.full((dm, F), float("nan"), **f32),
+         "dW2": torch.full((F, dm), float("nan"), **f32)}
+    moe.moe_layer_bwd(cfg, d.x, d.gamma, d.Wr, d.bias, d.W1, d.W3, d.W2, dout, G["dx"], G["dgamma"],
+                      G["dWr"], G["dbias"], G["dW1"], G["dW3"], G["dW2"], tws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error(tws, raise_on_error=False) == 0
+    assert torch.equal(out, ref_out), "training forward differs from the inference forward"
+    idx = moe.train_saved_view(cfg, tws, "idx").cpu().numpy()
+    f = B.layer_forward(O.widen_bf16(p.x), O.widen_bf16(p.gamma), O.widen_bf16(p.Wr), p.bias,
+                        O.widen_bf16(p.W1), O.widen_bf16(p.W3), O.widen_bf16(p.W2), p.widths, w.k,
+                        w.eps, w.capacity_factor, renormalize, idx=idx)
+    ref = B.layer_backward(f, O.widen_bf16(g_bits))
+    errs = {}
+    for name, t in G.items():
+        got = t.cpu().numpy().astype(np.float64)
+        assert np.isfinite(got).all(), name
+        errs[name] = _rel(got, ref[name])
+    kept = f["kept"]
+    dg = moe.train_saved_view(cfg, tws, "dgate").cpu().numpy().astype(np.float64)
+    errs["dgate"] = _rel(dg[kept], ref["dgate"].reshape(-1)[kept])
+    errs["dr"] = _rel(moe.train_saved_view(cfg, tws, "dr").cpu().numpy().astype(np.float64), ref["dr"])
+    print(w.name, {k_: f"{v:.2e}" for k_, v in errs.items()})
+    for name, v in errs.items():
+        assert v <= GRAD_REL, (name, v)
+    return p, f, G
+
+
+def test_tiny_backward():
+    run_case(mw.WORKLOADS["tiny"])
+
+
+def test_variable_widths_renormalized_backward():
+    """Widths that are odd multiples of 128 (N tile 128 in the dS GEMM), a
+    ragged row count and renormalised gates."""
+    w = mw.Workload("bwd_var", T=300, d_model=256, E=4, k=2,
+                    expert_sizes=((1, 128), (1, 384), (1, 256), (1, 512)))
+    run_case(w, renormalize=True)
+
+
+def test_capacity_and_empty_expert_backward():
+    """Top-1 with capacity drops; expert 2 never chosen (large negative bias):
+    its weight gradients are exactly zero."""
+    w = mw.Workload("bwd_cap", T=512, d_model=256, E=4, k=1, expert_sizes=((4, 256),),
+                    capacity_factor=1.0)
+    p, f, G = run_case(w, bias_override=[0.5, 0.0, -60.0, 0.2])
+    o = O.expert_offsets(p.widths)
+    assert not (f["idx"] == 2).any()
+    assert torch.count_nonzero(G["dW1"][:, o[2]:o[3]]).item() == 0
+    assert torch.count_nonzero(G["dW3"][:, o[2]:o[3]]).item() == 0
+    assert torch.count_nonzero(G["dW2"][o[2]:o[3], :]).item() == 0
+    assert not f["kept"].all()
+
+
+def test_several_tiles_backward():
+    """Several 256-row M tiles and 64-row K blocks per expert."""
+    w = mw.Workload("bwd_tiles", T=1000, d_model=256, E=4, k=2, expert_sizes=((4, 512),), bias="normal")
+    run_case(w)
