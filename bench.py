@@ -45,8 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # profiles/grouped_gemm_traffic_mixtral_T16384.md).  Reported only while the
 # kernel sources still hash to `digest`; after any change it is null until
 # re-measured.
-MEASURED_TRAFFIC = {"workload": "mixtral", "T": 16384, "digest": "b1e688244d6e7377",
-                    "bytes": 4.92e9 + 0.931e9}   # dram read + write of the up launch
+MEASURED_TRAFFIC = {"workload": "mixtral", "T": 16384, "digest": "ec32e90f433f4d38",
+                    "bytes": 5.81e9 + 0.929e9}   # dram read + write of the up launch (median of 12)
 
 
 def kernel_digest() -> str:
@@ -70,6 +70,8 @@ def parse_args():
     ap.add_argument("--workload", default="mixtral", choices=mw.WORKLOAD_ORDER)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-train", action="store_true",
+                    help="skip the training leg (forward with saved state + backward)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (profiling of smaller cases)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -384,6 +386,12 @@ def run_ours(args, rank, world, local):
         e2e = {"value": replica_throughput(world, T, args.steps, e2e_total), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": int(x_h.numel() * 2), "d2h_bytes_per_step": int(out_h.numel() * 2)}
 
+    # ---- training leg: moe_layer_fwd_train + moe_layer_bwd (not in the timed region above)
+    train = None
+    if not args.no_train:
+        train = train_leg(moe, cfg, w, x, gamma, Wr, bias, W1, W3, W2, stream, args.steps, nf, sampler,
+                          barrier, world)
+
     clocks = sampler.stop()
     code = moe.moe_get_device_error(ws, stream=stream, raise_on_error=False)
 
@@ -433,6 +441,8 @@ def run_ours(args, rank, world, local):
     }
     if e2e is not None:
         result["e2e"] = e2e
+    if train is not None:
+        result["train"] = train
     if world > 1:
         dist.barrier()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -441,6 +451,62 @@ def run_ours(args, rank, world, local):
         print(json.dumps(result), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def train_leg(moe, cfg, w, x, gamma, Wr, bias, W1, W3, W2, stream, steps, nf, sampler, barrier, world):
+    """Times the training forward (saving r, routing, U, V, H, y) and the
+    backward separately with CUDA events; inputs resident, gradients fp32."""
+    import torch
+    T, d, E, F = w.T, w.d_model, w.E, cfg.F
+    tws = moe.alloc_train_workspace(cfg)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(11)
+    dout = torch.randn((T, d), generator=gen, device="cuda").to(torch.bfloat16)
+    G = [torch.empty((T, d), **f32), torch.empty((d,), **f32), torch.empty((d, E), **f32),
+         torch.empty((E,), **f32), torch.empty((d, F), **f32), torch.empty((d, F), **f32),
+         torch.empty((F, d), **f32)]
+
+    def fwd():
+        moe.moe_layer_fwd_train(cfg, x, gamma, Wr, bias, W1, W3, W2, out, tws, stream=stream)
+
+    def bwd():
+        moe.moe_layer_bwd(cfg, x, gamma, Wr, bias, W1, W3, W2, dout, *G, tws, stream=stream)
+
+    for _ in range(3):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    n = max(min(steps, 20), 3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    barrier()
+    torch.cuda.synchronize()
+    tw0 = time.time()
+    for ev in evs:
+        ev[0].record(stream)
+        fwd()
+        ev[1].record(stream)
+        bwd()
+        ev[2].record(stream)
+    torch.cuda.synchronize()
+    sampler.window(tw0, time.time())
+    barrier()
+    fwd_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs) / n, world, "cuda")
+    bwd_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in evs) / n, world, "cuda")
+    code = moe.moe_get_device_error(tws, stream=stream, raise_on_error=False)
+    peaks = load_peaks()
+    # dS (2 d nf) + dX (4 d nf) + dW1|dW3 (4 d nf) + dW2 (2 d nf) + router dWr and dX (4 T d E)
+    fl_bwd = 12.0 * d * nf + 4.0 * T * d * E
+    res = {"fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "step_ms": fwd_ms + bwd_ms,
+           "tokens_per_s": world * T / ((fwd_ms + bwd_ms) * 1e-3),
+           "bwd_flops": fl_bwd, "bwd_tflops": fl_bwd / (bwd_ms * 1e-3) / 1e12,
+           "bwd_frac": fl_bwd / (bwd_ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
+           "peak_note": f"{peaks['source']} sustained cuBLAS bf16", "steps": n,
+           "grad_dtype": "f32", "device_error": code}
+    del tws, G
+    torch.cuda.empty_cache()
+    return res
 
 
 # ----------------------------------------------------------------- oracle legs

@@ -12,9 +12,9 @@ What it computes, in the order the sources give it:
    that follows the norm, so it can be applied in that GEMM's epilogue).
 2. Router: a plain linear layer on the normalised token,
    l_te = r_t * sum_i x_ti gamma_i Wr_ie + b_e, with r applied after the GEMM
-   and before the top-k (CODA thread: the router is "a normal GEMM right after
-   the RMSNorm" with the r-scale fused right before the top-k; MoE glossary,
-   "gating network").
+   and before the top-k (CODA thread: the router is a plain GEMM that follows
+   the RMSNorm, so its epilogue applies the r-scale just ahead of the top-k;
+   MoE glossary, "gating network").
 3. Top-k gating: the k experts with the largest logits (MoE glossary,
    "Top-k Gating" / "Switch Routing"); ties go to the lower expert index and
    the k slots are in descending logit order (the sources are silent; this is
