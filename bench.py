@@ -67,7 +67,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mixtral", choices=mw.WORKLOAD_ORDER)
+    ap.add_argument("--workload", default="mixtral",
+                    choices=mw.WORKLOAD_ORDER + sorted(mw.PROFILE_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-train", action="store_true",

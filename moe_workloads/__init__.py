@@ -102,6 +102,17 @@ WORKLOADS: Dict[str, Workload] = {
 
 WORKLOAD_ORDER = ["tiny", "switch_capacity", "variable_size", "fine_grained", "mixtral"]
 
+# Small cases for profiler captures: the per-tile work of a full-size
+# workload (same d and expert width) with few experts, so that a multi-pass
+# capture holds a few GB on the device.
+PROFILE_WORKLOADS: Dict[str, Workload] = {
+    "mixtral_2e": Workload("mixtral_2e", T=4096, d_model=4096, E=2, k=1,
+                           expert_sizes=((2, 14336),),
+                           description="two Mixtral-shaped experts: T=4096, d=4096, E=2, "
+                                       "top-1, d_ffn=14336 (profiling case)"),
+}
+WORKLOADS.update(PROFILE_WORKLOADS)
+
 
 def _philox(seed: int, stream: int) -> np.random.Generator:
     return np.random.Generator(np.random.Philox(key=[int(seed), int(stream)]))

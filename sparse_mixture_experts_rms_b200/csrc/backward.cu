@@ -191,21 +191,34 @@ __global__ void __launch_bounds__(kBwdNormCols) bwd_norm_kernel(const BwdArgs a)
       s_coef[i] = r * r * r / static_cast<float>(d) * a.dr[tb + i];
     }
     __syncthreads();
-    for (int i = 0; i < nt; ++i) {
-      const size_t t = static_cast<size_t>(tb + i);
-      const float xv = __bfloat162float(a.x[t * d + c]);
-      float dxg = 0.f;
-      for (int j = 0; j < k; ++j) {
-        const int p = s_pos[i][j];
-        if (p >= 0) dxg += a.dXp[static_cast<size_t>(p) * d + c];
+    // 8 tokens at a time: their loads are independent, so they are in flight together
+    for (int i0 = 0; i0 < nt; i0 += 8) {
+      float xv[8], dxg[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u;
+        xv[u] = 0.f;
+        dxg[u] = 0.f;
+        if (i < nt) {
+          xv[u] = __bfloat162float(__ldg(a.x + static_cast<size_t>(tb + i) * d + c));
+          for (int j = 0; j < k; ++j) {
+            const int p = s_pos[i][j];
+            if (p >= 0) dxg[u] += __ldg(a.dXp + static_cast<size_t>(p) * d + c);
+          }
+        }
       }
 #pragma unroll
-      for (int e = 0; e < EMAX; ++e) dxg += s_rdl[i][e < E ? e : 0] * (e < E ? wr[e] : 0.f);
-      a.dx[t * d + c] = gam * dxg - s_coef[i] * xv;
-      acc_g += dxg * xv;
-      const float xg = xv * gam;
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u;
+        if (i >= nt) break;
 #pragma unroll
-      for (int e = 0; e < EMAX; ++e) acc_w[e] += xg * (e < E ? s_rdl[i][e] : 0.f);
+        for (int e = 0; e < EMAX; ++e) dxg[u] += s_rdl[i][e < E ? e : 0] * (e < E ? wr[e] : 0.f);
+        a.dx[static_cast<size_t>(tb + i) * d + c] = gam * dxg[u] - s_coef[i] * xv[u];
+        acc_g += dxg[u] * xv[u];
+        const float xg = xv[u] * gam;
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) acc_w[e] += xg * (e < E ? s_rdl[i][e] : 0.f);
+      }
     }
   }
   a.dgamma_part[static_cast<size_t>(blockIdx.y) * d + c] = acc_g;

@@ -301,6 +301,17 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
     float dr = 0.f;
 #pragma unroll 1
     for (int cc = 0; cc < a.bn; cc += 32) {
+      // the saved U, V of this chunk are fetched while the accumulator is read
+      uint4 ur[4], vr[4];
+      if (valid && !pad) {
+        const uint4* u4 = reinterpret_cast<const uint4*>(a.in_u + off + cc);
+        const uint4* v4 = reinterpret_cast<const uint4*>(a.in_v + off + cc);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          ur[j] = u4[j];
+          vr[j] = v4[j];
+        }
+      }
       uint32_t g[32];
       tmem_ld_32x32b_x32(taddr + cc, g);
       tmem_ld_wait();
@@ -311,13 +322,10 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
         continue;
       }
       uint32_t uw[16], vw[16];
-      const uint4* u4 = reinterpret_cast<const uint4*>(a.in_u + off + cc);
-      const uint4* v4 = reinterpret_cast<const uint4*>(a.in_v + off + cc);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint4 x = u4[j], y = v4[j];
-        uw[4 * j] = x.x; uw[4 * j + 1] = x.y; uw[4 * j + 2] = x.z; uw[4 * j + 3] = x.w;
-        vw[4 * j] = y.x; vw[4 * j + 1] = y.y; vw[4 * j + 2] = y.z; vw[4 * j + 3] = y.w;
+        uw[4 * j] = ur[j].x; uw[4 * j + 1] = ur[j].y; uw[4 * j + 2] = ur[j].z; uw[4 * j + 3] = ur[j].w;
+        vw[4 * j] = vr[j].x; vw[4 * j + 1] = vr[j].y; vw[4 * j + 2] = vr[j].z; vw[4 * j + 3] = vr[j].w;
       }
       uint32_t o1[16], o3[16];
 #pragma unroll
