@@ -191,21 +191,26 @@ __global__ void __launch_bounds__(kBwdNormCols) bwd_norm_kernel(const BwdArgs a)
       s_coef[i] = r * r * r / static_cast<float>(d) * a.dr[tb + i];
     }
     __syncthreads();
-    // 8 tokens at a time: their loads are independent, so they are in flight together
+    // 8 tokens at a time: per slot, the 8 tokens' loads are all issued before any
+    // is used, so they are in flight together
     for (int i0 = 0; i0 < nt; i0 += 8) {
       float xv[8], dxg[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int i = i0 + u;
-        xv[u] = 0.f;
+        xv[u] = i < nt ? __bfloat162float(__ldg(a.x + static_cast<size_t>(tb + i) * d + c)) : 0.f;
         dxg[u] = 0.f;
-        if (i < nt) {
-          xv[u] = __bfloat162float(__ldg(a.x + static_cast<size_t>(tb + i) * d + c));
-          for (int j = 0; j < k; ++j) {
-            const int p = s_pos[i][j];
-            if (p >= 0) dxg[u] += __ldg(a.dXp + static_cast<size_t>(p) * d + c);
-          }
+      }
+      for (int j = 0; j < k; ++j) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u;
+          const int p = i < nt ? s_pos[i][j] : -1;
+          v[u] = p >= 0 ? __ldg(a.dXp + static_cast<size_t>(p) * d + c) : 0.f;
         }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) dxg[u] += v[u];
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {

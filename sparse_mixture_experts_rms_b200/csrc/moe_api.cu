@@ -118,7 +118,7 @@ Layout layout_of(const moe_config_t& c, bool train = false) {
   if (train) {
     const size_t T = static_cast<size_t>(c.T), d = static_cast<size_t>(c.d_model);
     const size_t E = static_cast<size_t>(c.E);
-    L.ld_drp = fmax / kBlockN;
+    L.ld_drp = fmax / kBlockN;  // one dr partial per N tile of the dS GEMM
     L.route_blocks = (c.T + kBwdRouteTokens - 1) / kBwdRouteTokens;
     // bwd_norm grid: d/128 column slices x chunks, about 1024 CTAs
     const int slices = c.d_model / kBwdNormCols;

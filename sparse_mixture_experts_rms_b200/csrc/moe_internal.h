@@ -87,7 +87,7 @@ struct GemmArgs {
   const __nv_bfloat16* in_v;
   __nv_bfloat16* out_ds;    // bwd_h: dS = r*du, dS3 = r*dv [rows, ld_out]
   __nv_bfloat16* out_ds3;
-  float* drp;               // bwd_h: [rows, ld_drp] per-N-tile partials of dr
+  float* drp;               // bwd_h: [rows, ld_drp] partials of dr, one per N tile
   int ld_drp;
   float* out_f0;            // bwd_x: dX [rows, d]; wgrad_x: dW1 [d, F]; wgrad_h: dW2 [F, d]
   float* out_f1;            // wgrad_x: dW3 [d, F]
