@@ -71,6 +71,8 @@ def parse_args():
                     choices=mw.WORKLOAD_ORDER + sorted(mw.PROFILE_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--host-chunks", type=int, default=0,
+                    help="token chunks of the host-buffer call in the e2e leg (0: library default)")
     ap.add_argument("--no-train", action="store_true",
                     help="skip the training leg (forward with saved state + backward)")
     ap.add_argument("--tokens", type=int, default=0,
@@ -357,14 +359,16 @@ def run_ours(args, rank, world, local):
     # ---- end to end through the public call, host buffers, copies inside the timed region
     e2e = None
     if not args.no_e2e:
+        # the public host-buffer call: pinned x in, pinned out back, copies
+        # pipelined with the compute over token chunks inside the call
         x_h = x.cpu().pin_memory()
         out_h = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
-        x_d = torch.empty_like(x)
+        ws_h = moe.alloc_host_workspace(cfg, args.host_chunks)
+        n_chunks = moe.moe_host_chunks(cfg, args.host_chunks)
 
         def e2e_step():
-            x_d.copy_(x_h, non_blocking=True)
-            moe.moe_layer_fwd(cfg, x_d, gamma, Wr, bias, W1, W3, W2, out, ws, stream=stream)
-            out_h.copy_(out, non_blocking=True)
+            moe.moe_layer_fwd_host(cfg, x_h, gamma, Wr, bias, W1, W3, W2, out_h, ws_h,
+                                   n_chunks=args.host_chunks, stream=stream)
 
         with torch.cuda.stream(stream):
             for _ in range(2):
@@ -384,8 +388,11 @@ def run_ours(args, rank, world, local):
         barrier()
         e2e_total = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
         e2e_ms = e2e_total / args.steps
+        e2e_err = moe.moe_get_device_error(ws_h, stream=stream, raise_on_error=False)
         e2e = {"value": replica_throughput(world, T, args.steps, e2e_total), "unit": UNIT, "ms_per_step": e2e_ms,
-               "h2d_bytes_per_step": int(x_h.numel() * 2), "d2h_bytes_per_step": int(out_h.numel() * 2)}
+               "h2d_bytes_per_step": int(x_h.numel() * 2), "d2h_bytes_per_step": int(out_h.numel() * 2),
+               "call": "moe_layer_fwd_host", "chunks": n_chunks, "device_error": e2e_err}
+        del ws_h
 
     # ---- training leg: moe_layer_fwd_train + moe_layer_bwd (not in the timed region above)
     train = None

@@ -253,6 +253,33 @@ MOE_API moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x,
                            int32_t* expert_idx, float* gate, float* r, int32_t* counts,
                            float* prob_mean, float* stats, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- the layer on HOST buffers: copies in and out pipelined with the compute
+ *
+ * moe_layer_fwd with x and out in host memory (pinned memory, e.g. from
+ * cudaHostAlloc, lets the copies overlap; pageable memory works but does not
+ * overlap).  Without a capacity limit a token's output depends only on that
+ * token, so the batch is cut into n_chunks chunks (sizes in the ratio
+ * 1 : 2 : ... : 2 : 1, since only the first copy in and the last copy out are
+ * exposed) and the copy of chunk i+1 in and of chunk i-1 out run on the library's own
+ * copy streams while the layer runs on chunk i: out is bit-identical to
+ * moe_layer_fwd on the whole batch.  With a capacity limit (capacity_factor >
+ * 0) the drops depend on every token's rank, so the batch is one chunk.
+ * n_chunks <= 0 picks the default (3); at most 64, at most T.  Asynchronous on `stream`: when the
+ * stream reaches this point, out_host holds the result; x_host and out_host
+ * must stay valid until then.  The workspace (moe_host_workspace_size for the
+ * same n_chunks) holds one chunk's layer workspace, whose first 256 bytes
+ * carry the device error word (moe_get_device_error works on it), and the
+ * double-buffered device staging of x and out.  Calls on one device are
+ * serialised while they enqueue (the copy streams are per device). */
+MOE_API size_t moe_host_workspace_size(const moe_config_t* cfg, int32_t n_chunks);
+/* Chunks moe_layer_fwd_host will use for `cfg` and n_chunks (-1 if invalid). */
+MOE_API int32_t moe_host_chunks(const moe_config_t* cfg, int32_t n_chunks);
+MOE_API moe_status_t moe_layer_fwd_host(const moe_config_t* cfg, const moe_bf16_t* x_host,
+                                        const moe_bf16_t* gamma, const moe_bf16_t* Wr, const float* bias,
+                                        const moe_bf16_t* W1, const moe_bf16_t* W3, const moe_bf16_t* W2,
+                                        moe_bf16_t* out_host, int32_t n_chunks, void* ws, size_t ws_bytes,
+                                        void* stream);
+
 /* ---- training: forward that saves what the backward reads, and the backward
  *
  * CODA sparse-MoE thread (digg.com): the RMSNorm backward is fused into the

@@ -42,7 +42,8 @@ EXPORTED = ["moe_status_string", "moe_capacity", "moe_max_kept", "moe_workspace_
             "moe_dispatch_noalloc",
             "moe_experts_fwd", "moe_experts_up", "moe_experts_down", "moe_combine",
             "moe_layer_fwd", "moe_router_stats", "moe_train_workspace_size", "moe_train_rows",
-            "moe_train_saved", "moe_layer_fwd_train", "moe_layer_bwd"]
+            "moe_train_saved", "moe_layer_fwd_train", "moe_layer_bwd",
+            "moe_host_workspace_size", "moe_host_chunks", "moe_layer_fwd_host"]
 
 # ids of moe_train_saved
 MOE_SAVED = {"r": 0, "idx": 1, "gate": 2, "logits": 3, "offsets": 4, "perm": 5, "inv_perm": 6,
@@ -115,6 +116,12 @@ def _lib():
         lib.moe_combine.argtypes = [cfgp, P, P, P, P]
         lib.moe_layer_fwd.restype = ctypes.c_int
         lib.moe_layer_fwd.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_host_workspace_size.restype = SZ
+        lib.moe_host_workspace_size.argtypes = [cfgp, ctypes.c_int32]
+        lib.moe_host_chunks.restype = ctypes.c_int32
+        lib.moe_host_chunks.argtypes = [cfgp, ctypes.c_int32]
+        lib.moe_layer_fwd_host.restype = ctypes.c_int
+        lib.moe_layer_fwd_host.argtypes = [cfgp, P, P, P, P, P, P, P, P, ctypes.c_int32, P, SZ, P]
         lib.moe_train_workspace_size.restype = SZ
         lib.moe_train_workspace_size.argtypes = [cfgp]
         lib.moe_train_rows.restype = ctypes.c_int64
@@ -386,6 +393,45 @@ def moe_layer_fwd(cfg: MoEConfig, x, gamma, Wr, bias, W1, W3, W2, out, ws: torch
         _ptr(prob_mean, "prob_mean", f32, (E,)), _ptr(stats, "stats", f32, (4,)),
         _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
     _check(st, "moe_layer_fwd")
+
+
+# ------------------------------------------------------------------ host buffers
+def _host_ptr(t: torch.Tensor, name: str, dtype, shape) -> ctypes.c_void_p:
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def moe_host_workspace_size(cfg: MoEConfig, n_chunks: int = 0) -> int:
+    return int(_lib().moe_host_workspace_size(ctypes.byref(cfg.c()), int(n_chunks)))
+
+
+def moe_host_chunks(cfg: MoEConfig, n_chunks: int = 0) -> int:
+    return int(_lib().moe_host_chunks(ctypes.byref(cfg.c()), int(n_chunks)))
+
+
+def alloc_host_workspace(cfg: MoEConfig, n_chunks: int = 0, device=None, stream=None) -> torch.Tensor:
+    n = moe_host_workspace_size(cfg, n_chunks)
+    if n == 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_host_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    moe_workspace_init(ws, stream)
+    return ws
+
+
+def moe_layer_fwd_host(cfg: MoEConfig, x_host, gamma, Wr, bias, W1, W3, W2, out_host,
+                       ws: torch.Tensor, n_chunks: int = 0, stream=None) -> None:
+    """The layer on host x/out (pin them for overlapped copies); see moe.h."""
+    T, d, E, F = cfg.T, cfg.d_model, cfg.E, cfg.F
+    bf, f32 = torch.bfloat16, torch.float32
+    st = _lib().moe_layer_fwd_host(
+        ctypes.byref(cfg.c()), _host_ptr(x_host, "x_host", bf, (T, d)), _ptr(gamma, "gamma", bf, (d,)),
+        _ptr(Wr, "Wr", bf, (d, E)), _ptr(bias, "bias", f32, (E,)), _ptr(W1, "W1", bf, (d, F)),
+        _ptr(W3, "W3", bf, (d, F)), _ptr(W2, "W2", bf, (F, d)), _host_ptr(out_host, "out_host", bf, (T, d)),
+        int(n_chunks), _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
+    _check(st, "moe_layer_fwd_host")
 
 
 # ------------------------------------------------------------------ training

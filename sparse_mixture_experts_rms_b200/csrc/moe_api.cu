@@ -4,6 +4,7 @@
 // moe_get_device_error.
 #include <cmath>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "moe_internal.h"
@@ -409,6 +410,110 @@ moe_status_t noalloc_scratch(int32_t** out) {
   return MOE_OK;
 }
 
+// ---- the layer on device buffers (cfg validated, T > 0, pointers checked)
+moe_status_t run_layer(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x,
+                       const moe_bf16_t* gamma, const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
+                       const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out, int32_t* expert_idx,
+                       float* gate, float* r, int32_t* counts, float* prob_mean, float* stats, int sms,
+                       cudaStream_t s) {
+  moe_status_t st;
+  int32_t* idx_ = expert_idx ? expert_idx : at<int32_t>(ws, L.idx);
+  float* gate_ = gate ? gate : at<float>(ws, L.gate);
+  float* r_ = r ? r : at<float>(ws, L.r);
+  int32_t* counts_ = counts ? counts : at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+  moe_bf16_t* x_perm = at<moe_bf16_t>(ws, L.x_perm);
+  moe_bf16_t* y = at<moe_bf16_t>(ws, L.y);
+  float* pm = prob_mean ? prob_mean : (stats ? at<float>(ws, L.prob_mean) : nullptr);
+  if ((st = run_route(c, x, gamma, Wr, bias, idx_, gate_, r_, nullptr, pm, L, ws, s)) != MOE_OK) return st;
+  if ((st = run_dispatch(c, L, ws, idx_, x, gamma, counts_, offsets, perm, inv_perm, x_perm, sms, s)) != MOE_OK)
+    return st;
+  if ((st = run_experts(c, L, ws, x_perm, r_, gate_, perm, offsets, W1, W3, W2, y, sms, s)) != MOE_OK)
+    return st;
+  if ((st = run_combine(c, y, inv_perm, out, sms, s)) != MOE_OK) return st;
+  if (stats != nullptr)
+    return cuda_status(launch_router_stats(pm, counts_, offsets, stats, c.T, c.E, c.k, s));
+  return MOE_OK;
+}
+
+// ---- host-buffer layer: token chunks pipelined over two copy streams
+//
+// Without a capacity limit a token's output depends on that token alone, so
+// the batch is cut into n token chunks: the copy of chunk i+1 to the device
+// and of chunk i-1 back to the host overlap the layer on chunk i.  Staging buffers are double-buffered in the workspace.  With a capacity
+// limit the drops depend on every token's rank, so the batch is one chunk.
+constexpr int kDefaultHostChunks = 3;  // measured best on the Mixtral-shaped layer (2..8 tried)
+
+struct HostPipe {
+  bool made = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, h2d_done[2] = {nullptr, nullptr}, comp_done[2] = {nullptr, nullptr},
+              d2h_done[2] = {nullptr, nullptr};
+};
+std::mutex g_pipe_mutex[kMaxDevices];
+HostPipe g_pipe[kMaxDevices];
+
+bool make_pipe(HostPipe& p) {
+  if (p.made) return true;
+  bool ok = cudaStreamCreateWithFlags(&p.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&p.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming) == cudaSuccess;
+  for (int b = 0; ok && b < 2; ++b)
+    ok = cudaEventCreateWithFlags(&p.h2d_done[b], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&p.comp_done[b], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&p.d2h_done[b], cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    return false;
+  }
+  p.made = true;
+  return true;
+}
+
+constexpr int kMaxHostChunks = 64;
+
+struct HostLayout {
+  int n;                         // chunks
+  int64_t start[kMaxHostChunks + 1];  // token offsets of the chunks
+  int64_t tc;                    // tokens of the largest chunk
+  size_t layer;                  // bytes of the per-chunk layer workspace (at offset 0)
+  size_t xs[2], os[2], total;
+};
+
+// Chunk sizes in the ratio 1 : 2 : ... : 2 : 1: only the first chunk's copy
+// in and the last chunk's copy out are not hidden behind compute, so those two
+// are half the size of the others.
+HostLayout host_layout_of(const moe_config_t& c, int n_chunks) {
+  HostLayout H{};
+  int n = n_chunks > 0 ? n_chunks : kDefaultHostChunks;
+  if (capacity_of(c) >= 0) n = 1;          // capacity ranks span the whole batch
+  if (n > kMaxHostChunks) n = kMaxHostChunks;
+  if (n > c.T) n = c.T > 0 ? c.T : 1;
+  const int64_t wsum = n <= 2 ? n : 2 * n - 2;
+  int64_t acc = 0;
+  H.start[0] = 0;
+  for (int i = 0; i < n; ++i) {
+    acc += (n <= 2 || i == 0 || i == n - 1) ? 1 : 2;
+    H.start[i + 1] = (static_cast<int64_t>(c.T) * acc) / wsum;
+  }
+  for (int i = 1; i < n; ++i)  // no empty chunk (n <= T leaves room for one token each)
+    H.start[i] = std::min<int64_t>(std::max<int64_t>(H.start[i], H.start[i - 1] + 1), c.T - (n - i));
+  H.n = n;
+  H.tc = 0;
+  for (int i = 0; i < n; ++i) H.tc = std::max<int64_t>(H.tc, H.start[i + 1] - H.start[i]);
+  moe_config_t cc = c;
+  cc.T = static_cast<int32_t>(H.tc);
+  H.layer = align_up(layout_of(cc).total, 1024);
+  const size_t chunk_bytes = align_up(static_cast<size_t>(H.tc) * c.d_model * 2, 1024);
+  size_t off = H.layer;
+  for (int b = 0; b < 2; ++b) { H.xs[b] = off; off += chunk_bytes; }
+  for (int b = 0; b < 2; ++b) { H.os[b] = off; off += chunk_bytes; }
+  H.total = off;
+  return H;
+}
+
 // ---- training backward: gather -> bwd_h -> bwd_x -> weight gradients ->
 // router/statistic backward -> norm backward -> reductions, on one stream.
 moe_status_t run_backward(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x,
@@ -785,27 +890,8 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x, const m
   if ((st = check_ws(*cfg, ws, ws_bytes, &L)) != MOE_OK) return st;
   int sms;
   if ((st = device_ready(&sms)) != MOE_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const moe_config_t& c = *cfg;
-  int32_t* idx_ = expert_idx ? expert_idx : at<int32_t>(ws, L.idx);
-  float* gate_ = gate ? gate : at<float>(ws, L.gate);
-  float* r_ = r ? r : at<float>(ws, L.r);
-  int32_t* counts_ = counts ? counts : at<int32_t>(ws, L.counts);
-  int32_t* offsets = at<int32_t>(ws, L.offsets);
-  int32_t* perm = at<int32_t>(ws, L.perm);
-  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
-  moe_bf16_t* x_perm = at<moe_bf16_t>(ws, L.x_perm);
-  moe_bf16_t* y = at<moe_bf16_t>(ws, L.y);
-  float* pm = prob_mean ? prob_mean : (stats ? at<float>(ws, L.prob_mean) : nullptr);
-  if ((st = run_route(c, x, gamma, Wr, bias, idx_, gate_, r_, nullptr, pm, L, ws, s)) != MOE_OK) return st;
-  if ((st = run_dispatch(c, L, ws, idx_, x, gamma, counts_, offsets, perm, inv_perm, x_perm, sms, s)) != MOE_OK)
-    return st;
-  if ((st = run_experts(c, L, ws, x_perm, r_, gate_, perm, offsets, W1, W3, W2, y, sms, s)) != MOE_OK)
-    return st;
-  if ((st = run_combine(c, y, inv_perm, out, sms, s)) != MOE_OK) return st;
-  if (stats != nullptr)
-    return cuda_status(launch_router_stats(pm, counts_, offsets, stats, c.T, c.E, c.k, s));
-  return MOE_OK;
+  return run_layer(*cfg, L, ws, x, gamma, Wr, bias, W1, W3, W2, out, expert_idx, gate, r, counts, prob_mean,
+                   stats, sms, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_router_stats(const moe_config_t* cfg, const float* prob_mean, const int32_t* counts,
@@ -820,6 +906,78 @@ moe_status_t moe_router_stats(const moe_config_t* cfg, const float* prob_mean, c
   if ((st = device_ready(&sms)) != MOE_OK) return st;
   return cuda_status(launch_router_stats(prob_mean, counts, expert_offsets, stats, cfg->T, cfg->E, cfg->k,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_host_workspace_size(const moe_config_t* cfg, int32_t n_chunks) {
+  if (validate(cfg) != MOE_OK) return 0;
+  return host_layout_of(*cfg, n_chunks).total;
+}
+
+int32_t moe_host_chunks(const moe_config_t* cfg, int32_t n_chunks) {
+  if (validate(cfg) != MOE_OK) return -1;
+  return host_layout_of(*cfg, n_chunks).n;
+}
+
+moe_status_t moe_layer_fwd_host(const moe_config_t* cfg, const moe_bf16_t* x_host, const moe_bf16_t* gamma,
+                                const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
+                                const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out_host,
+                                int32_t n_chunks, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config_t& c = *cfg;
+  if (c.T == 0) return MOE_OK;
+  if (!x_host || !gamma || !Wr || !W1 || !W3 || !W2 || !out_host) return MOE_ERR_INVALID_ARG;
+  if (!aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) || !aligned(W1, 16) || !aligned(W3, 16) ||
+      !aligned(W2, 16) || !aligned(x_host, 2) || !aligned(out_host, 2))
+    return MOE_ERR_ALIGNMENT;
+  const HostLayout H = host_layout_of(c, n_chunks);
+  if (ws == nullptr || ws_bytes < H.total) return MOE_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGNMENT;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(g_pipe_mutex[dev]);
+  HostPipe& P = g_pipe[dev];
+  if (!make_pipe(P)) return MOE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t row_bytes = static_cast<size_t>(c.d_model) * 2;
+  const char* xh = reinterpret_cast<const char*>(x_host);
+  char* oh = reinterpret_cast<char*>(out_host);
+  cudaError_t e = cudaEventRecord(P.start, s);  // copies start after earlier work on `stream`
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(P.h2d, P.start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(P.d2h, P.start, 0);
+  if (e != cudaSuccess) return cuda_status(e);
+  for (int i = 0; i < H.n; ++i) {
+    const int b = i & 1;
+    const int64_t t0 = H.start[i];
+    const int64_t ti = H.start[i + 1] - t0;  // >= 1: n <= T
+    moe_config_t ci = c;
+    ci.T = static_cast<int32_t>(ti);
+    const Layout Li = layout_of(ci);
+    moe_bf16_t* xs = at<moe_bf16_t>(ws, H.xs[b]);
+    moe_bf16_t* os = at<moe_bf16_t>(ws, H.os[b]);
+    const size_t bytes = static_cast<size_t>(ti) * row_bytes;
+    if (i >= 2) e = cudaStreamWaitEvent(P.h2d, P.comp_done[b], 0);  // xs[b] read by chunk i-2
+    if (e == cudaSuccess) e = cudaMemcpyAsync(xs, xh + t0 * row_bytes, bytes, cudaMemcpyHostToDevice, P.h2d);
+    if (e == cudaSuccess) e = cudaEventRecord(P.h2d_done[b], P.h2d);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, P.h2d_done[b], 0);
+    if (e == cudaSuccess && i >= 2) e = cudaStreamWaitEvent(s, P.d2h_done[b], 0);  // os[b] copied out
+    if (e != cudaSuccess) return cuda_status(e);
+    // the chunk's layer workspace: the error word lives in its header (offset 0)
+    if ((st = run_layer(ci, Li, ws, xs, gamma, Wr, bias, W1, W3, W2, os, nullptr, nullptr, nullptr, nullptr,
+                        nullptr, nullptr, sms, s)) != MOE_OK)
+      return st;
+    e = cudaEventRecord(P.comp_done[b], s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(P.d2h, P.comp_done[b], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(oh + t0 * row_bytes, os, bytes, cudaMemcpyDeviceToHost, P.d2h);
+    if (e == cudaSuccess) e = cudaEventRecord(P.d2h_done[b], P.d2h);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  // the caller's stream completes after the last copies out
+  e = cudaStreamWaitEvent(s, P.d2h_done[(H.n - 1) & 1], 0);
+  if (e == cudaSuccess && H.n >= 2) e = cudaStreamWaitEvent(s, P.d2h_done[H.n & 1], 0);
+  return cuda_status(e);
 }
 
 size_t moe_train_workspace_size(const moe_config_t* cfg) {

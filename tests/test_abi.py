@@ -194,3 +194,29 @@ def test_backward_rejects_bad_arguments_before_device_work(lib):
     assert lib.moe_layer_bwd(ctypes.byref(c.c()), *args, P(1 << 20), n, P(0)) == moe.MOE_ERR_ALIGNMENT
     # a workspace one byte short
     assert lib.moe_layer_bwd(ctypes.byref(c.c()), *ok, P(1 << 20), n - 1, P(0)) == moe.MOE_ERR_WORKSPACE
+
+
+def test_host_pipeline_chunking(lib):
+    """Dropless batches are cut into ceil(T/n)-token chunks with no empty
+    chunk; a capacity limit keeps the batch whole."""
+    mix = _cfg(mw.WORKLOADS["mixtral"])
+    assert moe.moe_host_chunks(mix, 0) == 3
+    assert moe.moe_host_chunks(mix, 3) == 3
+    small = _cfg(mw.WORKLOADS["tiny"].with_tokens(5))
+    assert moe.moe_host_chunks(small, 4) == 4          # 5 tokens, no chunk empty
+    assert moe.moe_host_chunks(small, 99) == 5
+    cap = _cfg(mw.WORKLOADS["switch_capacity"])
+    assert moe.moe_host_chunks(cap, 4) == 1
+    for c, n in ((mix, 4), (small, 4), (cap, 4)):
+        m = moe.moe_host_chunks(c, n)
+        w = [1] * m if m <= 2 else [1] + [2] * (m - 2) + [1]
+        bounds = [c.T * sum(w[:i]) // sum(w) for i in range(m + 1)]
+        for i in range(1, m):
+            bounds[i] = min(max(bounds[i], bounds[i - 1] + 1), c.T - (m - i))
+        assert all(b1 > b0 for b0, b1 in zip(bounds, bounds[1:])), bounds
+        T_c = max(b1 - b0 for b0, b1 in zip(bounds, bounds[1:]))
+        sub = _cfg(mw.WORKLOADS["tiny"])
+        sub.__dict__.update(c.__dict__)
+        sub.T = T_c
+        staging = 4 * T_c * c.d_model * 2
+        assert moe.moe_host_workspace_size(c, n) >= moe.moe_workspace_size(sub) + staging
