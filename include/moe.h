@@ -280,6 +280,64 @@ MOE_API moe_status_t moe_layer_fwd_host(const moe_config_t* cfg, const moe_bf16_
                                         moe_bf16_t* out_host, int32_t n_chunks, void* ws, size_t ws_bytes,
                                         void* stream);
 
+/* ---- MXFP8 expert GEMMs
+ *
+ * CODA sparse-MoE thread (digg.com): with low-precision expert GEMMs, the
+ * conversions of their inputs go into the epilogues of the producing kernels.
+ * Format: OCP Microscaling MXFP8 -- blocks of 32 consecutive values along a
+ * GEMM's reduction share an E8M0 scale 2^e with e = floor(log2 max|v|) - 8,
+ * and each value is v * 2^-e as FP8 E4M3 (round to nearest even, saturating
+ * at 448).  The layer is moe_layer_fwd's (router, dispatch, combine
+ * unchanged) with: x*gamma quantised per token along d by the dispatch, W1/W3
+ * along d and W2 along F by moe_quantize_weights_mx (once per set of
+ * weights), and the SwiGLU output H quantised along the expert width in the
+ * first expert GEMM's epilogue; both expert GEMMs run block-scaled on the
+ * tensor cores with fp32 accumulation; y and out stay bf16.  Each expert's
+ * rows are padded to a multiple of 128 in the workspace. */
+
+/* Bytes of the quantised weights for cfg (0 if invalid): K-major E4M3 copies
+ * of W1, W3 ([F, d]) and W2 ([d, F]) and their scale blocks. */
+MOE_API size_t moe_mx_weights_size(const moe_config_t* cfg);
+/* Quantise W1, W3 [d, F] and W2 [F, d] (bf16, device) into wq (device,
+ * 256-byte aligned, moe_mx_weights_size bytes, caller-owned). */
+MOE_API moe_status_t moe_quantize_weights_mx(const moe_config_t* cfg, const moe_bf16_t* W1,
+                                             const moe_bf16_t* W3, const moe_bf16_t* W2, void* wq,
+                                             size_t wq_bytes, void* stream);
+/* Bytes of workspace for moe_layer_fwd_mx (0 if invalid). */
+MOE_API size_t moe_mx_workspace_size(const moe_config_t* cfg);
+/* Rows of its permuted buffers: max kept + 127 E, rounded up to 128. */
+MOE_API int64_t moe_mx_rows(const moe_config_t* cfg);
+/* The layer with MXFP8 expert GEMMs: arguments as moe_layer_fwd, with the
+ * quantised weights wq in place of W1/W3/W2.  out [T, d] bf16. */
+MOE_API moe_status_t moe_layer_fwd_mx(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
+                                      const moe_bf16_t* Wr, const float* bias, const void* wq,
+                                      size_t wq_bytes, moe_bf16_t* out, void* ws, size_t ws_bytes,
+                                      void* stream);
+/* Device addresses of the MX buffers, for inspection: parts of wq (ids 0-4)
+ * or of the workspace of the last moe_layer_fwd_mx (5-13).  Scale blocks:
+ * 512 bytes per 128 rows x 128 k, block (r/128, k/128) at index
+ * (r/128) * (K/128) + k/128, scale of (r, k) at byte
+ * 16 (r % 32) + 4 ((r % 128) / 32) + (k % 128) / 32 of its block; sf13
+ * interleaves W1 (rows 0-63) and W3 (rows 64-127) columns of 64-column tiles. */
+typedef enum {
+  MOE_MX_W1 = 0,      /* [F, d] E4M3                                          */
+  MOE_MX_W3 = 1,      /* [F, d] E4M3                                          */
+  MOE_MX_W2 = 2,      /* [d, F] E4M3                                          */
+  MOE_MX_SF13 = 3,    /* (F/64) x (d/128) blocks                              */
+  MOE_MX_SF2 = 4,     /* (d/128) x (F/128) blocks                             */
+  MOE_MX_X8 = 5,      /* [rows, d] E4M3                                       */
+  MOE_MX_XSF = 6,     /* (rows/128) x (d/128) blocks                          */
+  MOE_MX_H8 = 7,      /* [rows, f_max] E4M3                                   */
+  MOE_MX_HSF = 8,     /* (rows/128) x (f_max/128) blocks                      */
+  MOE_MX_PERM = 9,    /* [rows] int32, -1 at padding                          */
+  MOE_MX_OFFSETS = 10, /* [E+1] int32 (128-row segments)                      */
+  MOE_MX_IDX = 11,    /* [T, k] int32                                         */
+  MOE_MX_GATE = 12,   /* [T, k] fp32                                          */
+  MOE_MX_R = 13       /* [T] fp32                                             */
+} moe_mx_part_t;
+MOE_API moe_status_t moe_mx_part(const moe_config_t* cfg, void* wq, void* ws, size_t ws_bytes, int32_t which,
+                                 void** ptr);
+
 /* ---- training: forward that saves what the backward reads, and the backward
  *
  * CODA sparse-MoE thread (digg.com): the RMSNorm backward is fused into the

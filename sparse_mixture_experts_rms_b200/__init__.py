@@ -43,7 +43,13 @@ EXPORTED = ["moe_status_string", "moe_capacity", "moe_max_kept", "moe_workspace_
             "moe_experts_fwd", "moe_experts_up", "moe_experts_down", "moe_combine",
             "moe_layer_fwd", "moe_router_stats", "moe_train_workspace_size", "moe_train_rows",
             "moe_train_saved", "moe_layer_fwd_train", "moe_layer_bwd",
-            "moe_host_workspace_size", "moe_host_chunks", "moe_layer_fwd_host"]
+            "moe_host_workspace_size", "moe_host_chunks", "moe_layer_fwd_host",
+            "moe_mx_weights_size", "moe_quantize_weights_mx", "moe_mx_workspace_size", "moe_mx_rows",
+            "moe_layer_fwd_mx", "moe_mx_part"]
+
+# ids of moe_mx_part
+MOE_MX = {"W1": 0, "W3": 1, "W2": 2, "SF13": 3, "SF2": 4, "X8": 5, "XSF": 6, "H8": 7, "HSF": 8,
+          "PERM": 9, "OFFSETS": 10, "IDX": 11, "GATE": 12, "R": 13}
 
 # ids of moe_train_saved
 MOE_SAVED = {"r": 0, "idx": 1, "gate": 2, "logits": 3, "offsets": 4, "perm": 5, "inv_perm": 6,
@@ -116,6 +122,18 @@ def _lib():
         lib.moe_combine.argtypes = [cfgp, P, P, P, P]
         lib.moe_layer_fwd.restype = ctypes.c_int
         lib.moe_layer_fwd.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_mx_weights_size.restype = SZ
+        lib.moe_mx_weights_size.argtypes = [cfgp]
+        lib.moe_quantize_weights_mx.restype = ctypes.c_int
+        lib.moe_quantize_weights_mx.argtypes = [cfgp, P, P, P, P, SZ, P]
+        lib.moe_mx_workspace_size.restype = SZ
+        lib.moe_mx_workspace_size.argtypes = [cfgp]
+        lib.moe_mx_rows.restype = ctypes.c_int64
+        lib.moe_mx_rows.argtypes = [cfgp]
+        lib.moe_layer_fwd_mx.restype = ctypes.c_int
+        lib.moe_layer_fwd_mx.argtypes = [cfgp, P, P, P, P, P, SZ, P, P, SZ, P]
+        lib.moe_mx_part.restype = ctypes.c_int
+        lib.moe_mx_part.argtypes = [cfgp, P, P, SZ, ctypes.c_int32, ctypes.POINTER(ctypes.c_void_p)]
         lib.moe_host_workspace_size.restype = SZ
         lib.moe_host_workspace_size.argtypes = [cfgp, ctypes.c_int32]
         lib.moe_host_chunks.restype = ctypes.c_int32
@@ -393,6 +411,84 @@ def moe_layer_fwd(cfg: MoEConfig, x, gamma, Wr, bias, W1, W3, W2, out, ws: torch
         _ptr(prob_mean, "prob_mean", f32, (E,)), _ptr(stats, "stats", f32, (4,)),
         _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
     _check(st, "moe_layer_fwd")
+
+
+# ------------------------------------------------------------------ MXFP8 expert GEMMs
+def moe_mx_weights_size(cfg: MoEConfig) -> int:
+    return int(_lib().moe_mx_weights_size(ctypes.byref(cfg.c())))
+
+
+def moe_mx_workspace_size(cfg: MoEConfig) -> int:
+    return int(_lib().moe_mx_workspace_size(ctypes.byref(cfg.c())))
+
+
+def moe_mx_rows(cfg: MoEConfig) -> int:
+    return int(_lib().moe_mx_rows(ctypes.byref(cfg.c())))
+
+
+def moe_quantize_weights_mx(cfg: MoEConfig, W1, W3, W2, wq: torch.Tensor, stream=None) -> None:
+    d, F = cfg.d_model, cfg.F
+    bf = torch.bfloat16
+    st = _lib().moe_quantize_weights_mx(
+        ctypes.byref(cfg.c()), _ptr(W1, "W1", bf, (d, F)), _ptr(W3, "W3", bf, (d, F)), _ptr(W2, "W2", bf, (F, d)),
+        _ptr(wq, "wq", torch.uint8), wq.numel(), _stream(stream))
+    _check(st, "moe_quantize_weights_mx")
+
+
+def alloc_mx_weights(cfg: MoEConfig, W1, W3, W2, stream=None) -> torch.Tensor:
+    """The MXFP8 copies of W1, W3, W2 (torch-owned device buffer)."""
+    n = moe_mx_weights_size(cfg)
+    if n == 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_mx_weights_size")
+    wq = torch.empty(n, dtype=torch.uint8, device=W1.device)
+    moe_quantize_weights_mx(cfg, W1, W3, W2, wq, stream)
+    return wq
+
+
+def alloc_mx_workspace(cfg: MoEConfig, device=None, stream=None) -> torch.Tensor:
+    n = moe_mx_workspace_size(cfg)
+    if n == 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_mx_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    moe_workspace_init(ws, stream)
+    return ws
+
+
+def moe_layer_fwd_mx(cfg: MoEConfig, x, gamma, Wr, bias, wq: torch.Tensor, out, ws: torch.Tensor,
+                     stream=None) -> None:
+    T, d, E = cfg.T, cfg.d_model, cfg.E
+    bf, f32 = torch.bfloat16, torch.float32
+    st = _lib().moe_layer_fwd_mx(
+        ctypes.byref(cfg.c()), _ptr(x, "x", bf, (T, d)), _ptr(gamma, "gamma", bf, (d,)),
+        _ptr(Wr, "Wr", bf, (d, E)), _ptr(bias, "bias", f32, (E,)), _ptr(wq, "wq", torch.uint8), wq.numel(),
+        _ptr(out, "out", bf, (T, d)), _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
+    _check(st, "moe_layer_fwd_mx")
+
+
+def mx_part_view(cfg: MoEConfig, wq: torch.Tensor, ws: Optional[torch.Tensor], name: str) -> torch.Tensor:
+    """A view of one MX buffer (weights parts from wq, the rest from ws)."""
+    T, d, E, k, F = cfg.T, cfg.d_model, cfg.E, cfg.k, cfg.F
+    fmax = max(b - a for a, b in zip(cfg.ffn_offsets[:-1], cfg.ffn_offsets[1:]))
+    rows = moe_mx_rows(cfg)
+    u8, i32, f32 = torch.uint8, torch.int32, torch.float32
+    spec = {"W1": (u8, (F, d)), "W3": (u8, (F, d)), "W2": (u8, (d, F)),
+            "SF13": (u8, ((F // 64) * (d // 128) * 512,)), "SF2": (u8, ((d // 128) * (F // 128) * 512,)),
+            "X8": (u8, (rows, d)), "XSF": (u8, ((rows // 128) * (d // 128) * 512,)),
+            "H8": (u8, (rows, fmax)), "HSF": (u8, ((rows // 128) * (fmax // 128) * 512,)),
+            "PERM": (i32, (rows,)), "OFFSETS": (i32, (E + 1,)), "IDX": (i32, (T, k)),
+            "GATE": (f32, (T, k)), "R": (f32, (T,))}[name]
+    out = ctypes.c_void_p(0)
+    base = wq if MOE_MX[name] <= MOE_MX["SF2"] else ws
+    st = _lib().moe_mx_part(ctypes.byref(cfg.c()), _ptr(wq, "wq", torch.uint8),
+                            _ptr(ws, "ws", torch.uint8) if ws is not None else ctypes.c_void_p(0),
+                            ws.numel() if ws is not None else 0, MOE_MX[name], ctypes.byref(out))
+    _check(st, "moe_mx_part")
+    dtype, shape = spec
+    off = int(out.value) - base.data_ptr()
+    n = 1
+    for v in shape:
+        n *= v
+    return base[off:off + n * torch.empty(0, dtype=dtype).element_size()].view(dtype).view(shape)
 
 
 # ------------------------------------------------------------------ host buffers

@@ -21,6 +21,7 @@
 //   permute:  x_perm[p] = bf16(x_t * gamma), t = perm[p] / k, one warp per row,
 //             16-byte loads and stores.
 #include "moe_internal.h"
+#include "mx.cuh"
 
 namespace moe {
 namespace {
@@ -166,6 +167,44 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const DispatchArgs a)
   }
 }
 
+// MX variant: x8[p] = E4M3 codes of x[perm[p]/k] * gamma in 32-column
+// blocks (the product of two bf16 values is exact in fp32), one scale byte
+// per block; zero codes and scales at padding rows.  One warp per row, one
+// block per lane at a time.
+__global__ void __launch_bounds__(256) permute_rows_mx_kernel(const DispatchArgs a) {
+  const int n_rows = min(a.offsets[a.E], a.max_kept);
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  const int nblk = a.d / 32;
+  for (int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; p < n_rows; p += warps) {
+    const int asg = a.perm[p];
+    uint4* dst = reinterpret_cast<uint4*>(a.x8 + static_cast<size_t>(p) * a.d);
+    for (int b = lane; b < nblk; b += 32) {
+      uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      uint32_t sb = 0u;
+      if (asg >= 0) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(asg / a.k) * a.d + b * 32);
+        const uint4* g4 = reinterpret_cast<const uint4*>(a.gamma + b * 32);
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 xv = __ldg(src + j), gv = __ldg(g4 + j);
+          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            v[8 * j + 2 * i] = __uint_as_float(xw[i] << 16) * __uint_as_float(gw[i] << 16);
+            v[8 * j + 2 * i + 1] = __uint_as_float(xw[i] & 0xFFFF0000u) * __uint_as_float(gw[i] & 0xFFFF0000u);
+          }
+        }
+        sb = mx_quantize32(v, w);
+      }
+      dst[2 * b] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[2 * b + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+      a.xsf[mx_sf_offset(p, b * 32, a.d)] = static_cast<uint8_t>(sb);
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_dispatch(const DispatchArgs& a, int num_sms, cudaStream_t s) {
@@ -174,10 +213,13 @@ cudaError_t launch_dispatch(const DispatchArgs& a, int num_sms, cudaStream_t s) 
   const int ntiles = (n + kDispatchTile - 1) / kDispatchTile;
   dispatch_count_kernel<<<ntiles, kDispThreads, 0, s>>>(a);
   dispatch_scatter_kernel<<<ntiles, kDispThreads, 0, s>>>(a, ntiles);
-  if (a.x_perm != nullptr && a.max_kept > 0) {
+  if ((a.x_perm != nullptr || a.x8 != nullptr) && a.max_kept > 0) {
     int grid = (a.max_kept + 7) / 8;
     grid = grid < num_sms * 8 ? grid : num_sms * 8;
-    permute_rows_kernel<<<grid, 256, 0, s>>>(a);
+    if (a.x8 != nullptr)
+      permute_rows_mx_kernel<<<grid, 256, 0, s>>>(a);
+    else
+      permute_rows_kernel<<<grid, 256, 0, s>>>(a);
   }
   return cudaGetLastError();
 }

@@ -41,13 +41,17 @@ struct Layout {
       inv_perm, x_perm, H, y, total;
   // training workspace only
   size_t logits, U, V, yu, dY, dS, dS3, drp, dXp, dgate, rdl, dr, dbias_part, dgamma_part, dWr_part;
+  // MXFP8 workspace only
+  size_t x8, xsf, h8, hsf;
   int64_t max_kept;  // rows of the permuted buffers (padded in the training layout)
   int ldh;
   int ld_drp, chunks, chunk_tokens, route_blocks;
   bool train;
+  bool mx;
 };
 
 constexpr int kTrainRowAlign = 64;  // row-segment padding of the training layout
+constexpr int kMxRowAlign = 128;    // MX path: a CTA's 128 rows are one scale block
 
 int64_t capacity_of(const moe_config_t& c) {
   if (!(c.capacity_factor > 0.0f)) return -1;
@@ -81,9 +85,10 @@ moe_status_t validate(const moe_config_t* c) {
   return MOE_OK;
 }
 
-Layout layout_of(const moe_config_t& c, bool train = false) {
+Layout layout_of(const moe_config_t& c, bool train = false, bool mx = false) {
   Layout L{};
   L.train = train;
+  L.mx = mx;
   size_t off = kHeaderBytes;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -98,6 +103,7 @@ Layout layout_of(const moe_config_t& c, bool train = false) {
     fmax = w > fmax ? w : fmax;
   }
   L.max_kept = max_kept_of(c) + (train ? static_cast<int64_t>(c.E) * (kTrainRowAlign - 1) : 0);
+  if (mx) L.max_kept = (max_kept_of(c) + static_cast<int64_t>(c.E) * (kMxRowAlign - 1) + 127) / 128 * 128;
   L.ldh = fmax;
   const size_t mk = static_cast<size_t>(L.max_kept);
   L.err = 0;
@@ -113,8 +119,16 @@ Layout layout_of(const moe_config_t& c, bool train = false) {
   L.offsets = take(static_cast<size_t>(c.E + 1) * 4);
   L.perm = take(mk * 4);
   L.inv_perm = take(tk * 4);
-  L.x_perm = take(mk * c.d_model * 2);
-  L.H = take(mk * static_cast<size_t>(fmax) * 2);
+  if (mx) {
+    const size_t d = static_cast<size_t>(c.d_model);
+    L.x8 = take(mk * d);
+    L.xsf = take((mk / 128) * (d / 128) * 512);
+    L.h8 = take(mk * static_cast<size_t>(fmax));
+    L.hsf = take((mk / 128) * (static_cast<size_t>(fmax) / 128) * 512);
+  } else {
+    L.x_perm = take(mk * c.d_model * 2);
+    L.H = take(mk * static_cast<size_t>(fmax) * 2);
+  }
   L.y = take(mk * c.d_model * 2);
   if (train) {
     const size_t T = static_cast<size_t>(c.T), d = static_cast<size_t>(c.d_model);
@@ -148,8 +162,9 @@ Layout layout_of(const moe_config_t& c, bool train = false) {
   return L;
 }
 
-moe_status_t check_ws(const moe_config_t& c, void* ws, size_t ws_bytes, Layout* L, bool train = false) {
-  *L = layout_of(c, train);
+moe_status_t check_ws(const moe_config_t& c, void* ws, size_t ws_bytes, Layout* L, bool train = false,
+                      bool mx = false) {
+  *L = layout_of(c, train, mx);
   if (ws == nullptr || ws_bytes < L->total) return MOE_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return MOE_ERR_ALIGNMENT;
   return MOE_OK;
@@ -172,7 +187,7 @@ moe_status_t device_ready(int* sms) {
       return MOE_ERR_NO_DEVICE;
     }
     if (prop.major != 10) return MOE_ERR_NO_DEVICE;
-    if (prepare_grouped_gemm() != cudaSuccess) {
+    if (prepare_grouped_gemm() != cudaSuccess || prepare_grouped_gemm_mx() != cudaSuccess) {
       cudaGetLastError();
       return MOE_ERR_CUDA;
     }
@@ -215,6 +230,29 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D E4M3 (byte) tensor map, 128-byte swizzle, box inner x outer.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                 uint32_t box_inner, uint32_t box_outer) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// MX scale blocks as a [nblocks, 128] array of 32-bit words; one block per box.
+bool make_map_sf(CUtensorMap* m, const void* base, uint64_t nblocks) {
+  const cuuint64_t dims[2] = {128, nblocks};
+  const cuuint64_t strides[1] = {512};
+  const cuuint32_t box[2] = {128, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 moe_status_t cuda_status(cudaError_t e) {
@@ -267,8 +305,11 @@ moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf1
 moe_status_t run_dispatch(const moe_config_t& c, const Layout& L, void* ws, const int32_t* idx,
                           const moe_bf16_t* x, const moe_bf16_t* gamma, int32_t* counts,
                           int32_t* offsets, int32_t* perm, int32_t* inv_perm, moe_bf16_t* x_perm,
-                          int sms, cudaStream_t s, int row_align = 1) {
+                          int sms, cudaStream_t s, int row_align = 1, uint8_t* x8 = nullptr,
+                          uint8_t* xsf = nullptr) {
   DispatchArgs a{};
+  a.x8 = x8;
+  a.xsf = xsf;
   a.idx = idx;
   a.x = reinterpret_cast<const __nv_bfloat16*>(x);
   a.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
@@ -436,6 +477,56 @@ moe_status_t run_layer(const moe_config_t& c, const Layout& L, void* ws, const m
   if (stats != nullptr)
     return cuda_status(launch_router_stats(pm, counts_, offsets, stats, c.T, c.E, c.k, s));
   return MOE_OK;
+}
+
+// ---- the layer with MXFP8 expert GEMMs (cfg validated, T > 0, pointers checked)
+moe_status_t run_layer_mx(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x,
+                          const moe_bf16_t* gamma, const moe_bf16_t* Wr, const float* bias, const MxWeights& q,
+                          moe_bf16_t* out, int sms, cudaStream_t s) {
+  moe_status_t st;
+  int32_t* idx = at<int32_t>(ws, L.idx);
+  float* gate = at<float>(ws, L.gate);
+  float* r = at<float>(ws, L.r);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
+  moe_bf16_t* y = at<moe_bf16_t>(ws, L.y);
+  if ((st = run_route(c, x, gamma, Wr, bias, idx, gate, r, nullptr, nullptr, L, ws, s)) != MOE_OK) return st;
+  if ((st = run_dispatch(c, L, ws, idx, x, gamma, at<int32_t>(ws, L.counts), offsets, perm, inv_perm, nullptr,
+                         sms, s, kMxRowAlign, at<uint8_t>(ws, L.x8), at<uint8_t>(ws, L.xsf))) != MOE_OK)
+    return st;
+  const uint64_t rows = static_cast<uint64_t>(L.max_kept);
+  const uint64_t d = static_cast<uint64_t>(c.d_model);
+  const uint64_t F = static_cast<uint64_t>(c.ffn_offsets[c.E]);
+  const uint64_t ldh = static_cast<uint64_t>(L.ldh);
+  MxGemmArgs g{};
+  g.E = c.E; g.k = c.k; g.d = c.d_model; g.F = static_cast<int>(F);
+  g.rows = static_cast<int>(L.max_kept);
+  g.ldh = L.ldh;
+  g.offsets = offsets;
+  g.perm = perm;
+  g.err = at<uint32_t>(ws, L.err);
+  for (int e = 0; e <= c.E; ++e) g.ffn.off[e] = c.ffn_offsets[e];
+  const int grid = gemm_grid_of_current_device();
+  CUtensorMap mA, mB0, mB1, mSA, mSB;
+  g.up = 1;
+  g.scale = r;
+  g.h8 = at<uint8_t>(ws, L.h8);
+  g.hsf = at<uint8_t>(ws, L.hsf);
+  if (!make_map_u8(&mA, at<void>(ws, L.x8), d, rows, d, 128, 128) || !make_map_u8(&mB0, q.w1, d, F, d, 128, 64) ||
+      !make_map_u8(&mB1, q.w3, d, F, d, 128, 64) || !make_map_sf(&mSA, at<void>(ws, L.xsf), (rows / 128) * (d / 128)) ||
+      !make_map_sf(&mSB, q.sf13, (F / 64) * (d / 128)))
+    return MOE_ERR_CUDA;
+  if ((st = cuda_status(launch_grouped_gemm_mx(g, mA, mB0, mB1, mSA, mSB, grid, s))) != MOE_OK) return st;
+  g.up = 0;
+  g.scale = gate;
+  g.y = reinterpret_cast<__nv_bfloat16*>(y);
+  if (!make_map_u8(&mA, at<void>(ws, L.h8), ldh, rows, ldh, 128, 128) || !make_map_u8(&mB0, q.w2, F, d, F, 128, 64) ||
+      !make_map_sf(&mSA, at<void>(ws, L.hsf), (rows / 128) * (ldh / 128)) ||
+      !make_map_sf(&mSB, q.sf2, (d / 128) * (F / 128)))
+    return MOE_ERR_CUDA;
+  if ((st = cuda_status(launch_grouped_gemm_mx(g, mA, mB0, mB0, mSA, mSB, grid, s))) != MOE_OK) return st;
+  return run_combine(c, y, inv_perm, out, sms, s);
 }
 
 // ---- host-buffer layer: token chunks pipelined over two copy streams
@@ -906,6 +997,90 @@ moe_status_t moe_router_stats(const moe_config_t* cfg, const float* prob_mean, c
   if ((st = device_ready(&sms)) != MOE_OK) return st;
   return cuda_status(launch_router_stats(prob_mean, counts, expert_offsets, stats, cfg->T, cfg->E, cfg->k,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_mx_weights_size(const moe_config_t* cfg) {
+  if (validate(cfg) != MOE_OK) return 0;
+  return mx_weights_bytes(cfg->d_model, cfg->ffn_offsets[cfg->E]);
+}
+
+moe_status_t moe_quantize_weights_mx(const moe_config_t* cfg, const moe_bf16_t* W1, const moe_bf16_t* W3,
+                                     const moe_bf16_t* W2, void* wq, size_t wq_bytes, void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (!W1 || !W3 || !W2 || !wq) return MOE_ERR_INVALID_ARG;
+  if (!aligned(W1, 16) || !aligned(W3, 16) || !aligned(W2, 16) || !aligned(wq, 256)) return MOE_ERR_ALIGNMENT;
+  const int d = cfg->d_model, F = cfg->ffn_offsets[cfg->E];
+  if (wq_bytes < mx_weights_bytes(d, F)) return MOE_ERR_WORKSPACE;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  return cuda_status(launch_quantize_weights_mx(reinterpret_cast<const __nv_bfloat16*>(W1),
+                                                reinterpret_cast<const __nv_bfloat16*>(W3),
+                                                reinterpret_cast<const __nv_bfloat16*>(W2), mx_weights_at(wq, d, F),
+                                                d, F, static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_mx_workspace_size(const moe_config_t* cfg) {
+  if (validate(cfg) != MOE_OK) return 0;
+  return layout_of(*cfg, false, true).total;
+}
+
+int64_t moe_mx_rows(const moe_config_t* cfg) {
+  if (validate(cfg) != MOE_OK) return -1;
+  return layout_of(*cfg, false, true).max_kept;
+}
+
+moe_status_t moe_layer_fwd_mx(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
+                              const moe_bf16_t* Wr, const float* bias, const void* wq, size_t wq_bytes,
+                              moe_bf16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !gamma || !Wr || !wq || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) || !aligned(wq, 256) ||
+      !aligned(out, 16))
+    return MOE_ERR_ALIGNMENT;
+  const int d = cfg->d_model, F = cfg->ffn_offsets[cfg->E];
+  if (wq_bytes < mx_weights_bytes(d, F)) return MOE_ERR_WORKSPACE;
+  Layout L;
+  if ((st = check_ws(*cfg, ws, ws_bytes, &L, false, true)) != MOE_OK) return st;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  return run_layer_mx(*cfg, L, ws, x, gamma, Wr, bias, mx_weights_at(const_cast<void*>(wq), d, F), out, sms,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_mx_part(const moe_config_t* cfg, void* wq, void* ws, size_t ws_bytes, int32_t which,
+                         void** ptr) {
+  if (ptr == nullptr) return MOE_ERR_INVALID_ARG;
+  *ptr = nullptr;
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (which < 0) return MOE_ERR_INVALID_ARG;
+  if (which <= MOE_MX_SF2) {
+    if (wq == nullptr) return MOE_ERR_INVALID_ARG;
+    const MxWeights q = mx_weights_at(wq, cfg->d_model, cfg->ffn_offsets[cfg->E]);
+    uint8_t* parts[] = {q.w1, q.w3, q.w2, q.sf13, q.sf2};
+    *ptr = parts[which];
+    return MOE_OK;
+  }
+  Layout L;
+  if ((st = check_ws(*cfg, ws, ws_bytes, &L, false, true)) != MOE_OK) return st;
+  size_t off;
+  switch (which) {
+    case MOE_MX_X8: off = L.x8; break;
+    case MOE_MX_XSF: off = L.xsf; break;
+    case MOE_MX_H8: off = L.h8; break;
+    case MOE_MX_HSF: off = L.hsf; break;
+    case MOE_MX_PERM: off = L.perm; break;
+    case MOE_MX_OFFSETS: off = L.offsets; break;
+    case MOE_MX_IDX: off = L.idx; break;
+    case MOE_MX_GATE: off = L.gate; break;
+    case MOE_MX_R: off = L.r; break;
+    default: return MOE_ERR_INVALID_ARG;
+  }
+  *ptr = at<void>(ws, off);
+  return MOE_OK;
 }
 
 size_t moe_host_workspace_size(const moe_config_t* cfg, int32_t n_chunks) {

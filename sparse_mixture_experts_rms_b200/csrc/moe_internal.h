@@ -56,9 +56,56 @@ struct DispatchArgs {
   int T, d, E, k;
   int capacity;             // -1: dropless
   int max_kept;             // rows of x_perm
-  int row_align;            // 1: dense segments; 64: each expert's segment padded
-                            // to a multiple of 64 rows (perm = -1, x_perm = 0 there)
+  int row_align;            // 1: dense segments; 64 / 128: each expert's segment
+                            // padded to that multiple (perm = -1, zero rows there)
+  uint8_t* x8;              // MX mode (x_perm == null): E4M3 codes [max_kept, d]
+  uint8_t* xsf;             // MX mode: E8M0 scale blocks of x8 (see mx_sf_offset)
 };
+
+// ---- MXFP8 (OCP MX: 32-element blocks along K, E4M3 codes, E8M0 scales)
+//
+// Scale factors of an operand with rows r and reduction index k are stored in
+// 512-byte blocks of 128 rows x 128 k (4 scales per row), the layout the
+// tensor memory expects: block (r / 128, k / 128) of a [rows, K] operand sits
+// at block index (r / 128) * (K / 128) + k / 128, and inside a block the scale
+// of (r, k) is byte 16 * (r % 32) + 4 * ((r % 128) / 32) + (k % 128) / 32.
+__host__ __device__ inline size_t mx_sf_offset(int64_t r, int64_t k, int64_t K) {
+  return static_cast<size_t>(((r >> 7) * (K >> 7) + (k >> 7)) * 512 + 16 * (r & 31) + 4 * ((r & 127) >> 5) +
+                             ((k & 127) >> 5));
+}
+
+// Quantised expert weights: K-major E4M3 copies and their scale blocks.
+//   w1, w3 [F, d]   (row n = column n of W1 / W3)      w2 [d, F] (row c = column c of W2)
+//   sf13: the up GEMM's B scales, one block per (64-column tile t, k block):
+//         rows 0..63 = W1 columns 64t.., rows 64..127 = W3 columns 64t..;
+//         block index t * (d / 128) + k / 128
+//   sf2:  standard blocks of w2 ([d, F] with K = F)
+struct MxWeights {
+  uint8_t *w1, *w3, *w2, *sf13, *sf2;
+};
+size_t mx_weights_bytes(int d, int F);
+MxWeights mx_weights_at(void* base, int d, int F);
+cudaError_t launch_quantize_weights_mx(const __nv_bfloat16* W1, const __nv_bfloat16* W3,
+                                       const __nv_bfloat16* W2, MxWeights q, int d, int F, cudaStream_t s);
+
+struct MxGemmArgs {
+  int up;                   // 1: x8 x (W1|W3) -> SwiGLU -> H8 (+ scales); 0: H8 x W2 -> gate * y
+  int E, k, d, F;
+  int rows;                 // rows of the permuted buffers (a multiple of 128)
+  int ldh;                  // row stride of H8 (max expert width)
+  const int32_t* offsets;   // [E+1] row segments, multiples of 128
+  const int32_t* perm;      // [rows]; -1 = padding
+  const float* scale;       // up: r [T]; down: gate [T*k]
+  uint8_t* h8;              // up: E4M3 H [rows, ldh]
+  uint8_t* hsf;             // up: scale blocks of h8 (K = ldh)
+  __nv_bfloat16* y;         // down: [rows, d]
+  uint32_t* err;
+  ExpertTable ffn;
+};
+cudaError_t launch_grouped_gemm_mx(const MxGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB0,
+                                   const CUtensorMap& mapB1, const CUtensorMap& mapSFA,
+                                   const CUtensorMap& mapSFB, int grid, cudaStream_t s);
+cudaError_t prepare_grouped_gemm_mx();
 
 // Modes of the grouped GEMM (one kernel template, one instantiation each).
 enum GemmMode : int {

@@ -218,6 +218,28 @@ __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc,
       : "memory");
 }
 
+// Block-scaled pair MMA (kind::mxf8f6f4, E4M3 x E4M3 -> fp32, E8M0 scales per
+// 32 K), issued by the leader CTA.  sfa / sfb: TMEM addresses of the scale
+// factors; bits 31:30 carry the byte (K sub-block) the descriptor's scale ids
+// also name.
+__device__ __forceinline__ void umma_mxf8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Pair copy shared memory -> TMEM of a 32-row x 128-bit block, replicated to
+// the four lane quarters (each CTA copies its own shared memory into its own
+// TMEM); issued by the leader CTA, ordered with its later MMAs.
+__device__ __forceinline__ void tmem_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrive once on the mbarrier at the same shared offset in every CTA of
 // `cta_mask` when all pair MMAs issued so far by this thread are done.
 __device__ __forceinline__ void umma_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {
@@ -298,6 +320,32 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;
   return d;
+}
+
+// Shared-memory descriptor of an unswizzled K-major operand made of 8-row x
+// 16-byte core matrices: sbo = byte distance between core matrices along the
+// rows, lbo = along K (layout SWIZZLE_NONE = 0, version 1).
+__device__ __forceinline__ uint64_t smem_desc_noswz(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
+// Instruction descriptor of tcgen05.mma kind::mxf8f6f4 with block scaling:
+// A and B E4M3 (format 0), both K-major, E8M0 scales (bit 23), shape M x N,
+// scale ids (the byte of the 32-bit TMEM scale word) for B at [4,6), A at [29,31).
+__host__ __device__ constexpr uint32_t umma_idesc_mxf8(uint32_t M, uint32_t N, uint32_t a_sf_id,
+                                                       uint32_t b_sf_id) {
+  return (b_sf_id << 4)             // B scale id
+         | (0u << 7)                // A format: E4M3
+         | (0u << 10)               // B format: E4M3
+         | ((N >> 3) << 17)         // N / 8
+         | (1u << 23)               // scale format: E8M0
+         | ((M >> 4) << 24)         // M / 16
+         | (a_sf_id << 29);         // A scale id
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate, bf16 A and
