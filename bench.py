@@ -73,6 +73,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--host-chunks", type=int, default=0,
                     help="token chunks of the host-buffer call in the e2e leg (0: library default)")
+    ap.add_argument("--no-mx", action="store_true",
+                    help="skip the MXFP8 leg (the layer with block-scaled E4M3 expert GEMMs)")
     ap.add_argument("--no-train", action="store_true",
                     help="skip the training leg (forward with saved state + backward)")
     ap.add_argument("--tokens", type=int, default=0,
@@ -394,6 +396,12 @@ def run_ours(args, rank, world, local):
                "call": "moe_layer_fwd_host", "chunks": n_chunks, "device_error": e2e_err}
         del ws_h
 
+    # ---- MXFP8 leg: the same layer with block-scaled E4M3 expert GEMMs
+    mx = None
+    if not args.no_mx:
+        mx = mx_leg(moe, cfg, w, x, gamma, Wr, bias, W1, W3, W2, stream, args.steps, F_alg, sampler, barrier,
+                    world)
+
     # ---- training leg: moe_layer_fwd_train + moe_layer_bwd (not in the timed region above)
     train = None
     if not args.no_train:
@@ -451,6 +459,8 @@ def run_ours(args, rank, world, local):
         result["e2e"] = e2e
     if train is not None:
         result["train"] = train
+    if mx is not None:
+        result["mx"] = mx
     if world > 1:
         dist.barrier()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -459,6 +469,44 @@ def run_ours(args, rank, world, local):
         print(json.dumps(result), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def mx_leg(moe, cfg, w, x, gamma, Wr, bias, W1, W3, W2, stream, steps, F_alg, sampler, barrier, world):
+    """Times moe_layer_fwd_mx (weights quantised once, outside the timing)."""
+    import torch
+    wq = moe.alloc_mx_weights(cfg, W1, W3, W2)
+    ws = moe.alloc_mx_workspace(cfg)
+    out = torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        moe.moe_layer_fwd_mx(cfg, x, gamma, Wr, bias, wq, out, ws, stream=stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n = max(min(steps, 30), 3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    tw0 = time.time()
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    sampler.window(tw0, time.time())
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda") / n
+    peaks = load_peaks()
+    fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]   # nominal fp8 : bf16 dense ratio 2
+    res = {"ms_per_step": ms, "tokens_per_s": world * w.T / (ms * 1e-3), "tflops": F_alg / (ms * 1e-3) / 1e12,
+           "layer_frac_of_fp8_peak": F_alg / (ms * 1e-3) / 1e12 / fp8_peak,
+           "peak_note": f"fp8 peak = 2 x {peaks['source']} sustained bf16 ({fp8_peak:.0f} TFLOP/s)",
+           "dtype": "mxfp8 expert GEMMs (E4M3, E8M0 per 32), bf16 router/out", "steps": n,
+           "device_error": moe.moe_get_device_error(ws, stream=stream, raise_on_error=False)}
+    del wq, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def train_leg(moe, cfg, w, x, gamma, Wr, bias, W1, W3, W2, stream, steps, nf, sampler, barrier, world):

@@ -313,27 +313,27 @@ MOE_API moe_status_t moe_layer_fwd_mx(const moe_config_t* cfg, const moe_bf16_t*
                                       const moe_bf16_t* Wr, const float* bias, const void* wq,
                                       size_t wq_bytes, moe_bf16_t* out, void* ws, size_t ws_bytes,
                                       void* stream);
-/* Device addresses of the MX buffers, for inspection: parts of wq (ids 0-4)
- * or of the workspace of the last moe_layer_fwd_mx (5-13).  Scale blocks:
+/* Device addresses of the MX buffers, for inspection: parts of wq (ids 0-5)
+ * or of the workspace of the last moe_layer_fwd_mx (6-14).  Scale blocks:
  * 512 bytes per 128 rows x 128 k, block (r/128, k/128) at index
  * (r/128) * (K/128) + k/128, scale of (r, k) at byte
- * 16 (r % 32) + 4 ((r % 128) / 32) + (k % 128) / 32 of its block; sf13
- * interleaves W1 (rows 0-63) and W3 (rows 64-127) columns of 64-column tiles. */
+ * 16 (r % 32) + 4 ((r % 128) / 32) + (k % 128) / 32 of its block. */
 typedef enum {
   MOE_MX_W1 = 0,      /* [F, d] E4M3                                          */
   MOE_MX_W3 = 1,      /* [F, d] E4M3                                          */
   MOE_MX_W2 = 2,      /* [d, F] E4M3                                          */
-  MOE_MX_SF13 = 3,    /* (F/64) x (d/128) blocks                              */
-  MOE_MX_SF2 = 4,     /* (d/128) x (F/128) blocks                             */
-  MOE_MX_X8 = 5,      /* [rows, d] E4M3                                       */
-  MOE_MX_XSF = 6,     /* (rows/128) x (d/128) blocks                          */
-  MOE_MX_H8 = 7,      /* [rows, f_max] E4M3                                   */
-  MOE_MX_HSF = 8,     /* (rows/128) x (f_max/128) blocks                      */
-  MOE_MX_PERM = 9,    /* [rows] int32, -1 at padding                          */
-  MOE_MX_OFFSETS = 10, /* [E+1] int32 (128-row segments)                      */
-  MOE_MX_IDX = 11,    /* [T, k] int32                                         */
-  MOE_MX_GATE = 12,   /* [T, k] fp32                                          */
-  MOE_MX_R = 13       /* [T] fp32                                             */
+  MOE_MX_SF1 = 3,     /* (F/128) x (d/128) blocks of w1                       */
+  MOE_MX_SF3 = 4,     /* (F/128) x (d/128) blocks of w3                       */
+  MOE_MX_SF2 = 5,     /* (d/128) x (F/128) blocks of w2                       */
+  MOE_MX_X8 = 6,      /* [rows, d] E4M3                                       */
+  MOE_MX_XSF = 7,     /* (rows/128) x (d/128) blocks                          */
+  MOE_MX_H8 = 8,      /* [rows, f_max] E4M3                                   */
+  MOE_MX_HSF = 9,     /* (rows/128) x (f_max/128) blocks                      */
+  MOE_MX_PERM = 10,   /* [rows] int32, -1 at padding                          */
+  MOE_MX_OFFSETS = 11, /* [E+1] int32 (128-row segments)                      */
+  MOE_MX_IDX = 12,    /* [T, k] int32                                         */
+  MOE_MX_GATE = 13,   /* [T, k] fp32                                          */
+  MOE_MX_R = 14       /* [T] fp32                                             */
 } moe_mx_part_t;
 MOE_API moe_status_t moe_mx_part(const moe_config_t* cfg, void* wq, void* ws, size_t ws_bytes, int32_t which,
                                  void** ptr);

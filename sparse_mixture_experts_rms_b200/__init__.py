@@ -48,8 +48,8 @@ EXPORTED = ["moe_status_string", "moe_capacity", "moe_max_kept", "moe_workspace_
             "moe_layer_fwd_mx", "moe_mx_part"]
 
 # ids of moe_mx_part
-MOE_MX = {"W1": 0, "W3": 1, "W2": 2, "SF13": 3, "SF2": 4, "X8": 5, "XSF": 6, "H8": 7, "HSF": 8,
-          "PERM": 9, "OFFSETS": 10, "IDX": 11, "GATE": 12, "R": 13}
+MOE_MX = {"W1": 0, "W3": 1, "W2": 2, "SF1": 3, "SF3": 4, "SF2": 5, "X8": 6, "XSF": 7, "H8": 8, "HSF": 9,
+          "PERM": 10, "OFFSETS": 11, "IDX": 12, "GATE": 13, "R": 14}
 
 # ids of moe_train_saved
 MOE_SAVED = {"r": 0, "idx": 1, "gate": 2, "logits": 3, "offsets": 4, "perm": 5, "inv_perm": 6,
@@ -472,7 +472,8 @@ def mx_part_view(cfg: MoEConfig, wq: torch.Tensor, ws: Optional[torch.Tensor], n
     rows = moe_mx_rows(cfg)
     u8, i32, f32 = torch.uint8, torch.int32, torch.float32
     spec = {"W1": (u8, (F, d)), "W3": (u8, (F, d)), "W2": (u8, (d, F)),
-            "SF13": (u8, ((F // 64) * (d // 128) * 512,)), "SF2": (u8, ((d // 128) * (F // 128) * 512,)),
+            "SF1": (u8, ((F // 128) * (d // 128) * 512,)), "SF3": (u8, ((F // 128) * (d // 128) * 512,)),
+            "SF2": (u8, ((d // 128) * (F // 128) * 512,)),
             "X8": (u8, (rows, d)), "XSF": (u8, ((rows // 128) * (d // 128) * 512,)),
             "H8": (u8, (rows, fmax)), "HSF": (u8, ((rows // 128) * (fmax // 128) * 512,)),
             "PERM": (i32, (rows,)), "OFFSETS": (i32, (E + 1,)), "IDX": (i32, (T, k)),

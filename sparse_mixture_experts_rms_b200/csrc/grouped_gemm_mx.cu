@@ -10,17 +10,27 @@
 // nanoMOE notes: variable widths through cumulative offsets.
 //
 //   up    H8[p, n] = MX( silu(r_t * acc1) * (r_t * acc3) ),  acc1 = x8[p] . W1[:, o_e+n] ...
-//         a pair tile is 256 rows x 128 columns: 64 columns of W1 (leader's B
-//         half) and the same 64 of W3 (peer's half)
-//   down  y[p, n] = bf16( gate * (H8[p, :f_e] . W2[o_e + :, n]) ), 128 columns per tile
+//         a pair tile is 256 rows x 256 columns: 128 columns of W1 (leader's B
+//         half) and the same 128 of W3 (peer's half)
+//   down  y[p, n] = bf16( gate * (H8[p, :f_e] . W2[o_e + :, n]) ), 256 columns per tile
+//         (128 when d is not a multiple of 256)
 //
-// Per pipeline stage each CTA holds 128 rows x 128 K of A (16 KB), 64 rows of
-// B (8 KB), and the scale blocks of its A rows and of all 128 B columns
-// (512 B each, the layout tcgen05.cp takes).  The MMA thread copies both
-// scale blocks into TMEM (columns 256..263) and then issues the stage's four
-// K=32 MMAs, naming the scale byte of each; tcgen05 operations of one thread
-// run in order, so the next stage's copy cannot overtake them.  Row segments
-// are padded to 128 rows, so a CTA's 128 rows are one scale block.
+// Per pipeline stage each CTA holds 128 rows x 128 K of A (16 KB), its 128
+// rows of B (16 KB), and the scale blocks of its A rows (512 B) and of all
+// 256 B columns (two 512-B blocks, the layout tcgen05.cp takes).  The MMA
+// thread copies the scale blocks into TMEM (columns 480..491) and then issues
+// the stage's four K=32 MMAs, naming the scale byte of each; tcgen05
+// operations of one thread run in order, so the next stage's copy cannot
+// overtake them.  Row segments are padded to 128 rows, so a CTA's 128 rows
+// are one scale block.
+//
+// N = 256 keeps the shared-memory operand traffic at 12 KB per 64 tensor
+// cycles (N = 128 would need 8 KB per 32 and saturate shared memory).  Two
+// 256-column accumulators and the scales exceed TMEM's 512 columns, so the
+// accumulators overlap by 32 columns: buffer 0 = [0, 256), buffer 1 =
+// [224, 480).  Each epilogue reads the shared 32 columns first and arrives on
+// an "overlap drained" barrier; the next tile's MMAs wait for that (short)
+// and for the full drain of the tile before it in their own buffer.
 #include "moe_internal.h"
 #include "mx.cuh"
 #include "ptx.cuh"
@@ -30,26 +40,28 @@ namespace {
 
 constexpr int BM = 256;
 constexpr int BM_CTA = 128;
-constexpr int BN = 128;                          // pair MMA N
+constexpr int BN = 256;                          // pair MMA N (the down GEMM may use 128)
 constexpr int BK = 128;                          // K per stage (E4M3 bytes per row)
-constexpr int kStages = 8;
+constexpr int kStages = 6;
 constexpr int kABytes = BM_CTA * BK;             // 16 KB
-constexpr int kBBytes = (BN / 2) * BK;           // 8 KB
-constexpr int kSfBytes = 512;
-constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;  // 25 KB, a multiple of 1024
+constexpr int kBBytes = (BN / 2) * BK;           // 16 KB
+constexpr int kSfBytes = 512;                    // one scale block: 128 rows x 4 scales
+constexpr int kLoadBytes = kABytes + kBBytes + 3 * kSfBytes;   // A, B, SFA, 2 x SFB
+constexpr int kStageBytes = (kLoadBytes + 1023) / 1024 * 1024;  // 1024-byte aligned stages
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
-constexpr int kAccCols = BN;                     // two accumulators: columns 0 and 128
-constexpr uint32_t kSfaCol = 256, kSfbCol = 260;
+constexpr uint32_t kBuf1Col = 224;              // accumulators [0, 256) and [224, 480) overlap in [224, 256)
+__device__ __forceinline__ uint32_t buf_col(uint32_t b) { return b ? kBuf1Col : 0u; }
+constexpr uint32_t kSfaCol = 480, kSfbCol = 484; // 4 + 8 scale columns
 constexpr int kEpiWarps = 4;
 constexpr long long kL2GroupBudget = 48ll << 20;
-static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned (128-byte swizzle)");
 
 struct __align__(8) MxShared {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t ovl[2];           // leader: both CTAs' epilogues read the buffer's overlap columns
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -88,11 +100,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 // TMA loads of K block kb of tile c into one stage (this CTA's half); every
-// x coordinate is a multiple of 128 bytes.
+// x coordinate is a multiple of 128 bytes.  Both CTAs load the scales of all
+// the tile's B columns.
 __device__ __forceinline__ void issue_loads(const MxGemmArgs& a, const CUtensorMap* mA, const CUtensorMap* mB0,
                                             const CUtensorMap* mB1, const CUtensorMap* mSFA,
-                                            const CUtensorMap* mSFB, const TileCoord& c, int kb, uint8_t* stage,
-                                            uint32_t bar, int seg_e, int o_e, uint32_t rank) {
+                                            const CUtensorMap* mSFB0, const CUtensorMap* mSFB1, const TileCoord& c,
+                                            int kb, uint8_t* stage, uint32_t bar, int seg_e, int o_e,
+                                            uint32_t rank, int bn) {
   uint8_t* sA = stage;
   uint8_t* sB = stage + kABytes;
   uint8_t* sSFA = sB + kBBytes;
@@ -102,19 +116,37 @@ __device__ __forceinline__ void issue_loads(const MxGemmArgs& a, const CUtensorM
   tma_load_2d_pair(sA, mA, bar, kb * BK, row0);
   tma_load_2d_pair(sSFA, mSFA, bar, 0, (row0 >> 7) * (KA >> 7) + kb);
   if (a.up) {
-    // leader: 64 columns of W1 (w1 rows), peer: the same 64 of W3
-    tma_load_2d_pair(sB, rank == 0 ? mB0 : mB1, bar, kb * BK, o_e + c.nt * (BN / 2));
-    tma_load_2d_pair(sSFB, mSFB, bar, 0, ((o_e >> 6) + c.nt) * (a.d >> 7) + kb);
+    // leader: 128 columns of W1 (w1 rows), peer: the same 128 of W3
+    const int n0 = o_e + c.nt * 128;
+    tma_load_2d_pair(sB, rank == 0 ? mB0 : mB1, bar, kb * BK, n0);
+    const int blk = (n0 >> 7) * (a.d >> 7) + kb;
+    tma_load_2d_pair(sSFB, mSFB0, bar, 0, blk);              // W1 columns' scales
+    tma_load_2d_pair(sSFB + kSfBytes, mSFB1, bar, 0, blk);   // W3 columns' scales
   } else {
-    tma_load_2d_pair(sB, mB0, bar, o_e + kb * BK, c.nt * BN + static_cast<int>(rank) * (BN / 2));
-    tma_load_2d_pair(sSFB, mSFB, bar, 0, c.nt * (a.F >> 7) + (o_e >> 7) + kb);
+    const int n0 = c.nt * bn;
+    tma_load_2d_pair(sB, mB0, bar, o_e + kb * BK, n0 + static_cast<int>(rank) * (bn / 2));
+    const int kblk = (o_e >> 7) + kb;
+    tma_load_2d_pair(sSFB, mSFB0, bar, 0, (n0 >> 7) * (a.F >> 7) + kblk);
+    if (bn == 256) tma_load_2d_pair(sSFB + kSfBytes, mSFB0, bar, 0, ((n0 >> 7) + 1) * (a.F >> 7) + kblk);
   }
 }
 
+// Arrive (once per warp) on the leader's overlap barrier of the buffer just
+// read: the TMEM loads of the overlapping columns have completed.
+__device__ __forceinline__ void signal_overlap(uint32_t ovl_leader, int lane) {
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive_cluster(ovl_leader);
+}
+
 // One thread per accumulator row (TMEM lane); tcgen05.ld is warp-wide, so
-// every lane loads and only the stores are predicated.
+// every lane loads and only the stores are predicated.  Chunks of 32 columns;
+// the chunk holding the buffer's overlap columns (the last for buffer 0, the
+// first for buffer 1) goes first, and the overlap barrier is signalled as
+// soon as it has been read.
 __device__ __forceinline__ void epilogue(const MxGemmArgs& a, const MxShared& sh, const TileCoord& c,
-                                         uint32_t taddr, int row_in_cta, uint32_t rank) {
+                                         uint32_t taddr, int row_in_cta, uint32_t rank, uint32_t buf, int bn,
+                                         uint32_t ovl_leader, int lane) {
   const int p = sh.seg[c.e] + c.mt * BM + static_cast<int>(rank) * BM_CTA + row_in_cta;
   const bool valid = p < sh.seg[c.e + 1];
   const int asg = valid ? a.perm[p] : -1;
@@ -122,21 +154,23 @@ __device__ __forceinline__ void epilogue(const MxGemmArgs& a, const MxShared& sh
   if (a.up) {
     const float r = asg >= 0 ? a.scale[asg / a.k] : 0.f;  // padding rows: r = 0 -> H = 0
 #pragma unroll 1
-    for (int cc = 0; cc < BN / 2; cc += 32) {
+    for (int i = 0; i < 4; ++i) {
+      const int j = buf == 0 ? (i + 3) & 3 : i;  // buffer 0: v of chunk 3 is the overlap
       uint32_t u[32], v[32];
-      tmem_ld_32x32b_x32(taddr + cc, u);
-      tmem_ld_32x32b_x32(taddr + BN / 2 + cc, v);
+      tmem_ld_32x32b_x32(taddr + 32 * j, u);
+      tmem_ld_32x32b_x32(taddr + 128 + 32 * j, v);
       tmem_ld_wait();
+      if (i == 0) signal_overlap(ovl_leader, lane);
       if (!valid) continue;
       float h[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float uu = r * __uint_as_float(u[j]);
-        h[j] = uu * sigmoid(uu) * (r * __uint_as_float(v[j]));
+      for (int t = 0; t < 32; ++t) {
+        const float uu = r * __uint_as_float(u[t]);
+        h[t] = uu * sigmoid(uu) * (r * __uint_as_float(v[t]));
       }
       uint32_t q[8];
       const uint32_t sb = mx_quantize32(h, q);
-      const int n = c.nt * (BN / 2) + cc;  // column of H within the expert
+      const int n = c.nt * 128 + 32 * j;  // column of H within the expert
       uint4* dst = reinterpret_cast<uint4*>(a.h8 + prow * a.ldh + n);
       dst[0] = make_uint4(q[0], q[1], q[2], q[3]);
       dst[1] = make_uint4(q[4], q[5], q[6], q[7]);
@@ -144,19 +178,22 @@ __device__ __forceinline__ void epilogue(const MxGemmArgs& a, const MxShared& sh
     }
   } else {
     const float g = asg >= 0 ? a.scale[asg] : 0.f;
-    __nv_bfloat16* dst = a.y + prow * a.d + c.nt * BN;
+    const int nchunk = bn / 32;
+    __nv_bfloat16* dst = a.y + prow * a.d + c.nt * bn;
 #pragma unroll 1
-    for (int cc = 0; cc < BN; cc += 32) {
+    for (int i = 0; i < nchunk; ++i) {
+      const int j = buf == 0 ? (i + nchunk - 1) % nchunk : i;
       uint32_t u[32];
-      tmem_ld_32x32b_x32(taddr + cc, u);
+      tmem_ld_32x32b_x32(taddr + 32 * j, u);
       tmem_ld_wait();
+      if (i == 0) signal_overlap(ovl_leader, lane);
       if (!valid) continue;
       uint32_t o[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) o[j] = pack_bf16(g * __uint_as_float(u[2 * j]), g * __uint_as_float(u[2 * j + 1]));
-      uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
+      for (int t = 0; t < 16; ++t) o[t] = pack_bf16(g * __uint_as_float(u[2 * t]), g * __uint_as_float(u[2 * t + 1]));
+      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * j);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) d4[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+      for (int t = 0; t < 4; ++t) d4[t] = make_uint4(o[4 * t], o[4 * t + 1], o[4 * t + 2], o[4 * t + 3]);
     }
   }
 }
@@ -164,7 +201,8 @@ __device__ __forceinline__ void epilogue(const MxGemmArgs& a, const MxShared& sh
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_mx_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
                            const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ CUtensorMap mapSFA,
-                           const __grid_constant__ CUtensorMap mapSFB, const __grid_constant__ MxGemmArgs a) {
+                           const __grid_constant__ CUtensorMap mapSFB0, const __grid_constant__ CUtensorMap mapSFB1,
+                           const __grid_constant__ MxGemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   MxShared& sh = *reinterpret_cast<MxShared*>(smem + kStages * kStageBytes);
@@ -182,6 +220,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.tfull[b], 1);
       mbar_init(&sh.tempty[b], 2 * kEpiWarps);
+      mbar_init(&sh.ovl[b], 2 * kEpiWarps);
     }
     mbar_init(&sh.drain, 1);
     sh.abort_flag = 0;
@@ -193,7 +232,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tma_prefetch_map(&mapB0);
     tma_prefetch_map(&mapB1);
     tma_prefetch_map(&mapSFA);
-    tma_prefetch_map(&mapSFB);
+    tma_prefetch_map(&mapSFB0);
+    tma_prefetch_map(&mapSFB1);
   }
   if (warp == 1) {
     tmem_alloc_pair(&sh.tmem_base, kTmemCols);
@@ -205,7 +245,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int rows = sh.seg[tid + 1] - sh.seg[tid];
     const int f = a.ffn.off[tid + 1] - a.ffn.off[tid];
     if ((sh.seg[tid] & 127) != 0 || rows < 0) sh.bad_segment = 1;  // scale blocks need 128-row segments
-    const int nt = a.up ? f / (BN / 2) : a.d / BN;
+    const int nt = a.up ? f / 128 : a.d / a.bn;
     const int kb = a.up ? a.d / BK : f / BK;
     const int mt = (rows + BM - 1) / BM;
     const long long a_rows_bytes = static_cast<long long>(BM) * kb * BK;
@@ -238,7 +278,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ================= TMA producer (one lane per CTA)
     if (lane == 0) {
       const uint32_t full_leader0 = map_to_cta(smem_addr(&sh.full[0]), 0);
-      const uint32_t tx_pair = 2u * static_cast<uint32_t>(kStageBytes);
+      const int sfb_blocks = (a.up || a.bn == 256) ? 2 : 1;
+      const uint32_t tx_pair =
+          2u * static_cast<uint32_t>(kABytes + (a.bn / 2) * BK + kSfBytes + sfb_blocks * kSfBytes);
       uint32_t it = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < total; tile += npairs) {
@@ -254,8 +296,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           const uint32_t bar = full_leader0 + static_cast<uint32_t>(s) * 8u;
           if (rank == 0) mbar_arrive_expect_tx(&sh.full[s], tx_pair);
-          issue_loads(a, &mapA, &mapB0, &mapB1, &mapSFA, &mapSFB, c, kb, smem + s * kStageBytes, bar, sh.seg[c.e],
-                      o_e, rank);
+          issue_loads(a, &mapA, &mapB0, &mapB1, &mapSFA, &mapSFB0, &mapSFB1, c, kb, smem + s * kStageBytes, bar,
+                      sh.seg[c.e], o_e, rank, a.bn);
         }
       }
       const uint32_t n_issued = it;
@@ -269,6 +311,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ================= MMA issuer (leader CTA, one lane)
     if (rank == 0 && lane == 0) {
       const uint32_t sfa_t = tmem_base + kSfaCol, sfb_t = tmem_base + kSfbCol;
+      const bool two_sfb = a.up || a.bn == 256;
+      const uint32_t idesc_n = static_cast<uint32_t>(a.bn);
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < total; tile += npairs, ++tcount) {
@@ -281,8 +325,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
+        // the previous tile's epilogues have read the columns both buffers share
+        if (tcount >= 1 && !mbar_wait(&sh.ovl[buf ^ 1u], ((tcount - 1) >> 1) & 1u, abort_flag, a.err,
+                                      MOE_DEVERR_TIMEOUT, kWaitTimeoutNs, true)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + buf * kAccCols;
+        const uint32_t d_tmem = tmem_base + buf_col(buf);
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1u;
@@ -297,11 +347,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // scale blocks: 32 lines x 16 bytes = four 8 x 16-byte core matrices, 128 bytes apart
           tmem_cp_pair_32x128b_warpx4(sfa_t, smem_desc_noswz(aSFA, 0, 128));
           tmem_cp_pair_32x128b_warpx4(sfb_t, smem_desc_noswz(aSFB, 0, 128));
+          if (two_sfb) tmem_cp_pair_32x128b_warpx4(sfb_t + 4, smem_desc_noswz(aSFB + kSfBytes, 0, 128));
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
             const uint64_t adesc = smem_desc_sw128(aA + kk * 32, 16, 1024);
             const uint64_t bdesc = smem_desc_sw128(aB + kk * 32, 16, 1024);
-            const uint32_t idesc = umma_idesc_mxf8(BM, BN, kk, kk);
+            const uint32_t idesc = umma_idesc_mxf8(BM, idesc_n, kk, kk);
             umma_mxf8_pair(d_tmem, adesc, bdesc, idesc, sfa_t | (static_cast<uint32_t>(kk) << 30),
                            sfb_t | (static_cast<uint32_t>(kk) << 30), (kb | kk) != 0 ? 1u : 0u);
           }
@@ -319,6 +370,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int row_in_cta = q * 32 + lane;
     const uint32_t tempty_leader0 = map_to_cta(smem_addr(&sh.tempty[0]), 0);
+    const uint32_t ovl_leader0 = map_to_cta(smem_addr(&sh.ovl[0]), 0);
     uint32_t tcount = 0;
     for (int tile = pair; tile < total; tile += npairs, ++tcount) {
       const TileCoord c = decode_tile(sh, E, tile);
@@ -329,7 +381,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       tc_fence_after();
-      epilogue(a, sh, c, tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kAccCols, row_in_cta, rank);
+      epilogue(a, sh, c, tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf_col(buf), row_in_cta, rank, buf,
+               a.bn, ovl_leader0 + buf * 8u, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + buf * 8u);
@@ -351,8 +404,10 @@ cudaError_t prepare_grouped_gemm_mx() {
 
 cudaError_t launch_grouped_gemm_mx(const MxGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB0,
                                    const CUtensorMap& mapB1, const CUtensorMap& mapSFA,
-                                   const CUtensorMap& mapSFB, int grid, cudaStream_t s) {
-  grouped_gemm_mx_kernel<<<grid, kThreads, kSmemBytes, s>>>(mapA, mapB0, mapB1, mapSFA, mapSFB, a);
+                                   const CUtensorMap& mapSFB0, const CUtensorMap& mapSFB1, int grid,
+                                   cudaStream_t s) {
+  if (a.bn != 256 && !(a.bn == 128 && !a.up)) return cudaErrorInvalidValue;
+  grouped_gemm_mx_kernel<<<grid, kThreads, kSmemBytes, s>>>(mapA, mapB0, mapB1, mapSFA, mapSFB0, mapSFB1, a);
   return cudaGetLastError();
 }
 

@@ -508,24 +508,28 @@ moe_status_t run_layer_mx(const moe_config_t& c, const Layout& L, void* ws, cons
   g.err = at<uint32_t>(ws, L.err);
   for (int e = 0; e <= c.E; ++e) g.ffn.off[e] = c.ffn_offsets[e];
   const int grid = gemm_grid_of_current_device();
-  CUtensorMap mA, mB0, mB1, mSA, mSB;
+  CUtensorMap mA, mB0, mB1, mSA, mSB0, mSB1;
   g.up = 1;
+  g.bn = 256;
   g.scale = r;
   g.h8 = at<uint8_t>(ws, L.h8);
   g.hsf = at<uint8_t>(ws, L.hsf);
-  if (!make_map_u8(&mA, at<void>(ws, L.x8), d, rows, d, 128, 128) || !make_map_u8(&mB0, q.w1, d, F, d, 128, 64) ||
-      !make_map_u8(&mB1, q.w3, d, F, d, 128, 64) || !make_map_sf(&mSA, at<void>(ws, L.xsf), (rows / 128) * (d / 128)) ||
-      !make_map_sf(&mSB, q.sf13, (F / 64) * (d / 128)))
+  if (!make_map_u8(&mA, at<void>(ws, L.x8), d, rows, d, 128, 128) || !make_map_u8(&mB0, q.w1, d, F, d, 128, 128) ||
+      !make_map_u8(&mB1, q.w3, d, F, d, 128, 128) ||
+      !make_map_sf(&mSA, at<void>(ws, L.xsf), (rows / 128) * (d / 128)) ||
+      !make_map_sf(&mSB0, q.sf1, (F / 128) * (d / 128)) || !make_map_sf(&mSB1, q.sf3, (F / 128) * (d / 128)))
     return MOE_ERR_CUDA;
-  if ((st = cuda_status(launch_grouped_gemm_mx(g, mA, mB0, mB1, mSA, mSB, grid, s))) != MOE_OK) return st;
+  if ((st = cuda_status(launch_grouped_gemm_mx(g, mA, mB0, mB1, mSA, mSB0, mSB1, grid, s))) != MOE_OK) return st;
   g.up = 0;
+  g.bn = (c.d_model % 256 == 0) ? 256 : 128;
   g.scale = gate;
   g.y = reinterpret_cast<__nv_bfloat16*>(y);
-  if (!make_map_u8(&mA, at<void>(ws, L.h8), ldh, rows, ldh, 128, 128) || !make_map_u8(&mB0, q.w2, F, d, F, 128, 64) ||
+  if (!make_map_u8(&mA, at<void>(ws, L.h8), ldh, rows, ldh, 128, 128) ||
+      !make_map_u8(&mB0, q.w2, F, d, F, 128, static_cast<uint32_t>(g.bn / 2)) ||
       !make_map_sf(&mSA, at<void>(ws, L.hsf), (rows / 128) * (ldh / 128)) ||
-      !make_map_sf(&mSB, q.sf2, (d / 128) * (F / 128)))
+      !make_map_sf(&mSB0, q.sf2, (d / 128) * (F / 128)))
     return MOE_ERR_CUDA;
-  if ((st = cuda_status(launch_grouped_gemm_mx(g, mA, mB0, mB0, mSA, mSB, grid, s))) != MOE_OK) return st;
+  if ((st = cuda_status(launch_grouped_gemm_mx(g, mA, mB0, mB0, mSA, mSB0, mSB0, grid, s))) != MOE_OK) return st;
   return run_combine(c, y, inv_perm, out, sms, s);
 }
 
@@ -1060,7 +1064,7 @@ moe_status_t moe_mx_part(const moe_config_t* cfg, void* wq, void* ws, size_t ws_
   if (which <= MOE_MX_SF2) {
     if (wq == nullptr) return MOE_ERR_INVALID_ARG;
     const MxWeights q = mx_weights_at(wq, cfg->d_model, cfg->ffn_offsets[cfg->E]);
-    uint8_t* parts[] = {q.w1, q.w3, q.w2, q.sf13, q.sf2};
+    uint8_t* parts[] = {q.w1, q.w3, q.w2, q.sf1, q.sf3, q.sf2};
     *ptr = parts[which];
     return MOE_OK;
   }

@@ -76,12 +76,9 @@ __host__ __device__ inline size_t mx_sf_offset(int64_t r, int64_t k, int64_t K) 
 
 // Quantised expert weights: K-major E4M3 copies and their scale blocks.
 //   w1, w3 [F, d]   (row n = column n of W1 / W3)      w2 [d, F] (row c = column c of W2)
-//   sf13: the up GEMM's B scales, one block per (64-column tile t, k block):
-//         rows 0..63 = W1 columns 64t.., rows 64..127 = W3 columns 64t..;
-//         block index t * (d / 128) + k / 128
-//   sf2:  standard blocks of w2 ([d, F] with K = F)
+//   sf1, sf3, sf2: the standard scale blocks of those [rows, K] operands
 struct MxWeights {
-  uint8_t *w1, *w3, *w2, *sf13, *sf2;
+  uint8_t *w1, *w3, *w2, *sf1, *sf3, *sf2;
 };
 size_t mx_weights_bytes(int d, int F);
 MxWeights mx_weights_at(void* base, int d, int F);
@@ -90,6 +87,7 @@ cudaError_t launch_quantize_weights_mx(const __nv_bfloat16* W1, const __nv_bfloa
 
 struct MxGemmArgs {
   int up;                   // 1: x8 x (W1|W3) -> SwiGLU -> H8 (+ scales); 0: H8 x W2 -> gate * y
+  int bn;                   // pair MMA N: 256 (the down GEMM: 128 when d % 256 != 0)
   int E, k, d, F;
   int rows;                 // rows of the permuted buffers (a multiple of 128)
   int ldh;                  // row stride of H8 (max expert width)
@@ -102,9 +100,11 @@ struct MxGemmArgs {
   uint32_t* err;
   ExpertTable ffn;
 };
+// up: mapSFB0 / mapSFB1 = scales of W1 / W3; down: both the scales of W2.
 cudaError_t launch_grouped_gemm_mx(const MxGemmArgs& a, const CUtensorMap& mapA, const CUtensorMap& mapB0,
                                    const CUtensorMap& mapB1, const CUtensorMap& mapSFA,
-                                   const CUtensorMap& mapSFB, int grid, cudaStream_t s);
+                                   const CUtensorMap& mapSFB0, const CUtensorMap& mapSFB1, int grid,
+                                   cudaStream_t s);
 cudaError_t prepare_grouped_gemm_mx();
 
 // Modes of the grouped GEMM (one kernel template, one instantiation each).

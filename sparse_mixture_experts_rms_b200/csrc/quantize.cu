@@ -15,11 +15,10 @@ namespace {
 size_t al(size_t v) { return (v + 1023) / 1024 * 1024; }
 
 // One thread per (column n, 32-block of K); consecutive threads take
-// consecutive n, so the reads of a K row are coalesced.
-// sf_mode 0: standard scale blocks of an [N, K] operand; 1 / 2: the up
-// GEMM's interleaved B blocks, W1 columns in rows 0..63 / W3 in rows 64..127.
+// consecutive n, so the reads of a K row are coalesced.  Scales go to the
+// standard blocks of the [N, K] copy.
 __global__ void __launch_bounds__(128) quantize_kn_mx_kernel(const __nv_bfloat16* W, int K, int N, uint8_t* q,
-                                                             uint8_t* sf, int sf_mode) {
+                                                             uint8_t* sf) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   const int k0 = blockIdx.y * 32;
   if (n >= N) return;
@@ -31,42 +30,37 @@ __global__ void __launch_bounds__(128) quantize_kn_mx_kernel(const __nv_bfloat16
   uint4* dst = reinterpret_cast<uint4*>(q + static_cast<size_t>(n) * K + k0);
   dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
   dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  size_t off;
-  if (sf_mode == 0) {
-    off = mx_sf_offset(n, k0, K);
-  } else {
-    const int row = (sf_mode == 2 ? 64 : 0) + (n & 63);
-    off = (static_cast<size_t>(n >> 6) * (K >> 7) + (k0 >> 7)) * 512 + 16 * (row & 31) + 4 * ((row & 127) >> 5) +
-          ((k0 & 127) >> 5);
-  }
-  sf[off] = static_cast<uint8_t>(sb);
+  sf[mx_sf_offset(n, k0, K)] = static_cast<uint8_t>(sb);
 }
 
 }  // namespace
 
 size_t mx_weights_bytes(int d, int F) {
   const size_t dd = static_cast<size_t>(d), ff = static_cast<size_t>(F);
-  return 3 * al(dd * ff) + al((ff / 64) * (dd / 128) * 512) + al((dd / 128) * (ff / 128) * 512);
+  const size_t sf = al((ff / 128) * (dd / 128) * 512);  // each of sf1, sf3, sf2
+  return 3 * al(dd * ff) + 3 * sf;
 }
 
 MxWeights mx_weights_at(void* base, int d, int F) {
   const size_t dd = static_cast<size_t>(d), ff = static_cast<size_t>(F);
+  const size_t sf = al((ff / 128) * (dd / 128) * 512);
   uint8_t* p = static_cast<uint8_t*>(base);
   MxWeights m;
   m.w1 = p;
   m.w3 = m.w1 + al(dd * ff);
   m.w2 = m.w3 + al(dd * ff);
-  m.sf13 = m.w2 + al(dd * ff);
-  m.sf2 = m.sf13 + al((ff / 64) * (dd / 128) * 512);
+  m.sf1 = m.w2 + al(dd * ff);
+  m.sf3 = m.sf1 + sf;
+  m.sf2 = m.sf3 + sf;
   return m;
 }
 
 cudaError_t launch_quantize_weights_mx(const __nv_bfloat16* W1, const __nv_bfloat16* W3,
                                        const __nv_bfloat16* W2, MxWeights q, int d, int F, cudaStream_t s) {
   const dim3 g13((F + 127) / 128, d / 32), g2((d + 127) / 128, F / 32);
-  quantize_kn_mx_kernel<<<g13, 128, 0, s>>>(W1, d, F, q.w1, q.sf13, 1);
-  quantize_kn_mx_kernel<<<g13, 128, 0, s>>>(W3, d, F, q.w3, q.sf13, 2);
-  quantize_kn_mx_kernel<<<g2, 128, 0, s>>>(W2, F, d, q.w2, q.sf2, 0);
+  quantize_kn_mx_kernel<<<g13, 128, 0, s>>>(W1, d, F, q.w1, q.sf1);
+  quantize_kn_mx_kernel<<<g13, 128, 0, s>>>(W3, d, F, q.w3, q.sf3);
+  quantize_kn_mx_kernel<<<g2, 128, 0, s>>>(W2, F, d, q.w2, q.sf2);
   return cudaGetLastError();
 }
 

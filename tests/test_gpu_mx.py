@@ -65,13 +65,11 @@ def test_weight_codes_and_scales_are_bit_exact():
     np.testing.assert_array_equal(e4m3(moe.mx_part_view(cfg, wq, None, "W1")).T, c1)
     np.testing.assert_array_equal(e4m3(moe.mx_part_view(cfg, wq, None, "W3")).T, c3)
     np.testing.assert_array_equal(e4m3(moe.mx_part_view(cfg, wq, None, "W2")).T, c2)
-    sf13 = moe.mx_part_view(cfg, wq, None, "SF13").cpu().numpy().astype(np.int64) - 127
     n = np.arange(F)[:, None]
     k = (np.arange(dm // 32) * 32)[None, :]
-    for half, s in ((0, s1), (64, s3)):
-        row = half + n % 64
-        off = ((n // 64) * (dm // 128) + k // 128) * 512 + 16 * (row % 32) + 4 * ((row % 128) // 32) + (k % 128) // 32
-        np.testing.assert_array_equal(sf13[off], s.T)
+    for name, s in (("SF1", s1), ("SF3", s3)):
+        sf = moe.mx_part_view(cfg, wq, None, name).cpu().numpy().astype(np.int64) - 127
+        np.testing.assert_array_equal(sf[sf_offset(n, k, dm)], s.T)
     sf2 = moe.mx_part_view(cfg, wq, None, "SF2").cpu().numpy().astype(np.int64) - 127
     c = np.arange(dm)[:, None]
     f = (np.arange(F // 32) * 32)[None, :]
