@@ -1,24 +1,23 @@
-// moe_api.cu -- the C ABI declared in include/moe.h: argument validation,
-// workspace layout, TMA descriptor encoding and launch sequencing on one
-// stream.  Allocates nothing; never synchronises except in
+// moe_api.cu -- the C ABI declared in include/moe.h (the forward layer and
+// its stages; training in api_train.cu, MXFP8 in api_mx.cu, host buffers in
+// api_host.cu): argument validation, workspace layout, TMA descriptor
+// encoding and launch sequencing on one stream.  Allocates nothing; never synchronises except in
 // moe_get_device_error.
 #include <cmath>
 #include <cstring>
 #include <algorithm>
 #include <mutex>
 
-#include "moe_internal.h"
+#include "api_detail.h"
 
 namespace moe {
-namespace {
+namespace api {
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-constexpr int kMaxDevices = 64;
-constexpr size_t kHeaderBytes = 256;
 
 struct DeviceState {
   bool ready = false;
@@ -31,27 +30,6 @@ std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
 bool g_encode_tried = false;
-
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
-
-bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
-struct Layout {
-  size_t err, ticket, rw, prob_partial, prob_mean, tile_counts, r, idx, gate, counts, offsets, perm,
-      inv_perm, x_perm, H, y, total;
-  // training workspace only
-  size_t logits, U, V, yu, dY, dS, dS3, drp, dXp, dgate, rdl, dr, dbias_part, dgamma_part, dWr_part;
-  // MXFP8 workspace only
-  size_t x8, xsf, h8, hsf;
-  int64_t max_kept;  // rows of the permuted buffers (padded in the training layout)
-  int ldh;
-  int ld_drp, chunks, chunk_tokens, route_blocks;
-  bool train;
-  bool mx;
-};
-
-constexpr int kTrainRowAlign = 64;  // row-segment padding of the training layout
-constexpr int kMxRowAlign = 128;    // MX path: a CTA's 128 rows are one scale block
 
 int64_t capacity_of(const moe_config_t& c) {
   if (!(c.capacity_factor > 0.0f)) return -1;
@@ -85,7 +63,7 @@ moe_status_t validate(const moe_config_t* c) {
   return MOE_OK;
 }
 
-Layout layout_of(const moe_config_t& c, bool train = false, bool mx = false) {
+Layout layout_of(const moe_config_t& c, bool train, bool mx) {
   Layout L{};
   L.train = train;
   L.mx = mx;
@@ -162,8 +140,8 @@ Layout layout_of(const moe_config_t& c, bool train = false, bool mx = false) {
   return L;
 }
 
-moe_status_t check_ws(const moe_config_t& c, void* ws, size_t ws_bytes, Layout* L, bool train = false,
-                      bool mx = false) {
+moe_status_t check_ws(const moe_config_t& c, void* ws, size_t ws_bytes, Layout* L, bool train,
+                      bool mx) {
   *L = layout_of(c, train, mx);
   if (ws == nullptr || ws_bytes < L->total) return MOE_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return MOE_ERR_ALIGNMENT;
@@ -261,10 +239,6 @@ moe_status_t cuda_status(cudaError_t e) {
   return MOE_ERR_CUDA;
 }
 
-template <typename T>
-T* at(void* ws, size_t off) {
-  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
-}
 
 moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf16_t* gamma,
                        const moe_bf16_t* Wr, const float* bias, int32_t* idx, float* gate, float* r,
@@ -305,8 +279,8 @@ moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf1
 moe_status_t run_dispatch(const moe_config_t& c, const Layout& L, void* ws, const int32_t* idx,
                           const moe_bf16_t* x, const moe_bf16_t* gamma, int32_t* counts,
                           int32_t* offsets, int32_t* perm, int32_t* inv_perm, moe_bf16_t* x_perm,
-                          int sms, cudaStream_t s, int row_align = 1, uint8_t* x8 = nullptr,
-                          uint8_t* xsf = nullptr) {
+                          int sms, cudaStream_t s, int row_align, uint8_t* x8,
+                          uint8_t* xsf) {
   DispatchArgs a{};
   a.x8 = x8;
   a.xsf = xsf;
@@ -353,7 +327,7 @@ void fill_gemm_common(GemmArgs& g, const moe_config_t& c, const Layout& L, void*
 moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x_perm,
                     const float* r, const int32_t* perm, const int32_t* offsets,
                     const moe_bf16_t* W1, const moe_bf16_t* W3, int sms, cudaStream_t s,
-                    moe_bf16_t* U = nullptr, moe_bf16_t* V = nullptr) {
+                    moe_bf16_t* U, moe_bf16_t* V) {
   if (L.max_kept == 0) return MOE_OK;
   const uint64_t rows = static_cast<uint64_t>(L.max_kept);
   const uint64_t d = static_cast<uint64_t>(c.d_model);
@@ -378,7 +352,7 @@ moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_
 // GEMM 2: H [rows, f_e] (workspace) x W2 [F, d] -> y [rows, d], gate in the epilogue
 moe_status_t run_down(const moe_config_t& c, const Layout& L, void* ws, const float* gate,
                       const int32_t* perm, const int32_t* offsets, const moe_bf16_t* W2,
-                      moe_bf16_t* y, int sms, cudaStream_t s, moe_bf16_t* yu = nullptr) {
+                      moe_bf16_t* y, int sms, cudaStream_t s, moe_bf16_t* yu) {
   if (L.max_kept == 0) return MOE_OK;
   const uint64_t rows = static_cast<uint64_t>(L.max_kept);
   const uint64_t d = static_cast<uint64_t>(c.d_model);
@@ -428,7 +402,7 @@ constexpr size_t kNoallocCountInts =
     static_cast<size_t>(kNoallocMaxAssignments / kDispatchTile) * kMaxExperts;  // 256 KiB
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoallocHeaderInts + kNoallocCountInts];
 
-int32_t* g_noalloc_ptr[kMaxDevices] = {};
+static int32_t* g_noalloc_ptr[kMaxDevices] = {};
 
 // Device address of g_noalloc_scratch on the current device (looked up once per
 // device; in host code the symbol itself is only a host-side stand-in).
@@ -479,260 +453,11 @@ moe_status_t run_layer(const moe_config_t& c, const Layout& L, void* ws, const m
   return MOE_OK;
 }
 
-// ---- the layer with MXFP8 expert GEMMs (cfg validated, T > 0, pointers checked)
-moe_status_t run_layer_mx(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x,
-                          const moe_bf16_t* gamma, const moe_bf16_t* Wr, const float* bias, const MxWeights& q,
-                          moe_bf16_t* out, int sms, cudaStream_t s) {
-  moe_status_t st;
-  int32_t* idx = at<int32_t>(ws, L.idx);
-  float* gate = at<float>(ws, L.gate);
-  float* r = at<float>(ws, L.r);
-  int32_t* offsets = at<int32_t>(ws, L.offsets);
-  int32_t* perm = at<int32_t>(ws, L.perm);
-  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
-  moe_bf16_t* y = at<moe_bf16_t>(ws, L.y);
-  if ((st = run_route(c, x, gamma, Wr, bias, idx, gate, r, nullptr, nullptr, L, ws, s)) != MOE_OK) return st;
-  if ((st = run_dispatch(c, L, ws, idx, x, gamma, at<int32_t>(ws, L.counts), offsets, perm, inv_perm, nullptr,
-                         sms, s, kMxRowAlign, at<uint8_t>(ws, L.x8), at<uint8_t>(ws, L.xsf))) != MOE_OK)
-    return st;
-  const uint64_t rows = static_cast<uint64_t>(L.max_kept);
-  const uint64_t d = static_cast<uint64_t>(c.d_model);
-  const uint64_t F = static_cast<uint64_t>(c.ffn_offsets[c.E]);
-  const uint64_t ldh = static_cast<uint64_t>(L.ldh);
-  MxGemmArgs g{};
-  g.E = c.E; g.k = c.k; g.d = c.d_model; g.F = static_cast<int>(F);
-  g.rows = static_cast<int>(L.max_kept);
-  g.ldh = L.ldh;
-  g.offsets = offsets;
-  g.perm = perm;
-  g.err = at<uint32_t>(ws, L.err);
-  for (int e = 0; e <= c.E; ++e) g.ffn.off[e] = c.ffn_offsets[e];
-  const int grid = gemm_grid_of_current_device();
-  CUtensorMap mA, mB0, mB1, mSA, mSB0, mSB1;
-  g.up = 1;
-  g.bn = 256;
-  g.scale = r;
-  g.h8 = at<uint8_t>(ws, L.h8);
-  g.hsf = at<uint8_t>(ws, L.hsf);
-  if (!make_map_u8(&mA, at<void>(ws, L.x8), d, rows, d, 128, 128) || !make_map_u8(&mB0, q.w1, d, F, d, 128, 128) ||
-      !make_map_u8(&mB1, q.w3, d, F, d, 128, 128) ||
-      !make_map_sf(&mSA, at<void>(ws, L.xsf), (rows / 128) * (d / 128)) ||
-      !make_map_sf(&mSB0, q.sf1, (F / 128) * (d / 128)) || !make_map_sf(&mSB1, q.sf3, (F / 128) * (d / 128)))
-    return MOE_ERR_CUDA;
-  if ((st = cuda_status(launch_grouped_gemm_mx(g, mA, mB0, mB1, mSA, mSB0, mSB1, grid, s))) != MOE_OK) return st;
-  g.up = 0;
-  g.bn = (c.d_model % 256 == 0) ? 256 : 128;
-  g.scale = gate;
-  g.y = reinterpret_cast<__nv_bfloat16*>(y);
-  if (!make_map_u8(&mA, at<void>(ws, L.h8), ldh, rows, ldh, 128, 128) ||
-      !make_map_u8(&mB0, q.w2, F, d, F, 128, static_cast<uint32_t>(g.bn / 2)) ||
-      !make_map_sf(&mSA, at<void>(ws, L.hsf), (rows / 128) * (ldh / 128)) ||
-      !make_map_sf(&mSB0, q.sf2, (d / 128) * (F / 128)))
-    return MOE_ERR_CUDA;
-  if ((st = cuda_status(launch_grouped_gemm_mx(g, mA, mB0, mB0, mSA, mSB0, mSB0, grid, s))) != MOE_OK) return st;
-  return run_combine(c, y, inv_perm, out, sms, s);
-}
-
-// ---- host-buffer layer: token chunks pipelined over two copy streams
-//
-// Without a capacity limit a token's output depends on that token alone, so
-// the batch is cut into n token chunks: the copy of chunk i+1 to the device
-// and of chunk i-1 back to the host overlap the layer on chunk i.  Staging buffers are double-buffered in the workspace.  With a capacity
-// limit the drops depend on every token's rank, so the batch is one chunk.
-constexpr int kDefaultHostChunks = 3;  // measured best on the Mixtral-shaped layer (2..8 tried)
-
-struct HostPipe {
-  bool made = false;
-  cudaStream_t h2d = nullptr, d2h = nullptr;
-  cudaEvent_t start = nullptr, h2d_done[2] = {nullptr, nullptr}, comp_done[2] = {nullptr, nullptr},
-              d2h_done[2] = {nullptr, nullptr};
-};
-std::mutex g_pipe_mutex[kMaxDevices];
-HostPipe g_pipe[kMaxDevices];
-
-bool make_pipe(HostPipe& p) {
-  if (p.made) return true;
-  bool ok = cudaStreamCreateWithFlags(&p.h2d, cudaStreamNonBlocking) == cudaSuccess &&
-            cudaStreamCreateWithFlags(&p.d2h, cudaStreamNonBlocking) == cudaSuccess &&
-            cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming) == cudaSuccess;
-  for (int b = 0; ok && b < 2; ++b)
-    ok = cudaEventCreateWithFlags(&p.h2d_done[b], cudaEventDisableTiming) == cudaSuccess &&
-         cudaEventCreateWithFlags(&p.comp_done[b], cudaEventDisableTiming) == cudaSuccess &&
-         cudaEventCreateWithFlags(&p.d2h_done[b], cudaEventDisableTiming) == cudaSuccess;
-  if (!ok) {
-    cudaGetLastError();
-    return false;
-  }
-  p.made = true;
-  return true;
-}
-
-constexpr int kMaxHostChunks = 64;
-
-struct HostLayout {
-  int n;                         // chunks
-  int64_t start[kMaxHostChunks + 1];  // token offsets of the chunks
-  int64_t tc;                    // tokens of the largest chunk
-  size_t layer;                  // bytes of the per-chunk layer workspace (at offset 0)
-  size_t xs[2], os[2], total;
-};
-
-// Chunk sizes in the ratio 1 : 2 : ... : 2 : 1: only the first chunk's copy
-// in and the last chunk's copy out are not hidden behind compute, so those two
-// are half the size of the others.
-HostLayout host_layout_of(const moe_config_t& c, int n_chunks) {
-  HostLayout H{};
-  int n = n_chunks > 0 ? n_chunks : kDefaultHostChunks;
-  if (capacity_of(c) >= 0) n = 1;          // capacity ranks span the whole batch
-  if (n > kMaxHostChunks) n = kMaxHostChunks;
-  if (n > c.T) n = c.T > 0 ? c.T : 1;
-  const int64_t wsum = n <= 2 ? n : 2 * n - 2;
-  int64_t acc = 0;
-  H.start[0] = 0;
-  for (int i = 0; i < n; ++i) {
-    acc += (n <= 2 || i == 0 || i == n - 1) ? 1 : 2;
-    H.start[i + 1] = (static_cast<int64_t>(c.T) * acc) / wsum;
-  }
-  for (int i = 1; i < n; ++i)  // no empty chunk (n <= T leaves room for one token each)
-    H.start[i] = std::min<int64_t>(std::max<int64_t>(H.start[i], H.start[i - 1] + 1), c.T - (n - i));
-  H.n = n;
-  H.tc = 0;
-  for (int i = 0; i < n; ++i) H.tc = std::max<int64_t>(H.tc, H.start[i + 1] - H.start[i]);
-  moe_config_t cc = c;
-  cc.T = static_cast<int32_t>(H.tc);
-  H.layer = align_up(layout_of(cc).total, 1024);
-  const size_t chunk_bytes = align_up(static_cast<size_t>(H.tc) * c.d_model * 2, 1024);
-  size_t off = H.layer;
-  for (int b = 0; b < 2; ++b) { H.xs[b] = off; off += chunk_bytes; }
-  for (int b = 0; b < 2; ++b) { H.os[b] = off; off += chunk_bytes; }
-  H.total = off;
-  return H;
-}
-
-// ---- training backward: gather -> bwd_h -> bwd_x -> weight gradients ->
-// router/statistic backward -> norm backward -> reductions, on one stream.
-moe_status_t run_backward(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x,
-                          const moe_bf16_t* gamma, const moe_bf16_t* Wr, const float* bias,
-                          const moe_bf16_t* W1, const moe_bf16_t* W3, const moe_bf16_t* W2,
-                          const moe_bf16_t* dout, float* dx, float* dgamma, float* dWr, float* dbias,
-                          float* dW1, float* dW3, float* dW2, int sms, cudaStream_t s) {
-  const uint64_t rows = static_cast<uint64_t>(L.max_kept);
-  const uint64_t d = static_cast<uint64_t>(c.d_model);
-  const uint64_t F = static_cast<uint64_t>(c.ffn_offsets[c.E]);
-  const uint64_t ldh = static_cast<uint64_t>(L.ldh);
-  int32_t* offsets = at<int32_t>(ws, L.offsets);
-  int32_t* perm = at<int32_t>(ws, L.perm);
-  bool all256 = true;
-  for (int e = 0; e < c.E; ++e) all256 = all256 && ((c.ffn_offsets[e + 1] - c.ffn_offsets[e]) % 256 == 0);
-  const int bn_h = all256 ? 256 : 128;
-  const int bn_d = (c.d_model % 256 == 0) ? 256 : 128;
-  const int grid = gemm_grid_of_current_device();
-
-  BwdArgs b{};
-  b.T = c.T; b.d = c.d_model; b.E = c.E; b.k = c.k; b.renormalize = c.renormalize;
-  b.rows = static_cast<int>(L.max_kept);
-  b.x = reinterpret_cast<const __nv_bfloat16*>(x);
-  b.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
-  b.Wr = reinterpret_cast<const __nv_bfloat16*>(Wr);
-  b.bias = bias;
-  b.dout = reinterpret_cast<const __nv_bfloat16*>(dout);
-  b.r = at<float>(ws, L.r);
-  b.idx = at<int32_t>(ws, L.idx);
-  b.gate = at<float>(ws, L.gate);
-  b.logits = at<float>(ws, L.logits);
-  b.offsets = offsets;
-  b.perm = perm;
-  b.inv_perm = at<int32_t>(ws, L.inv_perm);
-  b.yu = at<__nv_bfloat16>(ws, L.yu);
-  b.dY = at<__nv_bfloat16>(ws, L.dY);
-  b.dgate = at<float>(ws, L.dgate);
-  b.drp = at<float>(ws, L.drp);
-  b.ld_drp = L.ld_drp;
-  b.bn_h = bn_h;
-  b.dXp = at<float>(ws, L.dXp);
-  b.rdl = at<float>(ws, L.rdl);
-  b.dr = at<float>(ws, L.dr);
-  b.dbias_part = at<float>(ws, L.dbias_part);
-  b.route_blocks = L.route_blocks;
-  b.dx = dx;
-  b.dgamma_part = at<float>(ws, L.dgamma_part);
-  b.dWr_part = at<float>(ws, L.dWr_part);
-  b.chunks = L.chunks;
-  b.chunk_tokens = L.chunk_tokens;
-  b.dgamma = dgamma;
-  b.dWr = dWr;
-  b.dbias = dbias;
-  b.err = at<uint32_t>(ws, L.err);
-  for (int e = 0; e <= c.E; ++e) b.ffn.off[e] = c.ffn_offsets[e];
-
-  moe_status_t st = cuda_status(launch_bwd_gather(b, sms, s));
-  if (st != MOE_OK) return st;
-  void* dY = at<void>(ws, L.dY);
-  void* dS = at<void>(ws, L.dS);
-  void* dS3 = at<void>(ws, L.dS3);
-  CUtensorMap mA0, mA1, mB0, mB1;
-  {  // dS, dS3, dr partials: dY [rows, d] x W2 rows (K-major)
-    GemmArgs g{};
-    fill_gemm_common(g, c, L, ws, perm, offsets);
-    g.mode = kGemmBwdH;
-    g.bn = bn_h;
-    g.scale = b.r;
-    g.ld_out = L.ldh;
-    g.in_u = at<__nv_bfloat16>(ws, L.U);
-    g.in_v = at<__nv_bfloat16>(ws, L.V);
-    g.out_ds = static_cast<__nv_bfloat16*>(dS);
-    g.out_ds3 = static_cast<__nv_bfloat16*>(dS3);
-    g.drp = at<float>(ws, L.drp);
-    g.ld_drp = L.ld_drp;
-    if (!make_map(&mA0, dY, d, rows, d, 64, 128) || !make_map(&mB0, W2, d, F, d, 64, bn_h / 2))
-      return MOE_ERR_CUDA;
-    if ((st = cuda_status(launch_grouped_gemm(g, mA0, mA0, mB0, mB0, grid, s))) != MOE_OK) return st;
-  }
-  {  // dX per kept row: [dS | dS3] x [W1 | W3]^T (W rows, K-major)
-    GemmArgs g{};
-    fill_gemm_common(g, c, L, ws, perm, offsets);
-    g.mode = kGemmBwdX;
-    g.bn = bn_d;
-    g.out_f0 = at<float>(ws, L.dXp);
-    g.ld_f = c.d_model;
-    if (!make_map(&mA0, dS, ldh, rows, ldh, 64, 128) || !make_map(&mA1, dS3, ldh, rows, ldh, 64, 128) ||
-        !make_map(&mB0, W1, F, d, F, 64, bn_d / 2) || !make_map(&mB1, W3, F, d, F, 64, bn_d / 2))
-      return MOE_ERR_CUDA;
-    if ((st = cuda_status(launch_grouped_gemm(g, mA0, mA1, mB0, mB1, grid, s))) != MOE_OK) return st;
-  }
-  {  // dW1 | dW3 = x_perm^T [dS | dS3]  (both operands MN-major, K = rows)
-    GemmArgs g{};
-    fill_gemm_common(g, c, L, ws, perm, offsets);
-    g.mode = kGemmWgradX;
-    g.bn = 256;
-    g.out_f0 = dW1;
-    g.out_f1 = dW3;
-    g.ld_f = static_cast<int>(F);
-    if (!make_map(&mA0, at<void>(ws, L.x_perm), d, rows, d, 64, 64) ||
-        !make_map(&mB0, dS, ldh, rows, ldh, 64, 64) || !make_map(&mB1, dS3, ldh, rows, ldh, 64, 64))
-      return MOE_ERR_CUDA;
-    if ((st = cuda_status(launch_grouped_gemm(g, mA0, mA0, mB0, mB1, grid, s))) != MOE_OK) return st;
-  }
-  {  // dW2 = H^T dY
-    GemmArgs g{};
-    fill_gemm_common(g, c, L, ws, perm, offsets);
-    g.mode = kGemmWgradH;
-    g.bn = bn_d;
-    g.out_f0 = dW2;
-    g.ld_f = c.d_model;
-    if (!make_map(&mA0, at<void>(ws, L.H), ldh, rows, ldh, 64, 64) || !make_map(&mB0, dY, d, rows, d, 64, 64))
-      return MOE_ERR_CUDA;
-    if ((st = cuda_status(launch_grouped_gemm(g, mA0, mA0, mB0, mB0, grid, s))) != MOE_OK) return st;
-  }
-  if ((st = cuda_status(launch_bwd_route(b, s))) != MOE_OK) return st;
-  if ((st = cuda_status(launch_bwd_norm(b, s))) != MOE_OK) return st;
-  return cuda_status(launch_bwd_reduce(b, s));
-}
-
-}  // namespace
+}  // namespace api
 }  // namespace moe
 
 using namespace moe;
+using namespace moe::api;
 
 extern "C" {
 
@@ -1001,278 +726,6 @@ moe_status_t moe_router_stats(const moe_config_t* cfg, const float* prob_mean, c
   if ((st = device_ready(&sms)) != MOE_OK) return st;
   return cuda_status(launch_router_stats(prob_mean, counts, expert_offsets, stats, cfg->T, cfg->E, cfg->k,
                                          static_cast<cudaStream_t>(stream)));
-}
-
-size_t moe_mx_weights_size(const moe_config_t* cfg) {
-  if (validate(cfg) != MOE_OK) return 0;
-  return mx_weights_bytes(cfg->d_model, cfg->ffn_offsets[cfg->E]);
-}
-
-moe_status_t moe_quantize_weights_mx(const moe_config_t* cfg, const moe_bf16_t* W1, const moe_bf16_t* W3,
-                                     const moe_bf16_t* W2, void* wq, size_t wq_bytes, void* stream) {
-  moe_status_t st = validate(cfg);
-  if (st != MOE_OK) return st;
-  if (!W1 || !W3 || !W2 || !wq) return MOE_ERR_INVALID_ARG;
-  if (!aligned(W1, 16) || !aligned(W3, 16) || !aligned(W2, 16) || !aligned(wq, 256)) return MOE_ERR_ALIGNMENT;
-  const int d = cfg->d_model, F = cfg->ffn_offsets[cfg->E];
-  if (wq_bytes < mx_weights_bytes(d, F)) return MOE_ERR_WORKSPACE;
-  int sms;
-  if ((st = device_ready(&sms)) != MOE_OK) return st;
-  return cuda_status(launch_quantize_weights_mx(reinterpret_cast<const __nv_bfloat16*>(W1),
-                                                reinterpret_cast<const __nv_bfloat16*>(W3),
-                                                reinterpret_cast<const __nv_bfloat16*>(W2), mx_weights_at(wq, d, F),
-                                                d, F, static_cast<cudaStream_t>(stream)));
-}
-
-size_t moe_mx_workspace_size(const moe_config_t* cfg) {
-  if (validate(cfg) != MOE_OK) return 0;
-  return layout_of(*cfg, false, true).total;
-}
-
-int64_t moe_mx_rows(const moe_config_t* cfg) {
-  if (validate(cfg) != MOE_OK) return -1;
-  return layout_of(*cfg, false, true).max_kept;
-}
-
-moe_status_t moe_layer_fwd_mx(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
-                              const moe_bf16_t* Wr, const float* bias, const void* wq, size_t wq_bytes,
-                              moe_bf16_t* out, void* ws, size_t ws_bytes, void* stream) {
-  moe_status_t st = validate(cfg);
-  if (st != MOE_OK) return st;
-  if (cfg->T == 0) return MOE_OK;
-  if (!x || !gamma || !Wr || !wq || !out) return MOE_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) || !aligned(wq, 256) ||
-      !aligned(out, 16))
-    return MOE_ERR_ALIGNMENT;
-  const int d = cfg->d_model, F = cfg->ffn_offsets[cfg->E];
-  if (wq_bytes < mx_weights_bytes(d, F)) return MOE_ERR_WORKSPACE;
-  Layout L;
-  if ((st = check_ws(*cfg, ws, ws_bytes, &L, false, true)) != MOE_OK) return st;
-  int sms;
-  if ((st = device_ready(&sms)) != MOE_OK) return st;
-  return run_layer_mx(*cfg, L, ws, x, gamma, Wr, bias, mx_weights_at(const_cast<void*>(wq), d, F), out, sms,
-                      static_cast<cudaStream_t>(stream));
-}
-
-moe_status_t moe_mx_part(const moe_config_t* cfg, void* wq, void* ws, size_t ws_bytes, int32_t which,
-                         void** ptr) {
-  if (ptr == nullptr) return MOE_ERR_INVALID_ARG;
-  *ptr = nullptr;
-  moe_status_t st = validate(cfg);
-  if (st != MOE_OK) return st;
-  if (which < 0) return MOE_ERR_INVALID_ARG;
-  if (which <= MOE_MX_SF2) {
-    if (wq == nullptr) return MOE_ERR_INVALID_ARG;
-    const MxWeights q = mx_weights_at(wq, cfg->d_model, cfg->ffn_offsets[cfg->E]);
-    uint8_t* parts[] = {q.w1, q.w3, q.w2, q.sf1, q.sf3, q.sf2};
-    *ptr = parts[which];
-    return MOE_OK;
-  }
-  Layout L;
-  if ((st = check_ws(*cfg, ws, ws_bytes, &L, false, true)) != MOE_OK) return st;
-  size_t off;
-  switch (which) {
-    case MOE_MX_X8: off = L.x8; break;
-    case MOE_MX_XSF: off = L.xsf; break;
-    case MOE_MX_H8: off = L.h8; break;
-    case MOE_MX_HSF: off = L.hsf; break;
-    case MOE_MX_PERM: off = L.perm; break;
-    case MOE_MX_OFFSETS: off = L.offsets; break;
-    case MOE_MX_IDX: off = L.idx; break;
-    case MOE_MX_GATE: off = L.gate; break;
-    case MOE_MX_R: off = L.r; break;
-    default: return MOE_ERR_INVALID_ARG;
-  }
-  *ptr = at<void>(ws, off);
-  return MOE_OK;
-}
-
-size_t moe_host_workspace_size(const moe_config_t* cfg, int32_t n_chunks) {
-  if (validate(cfg) != MOE_OK) return 0;
-  return host_layout_of(*cfg, n_chunks).total;
-}
-
-int32_t moe_host_chunks(const moe_config_t* cfg, int32_t n_chunks) {
-  if (validate(cfg) != MOE_OK) return -1;
-  return host_layout_of(*cfg, n_chunks).n;
-}
-
-moe_status_t moe_layer_fwd_host(const moe_config_t* cfg, const moe_bf16_t* x_host, const moe_bf16_t* gamma,
-                                const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
-                                const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out_host,
-                                int32_t n_chunks, void* ws, size_t ws_bytes, void* stream) {
-  moe_status_t st = validate(cfg);
-  if (st != MOE_OK) return st;
-  const moe_config_t& c = *cfg;
-  if (c.T == 0) return MOE_OK;
-  if (!x_host || !gamma || !Wr || !W1 || !W3 || !W2 || !out_host) return MOE_ERR_INVALID_ARG;
-  if (!aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) || !aligned(W1, 16) || !aligned(W3, 16) ||
-      !aligned(W2, 16) || !aligned(x_host, 2) || !aligned(out_host, 2))
-    return MOE_ERR_ALIGNMENT;
-  const HostLayout H = host_layout_of(c, n_chunks);
-  if (ws == nullptr || ws_bytes < H.total) return MOE_ERR_WORKSPACE;
-  if (!aligned(ws, 256)) return MOE_ERR_ALIGNMENT;
-  int sms;
-  if ((st = device_ready(&sms)) != MOE_OK) return st;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  std::lock_guard<std::mutex> lock(g_pipe_mutex[dev]);
-  HostPipe& P = g_pipe[dev];
-  if (!make_pipe(P)) return MOE_ERR_CUDA;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t row_bytes = static_cast<size_t>(c.d_model) * 2;
-  const char* xh = reinterpret_cast<const char*>(x_host);
-  char* oh = reinterpret_cast<char*>(out_host);
-  cudaError_t e = cudaEventRecord(P.start, s);  // copies start after earlier work on `stream`
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(P.h2d, P.start, 0);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(P.d2h, P.start, 0);
-  if (e != cudaSuccess) return cuda_status(e);
-  for (int i = 0; i < H.n; ++i) {
-    const int b = i & 1;
-    const int64_t t0 = H.start[i];
-    const int64_t ti = H.start[i + 1] - t0;  // >= 1: n <= T
-    moe_config_t ci = c;
-    ci.T = static_cast<int32_t>(ti);
-    const Layout Li = layout_of(ci);
-    moe_bf16_t* xs = at<moe_bf16_t>(ws, H.xs[b]);
-    moe_bf16_t* os = at<moe_bf16_t>(ws, H.os[b]);
-    const size_t bytes = static_cast<size_t>(ti) * row_bytes;
-    if (i >= 2) e = cudaStreamWaitEvent(P.h2d, P.comp_done[b], 0);  // xs[b] read by chunk i-2
-    if (e == cudaSuccess) e = cudaMemcpyAsync(xs, xh + t0 * row_bytes, bytes, cudaMemcpyHostToDevice, P.h2d);
-    if (e == cudaSuccess) e = cudaEventRecord(P.h2d_done[b], P.h2d);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, P.h2d_done[b], 0);
-    if (e == cudaSuccess && i >= 2) e = cudaStreamWaitEvent(s, P.d2h_done[b], 0);  // os[b] copied out
-    if (e != cudaSuccess) return cuda_status(e);
-    // the chunk's layer workspace: the error word lives in its header (offset 0)
-    if ((st = run_layer(ci, Li, ws, xs, gamma, Wr, bias, W1, W3, W2, os, nullptr, nullptr, nullptr, nullptr,
-                        nullptr, nullptr, sms, s)) != MOE_OK)
-      return st;
-    e = cudaEventRecord(P.comp_done[b], s);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(P.d2h, P.comp_done[b], 0);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(oh + t0 * row_bytes, os, bytes, cudaMemcpyDeviceToHost, P.d2h);
-    if (e == cudaSuccess) e = cudaEventRecord(P.d2h_done[b], P.d2h);
-    if (e != cudaSuccess) return cuda_status(e);
-  }
-  // the caller's stream completes after the last copies out
-  e = cudaStreamWaitEvent(s, P.d2h_done[(H.n - 1) & 1], 0);
-  if (e == cudaSuccess && H.n >= 2) e = cudaStreamWaitEvent(s, P.d2h_done[H.n & 1], 0);
-  return cuda_status(e);
-}
-
-size_t moe_train_workspace_size(const moe_config_t* cfg) {
-  if (validate(cfg) != MOE_OK) return 0;
-  return layout_of(*cfg, true).total;
-}
-
-int64_t moe_train_rows(const moe_config_t* cfg) {
-  if (validate(cfg) != MOE_OK) return -1;
-  return layout_of(*cfg, true).max_kept;
-}
-
-moe_status_t moe_train_saved(const moe_config_t* cfg, void* tws, size_t tws_bytes, int32_t which,
-                             void** ptr) {
-  if (ptr == nullptr) return MOE_ERR_INVALID_ARG;
-  *ptr = nullptr;
-  moe_status_t st = validate(cfg);
-  if (st != MOE_OK) return st;
-  Layout L;
-  if ((st = check_ws(*cfg, tws, tws_bytes, &L, true)) != MOE_OK) return st;
-  size_t off;
-  switch (which) {
-    case MOE_SAVED_R: off = L.r; break;
-    case MOE_SAVED_IDX: off = L.idx; break;
-    case MOE_SAVED_GATE: off = L.gate; break;
-    case MOE_SAVED_LOGITS: off = L.logits; break;
-    case MOE_SAVED_OFFSETS: off = L.offsets; break;
-    case MOE_SAVED_PERM: off = L.perm; break;
-    case MOE_SAVED_INV_PERM: off = L.inv_perm; break;
-    case MOE_SAVED_U: off = L.U; break;
-    case MOE_SAVED_V: off = L.V; break;
-    case MOE_SAVED_H: off = L.H; break;
-    case MOE_SAVED_Y: off = L.yu; break;
-    case MOE_SAVED_DGATE: off = L.dgate; break;
-    case MOE_SAVED_DR: off = L.dr; break;
-    case MOE_SAVED_COUNTS: off = L.counts; break;
-    default: return MOE_ERR_INVALID_ARG;
-  }
-  *ptr = at<void>(tws, off);
-  return MOE_OK;
-}
-
-moe_status_t moe_layer_fwd_train(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
-                                 const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
-                                 const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out, void* tws,
-                                 size_t tws_bytes, void* stream) {
-  moe_status_t st = validate(cfg);
-  if (st != MOE_OK) return st;
-  if (cfg->T == 0) return MOE_OK;
-  if (!x || !gamma || !Wr || !W1 || !W3 || !W2 || !out) return MOE_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) ||
-      !aligned(W1, 16) || !aligned(W3, 16) || !aligned(W2, 16) || !aligned(out, 16))
-    return MOE_ERR_ALIGNMENT;
-  Layout L;
-  if ((st = check_ws(*cfg, tws, tws_bytes, &L, true)) != MOE_OK) return st;
-  int sms;
-  if ((st = device_ready(&sms)) != MOE_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const moe_config_t& c = *cfg;
-  void* ws = tws;
-  int32_t* idx = at<int32_t>(ws, L.idx);
-  float* gate = at<float>(ws, L.gate);
-  float* r = at<float>(ws, L.r);
-  int32_t* offsets = at<int32_t>(ws, L.offsets);
-  int32_t* perm = at<int32_t>(ws, L.perm);
-  int32_t* inv_perm = at<int32_t>(ws, L.inv_perm);
-  moe_bf16_t* x_perm = at<moe_bf16_t>(ws, L.x_perm);
-  moe_bf16_t* y = at<moe_bf16_t>(ws, L.y);
-  if ((st = run_route(c, x, gamma, Wr, bias, idx, gate, r, at<float>(ws, L.logits), nullptr, L, ws, s)) !=
-      MOE_OK)
-    return st;
-  if ((st = run_dispatch(c, L, ws, idx, x, gamma, at<int32_t>(ws, L.counts), offsets, perm, inv_perm, x_perm,
-                         sms, s, kTrainRowAlign)) != MOE_OK)
-    return st;
-  if ((st = run_up(c, L, ws, x_perm, r, perm, offsets, W1, W3, sms, s, at<moe_bf16_t>(ws, L.U),
-                   at<moe_bf16_t>(ws, L.V))) != MOE_OK)
-    return st;
-  if ((st = run_down(c, L, ws, gate, perm, offsets, W2, y, sms, s, at<moe_bf16_t>(ws, L.yu))) != MOE_OK)
-    return st;
-  return run_combine(c, y, inv_perm, out, sms, s);
-}
-
-moe_status_t moe_layer_bwd(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
-                           const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
-                           const moe_bf16_t* W3, const moe_bf16_t* W2, const moe_bf16_t* dout, float* dx,
-                           float* dgamma, float* dWr, float* dbias, float* dW1, float* dW3, float* dW2,
-                           void* tws, size_t tws_bytes, void* stream) {
-  moe_status_t st = validate(cfg);
-  if (st != MOE_OK) return st;
-  const moe_config_t& c = *cfg;
-  if (!dgamma || !dWr || !dbias || !dW1 || !dW3 || !dW2) return MOE_ERR_INVALID_ARG;
-  if (!aligned(dgamma, 4) || !aligned(dWr, 16) || !aligned(dbias, 4) || !aligned(dW1, 16) ||
-      !aligned(dW3, 16) || !aligned(dW2, 16))
-    return MOE_ERR_ALIGNMENT;
-  int sms;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t d = static_cast<size_t>(c.d_model), F = static_cast<size_t>(c.ffn_offsets[c.E]);
-  if (c.T == 0) {  // no tokens: every parameter gradient is zero
-    if ((st = device_ready(&sms)) != MOE_OK) return st;
-    cudaError_t e = cudaMemsetAsync(dgamma, 0, d * 4, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(dWr, 0, d * c.E * 4, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(dbias, 0, static_cast<size_t>(c.E) * 4, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(dW1, 0, d * F * 4, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(dW3, 0, d * F * 4, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(dW2, 0, d * F * 4, s);
-    return cuda_status(e);
-  }
-  if (!x || !gamma || !Wr || !W1 || !W3 || !W2 || !dout || !dx) return MOE_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) ||
-      !aligned(W1, 16) || !aligned(W3, 16) || !aligned(W2, 16) || !aligned(dout, 16) || !aligned(dx, 16))
-    return MOE_ERR_ALIGNMENT;
-  Layout L;
-  if ((st = check_ws(c, tws, tws_bytes, &L, true)) != MOE_OK) return st;
-  if ((st = device_ready(&sms)) != MOE_OK) return st;
-  return run_backward(c, L, tws, x, gamma, Wr, bias, W1, W3, W2, dout, dx, dgamma, dWr, dbias, dW1, dW3, dW2,
-                      sms, s);
 }
 
 }  // extern "C"
