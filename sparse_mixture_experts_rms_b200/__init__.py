@@ -625,3 +625,49 @@ class MoELayer:
         return out
 
     __call__ = forward
+
+
+class _MoETrainFn(torch.autograd.Function):
+    """autograd glue: forward = moe_layer_fwd_train, backward = moe_layer_bwd.
+    Gradients come back in fp32 and are cast to each input's dtype."""
+
+    @staticmethod
+    def forward(ctx, cfg, tws, x, gamma, Wr, bias, W1, W3, W2):
+        out = torch.empty((cfg.T, cfg.d_model), dtype=torch.bfloat16, device=x.device)
+        moe_layer_fwd_train(cfg, x, gamma, Wr, bias, W1, W3, W2, out, tws)
+        ctx.cfg, ctx.tws = cfg, tws
+        ctx.save_for_backward(x, gamma, Wr, bias if bias is not None else torch.empty(0), W1, W3, W2)
+        ctx.has_bias = bias is not None
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        cfg, tws = ctx.cfg, ctx.tws
+        x, gamma, Wr, bias, W1, W3, W2 = ctx.saved_tensors
+        bias = bias if ctx.has_bias else None
+        T, d, E, F = cfg.T, cfg.d_model, cfg.E, cfg.F
+        f32 = dict(dtype=torch.float32, device=x.device)
+        g = [torch.empty((T, d), **f32), torch.empty((d,), **f32), torch.empty((d, E), **f32),
+             torch.empty((E,), **f32), torch.empty((d, F), **f32), torch.empty((d, F), **f32),
+             torch.empty((F, d), **f32)]
+        moe_layer_bwd(cfg, x, gamma, Wr, bias, W1, W3, W2, dout.to(torch.bfloat16).contiguous(), *g, tws)
+        dx, dgamma, dWr, dbias, dW1, dW3, dW2 = g
+        return (None, None, dx.to(x.dtype), dgamma.to(gamma.dtype), dWr.to(Wr.dtype),
+                dbias if ctx.has_bias else None, dW1.to(W1.dtype), dW3.to(W3.dtype), dW2.to(W2.dtype))
+
+
+class MoETrainLayer:
+    """A layer for training: ``forward(x)`` runs the training forward and
+    returns an output whose backward runs moe_layer_bwd (one forward in flight
+    per layer: the training workspace holds one forward's saved state)."""
+
+    def __init__(self, cfg: MoEConfig, gamma, Wr, bias, W1, W3, W2):
+        self.cfg = cfg
+        self.gamma, self.Wr, self.bias = gamma, Wr, bias
+        self.W1, self.W3, self.W2 = W1, W3, W2
+        self.tws = alloc_train_workspace(cfg, device=gamma.device)
+
+    def forward(self, x):
+        return _MoETrainFn.apply(self.cfg, self.tws, x, self.gamma, self.Wr, self.bias, self.W1, self.W3, self.W2)
+
+    __call__ = forward

@@ -113,3 +113,33 @@ def test_several_tiles_backward():
     """Several 256-row M tiles and 64-row K blocks per expert."""
     w = mw.Workload("bwd_tiles", T=1000, d_model=256, E=4, k=2, expert_sizes=((4, 512),), bias="normal")
     run_case(w)
+
+
+def test_autograd_layer_gives_the_direct_gradients():
+    """MoETrainLayer under torch autograd returns what moe_layer_bwd returns
+    (cast to the parameters' dtypes) and the forward's output."""
+    w = mw.WORKLOADS["tiny"]
+    p = H.make_problem(w)
+    cfg = H.make_cfg(p)
+    d = H.Dev(p, cfg)
+    params = [t.clone().requires_grad_(True) for t in (d.gamma, d.Wr, d.W1, d.W3, d.W2)]
+    x = d.x.clone().requires_grad_(True)
+    layer = moe.MoETrainLayer(cfg, params[0], params[1], None, params[2], params[3], params[4])
+    out = layer(x)
+    dout = H.bits_to_dev(_upstream(w.T, w.d_model))
+    out.backward(dout)
+    torch.cuda.synchronize()
+    ref_out = torch.empty_like(out)
+    moe.moe_layer_fwd(cfg, d.x, d.gamma, d.Wr, None, d.W1, d.W3, d.W2, ref_out, d.ws)
+    assert torch.equal(out.detach(), ref_out)
+    tws = moe.alloc_train_workspace(cfg)
+    moe.moe_layer_fwd_train(cfg, d.x, d.gamma, d.Wr, None, d.W1, d.W3, d.W2, torch.empty_like(out), tws)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    T, dm, E, F = cfg.T, cfg.d_model, cfg.E, cfg.F
+    G = [torch.empty((T, dm), **f32), torch.empty((dm,), **f32), torch.empty((dm, E), **f32),
+         torch.empty((E,), **f32), torch.empty((dm, F), **f32), torch.empty((dm, F), **f32),
+         torch.empty((F, dm), **f32)]
+    moe.moe_layer_bwd(cfg, d.x, d.gamma, d.Wr, None, d.W1, d.W3, d.W2, dout, *G, tws)
+    torch.cuda.synchronize()
+    for got, ref in zip([x.grad] + [t.grad for t in params], [G[0], G[1], G[2], G[4], G[5], G[6]]):
+        assert torch.equal(got, ref.to(got.dtype))
