@@ -143,3 +143,10 @@ def test_autograd_layer_gives_the_direct_gradients():
     torch.cuda.synchronize()
     for got, ref in zip([x.grad] + [t.grad for t in params], [G[0], G[1], G[2], G[4], G[5], G[6]]):
         assert torch.equal(got, ref.to(got.dtype))
+
+
+def test_fine_grained_backward():
+    """E = 64, top-8 with renormalised gates and a normal logit bias: the
+    E <= 64 variant of the norm backward and the router backward over 8 slots."""
+    w = mw.Workload("bwd_fine", T=300, d_model=256, E=64, k=8, expert_sizes=((64, 128),), bias="normal")
+    run_case(w, renormalize=True)

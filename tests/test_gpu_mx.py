@@ -120,3 +120,15 @@ def test_layer_with_capacity_and_an_empty_expert():
     w = mw.Workload("mx_cap", T=600, d_model=256, E=4, k=1, expert_sizes=((4, 512),), capacity_factor=1.0)
     p, cfg, d, wq, ws, out = run_mx(w, bias=[0.5, 0.0, -60.0, 0.2])
     _check_layer(p, cfg, d, wq, ws, out)
+
+
+def test_layer_fine_grained_many_experts():
+    """E = 64 experts of width 128, top-8: 64 row segments padded to 128 rows."""
+    w = mw.Workload("mx_fine", T=512, d_model=256, E=64, k=8, expert_sizes=((64, 128),), bias="normal")
+    _check_layer(*run_mx(w))
+
+
+def test_layer_every_expert_chosen():
+    """k = E: every token visits every expert."""
+    w = mw.Workload("mx_kE", T=200, d_model=128, E=4, k=4, expert_sizes=((4, 256),))
+    _check_layer(*run_mx(w))
