@@ -88,7 +88,8 @@ struct __align__(8) GemmShared {
   int m_tiles[kMaxExperts];
   int n_tiles[kMaxExperts];
   int k_blocks[kMaxExperts];
-  int group_m[kMaxExperts];  // m tiles per raster group (see decode_tile)
+  int group_m[kMaxExperts];  // raster block: group_m x group_n tiles (see decode_tile)
+  int group_n[kMaxExperts];
   int seg[kMaxExperts + 1];
 };
 
@@ -98,20 +99,26 @@ struct TileCoord {
   int e, nt, mt;
 };
 
-// Tiles of expert e are rastered in groups of group_m[e] M tiles: inside a
-// group, M is fastest and N next, so the pairs running together share the
-// group's A rows (kept in L2) and a few B column blocks.  group_m is chosen so
-// that a group's A rows fit an L2 budget; when the whole expert fits, the
-// order is plain M-fastest.
+// Tiles of expert e are rastered in blocks of group_m[e] x group_n[e] (M x N)
+// tiles, M fastest inside a block, blocks N-fastest along a row of blocks, so
+// the pairs running together share a few A row panels and B column panels in
+// L2.  When all of an expert's A panels fit an L2 budget the block spans the
+// expert (plain M-fastest order: every B panel is read once); when they do
+// not (a long reduction), blocks are about as square as the resident pairs
+// allow, so a wave touches about 2 sqrt(pairs) panels instead of
+// group_m + every N panel.
 __device__ __forceinline__ TileCoord decode_tile(const GemmShared& sh, int E, int tile) {
   int e = 0;
   while (e + 1 < E && tile >= sh.tile_start[e + 1]) ++e;
   const int local = tile - sh.tile_start[e];
-  const int mt_count = sh.m_tiles[e], nt_count = sh.n_tiles[e], gm = sh.group_m[e];
-  const int g = local / (gm * nt_count);
-  const int rem = local - g * gm * nt_count;
-  const int gm_g = min(gm, mt_count - g * gm);  // the last group may be short
-  return TileCoord{e, rem / gm_g, g * gm + rem % gm_g};
+  const int mt_count = sh.m_tiles[e], nt_count = sh.n_tiles[e];
+  const int gm = sh.group_m[e], gn = sh.group_n[e];
+  const int bm = local / (gm * nt_count);            // row of blocks
+  const int rem = local - bm * gm * nt_count;
+  const int gm_b = min(gm, mt_count - bm * gm);      // the last row may be short
+  const int bn = rem / (gm_b * gn);                  // block in the row
+  const int rem2 = rem - bn * gm_b * gn;
+  return TileCoord{e, bn * gn + rem2 / gm_b, bm * gm + rem2 % gm_b};
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -442,13 +449,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // K of the weight gradients is a row segment: it must be whole K blocks
     if (!Traits<MODE>::row_tiles && (rows < 0 || rows % BK != 0)) sh.bad_segment = 1;
     const int mt = (mext + BM - 1) / BM;
-    const long long a_rows_bytes = static_cast<long long>(BM) * kb * BK * 2;
-    int gm = static_cast<int>(kL2GroupBudget / (a_rows_bytes > 0 ? a_rows_bytes : 1));
-    gm = gm < 1 ? 1 : gm;
-    sh.m_tiles[tid] = mt > 0 ? mt : 1;
-    sh.n_tiles[tid] = nt > 0 ? nt : 1;
+    const long long a_panel = static_cast<long long>(BM) * kb * BK * 2;  // one M tile's A over all K
+    const long long b_panel = static_cast<long long>(a.bn) * kb * BK * 2;  // one N tile's B over all K
+    const int mtc = mt > 0 ? mt : 1, ntc = nt > 0 ? nt : 1;
+    int gm = mtc, gn = ntc;
+    if (a_panel > 0 && static_cast<long long>(mtc) * a_panel > kL2GroupBudget) {
+      // square-ish blocks of about one wave of pairs
+      const int pairs = static_cast<int>(gridDim.x >> 1);
+      gm = static_cast<int>(sqrtf(static_cast<float>(pairs) * static_cast<float>(b_panel) /
+                                  static_cast<float>(a_panel)));
+      gm = gm < 1 ? 1 : (gm > mtc ? mtc : gm);
+      gn = pairs / gm;
+      gn = gn < 1 ? 1 : (gn > ntc ? ntc : gn);
+    }
+    sh.m_tiles[tid] = mtc;
+    sh.n_tiles[tid] = ntc;
     sh.k_blocks[tid] = kb;
-    sh.group_m[tid] = gm < sh.m_tiles[tid] ? gm : sh.m_tiles[tid];
+    sh.group_m[tid] = gm;
+    sh.group_n[tid] = gn;
     sh.tile_start[tid + 1] = (mt > 0 && nt > 0) ? mt * nt : 0;  // count for now
   }
   __syncthreads();
