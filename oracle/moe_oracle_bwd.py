@@ -53,6 +53,21 @@ def _f64(a) -> np.ndarray:
     return np.asarray(a, dtype=np.float64)
 
 
+class _ExpertSlices:
+    """Expert e's (W1[:, o_e:o_e+1], W3[...], W2[o_e:o_e+1, :]) as float64,
+    widened on first use and kept."""
+
+    def __init__(self, W1, W3, W2, offs):
+        self.W, self.offs, self.cache = (W1, W3, W2), offs, {}
+
+    def __getitem__(self, e):
+        if e not in self.cache:
+            W1, W3, W2 = self.W
+            o0, o1 = self.offs[e], self.offs[e + 1]
+            self.cache[e] = (O.as_f64(W1[:, o0:o1]), O.as_f64(W3[:, o0:o1]), O.as_f64(W2[o0:o1, :]))
+        return self.cache[e]
+
+
 # --------------------------------------------------------------------------
 # forward in float64 with everything the backward reads
 # --------------------------------------------------------------------------
@@ -60,8 +75,10 @@ def layer_forward(x, gamma, Wr, bias, W1, W3, W2, widths: Sequence[int], k: int,
                   eps: float = 1e-5, capacity_factor: float = 0.0,
                   renormalize: bool = False, idx: Optional[np.ndarray] = None) -> Dict[str, object]:
     """Steps 1-7 on float64 values (no fp32 rounding of the logits), keeping
-    the per-assignment intermediates.  ``idx`` replays a given routing."""
-    x, gamma, Wr, W1, W3, W2 = (_f64(v) for v in (x, gamma, Wr, W1, W3, W2))
+    the per-assignment intermediates.  ``idx`` replays a given routing.  The
+    expert weights may be float64 or bf16 bit patterns (uint16); their expert
+    slices are widened where used, one expert at a time."""
+    x, gamma, Wr = (_f64(v) for v in (x, gamma, Wr))
     T, d = x.shape
     E = Wr.shape[1]
     r = O.rms_stat(x, eps)
@@ -83,22 +100,23 @@ def layer_forward(x, gamma, Wr, bias, W1, W3, W2, widths: Sequence[int], k: int,
     s3 = [None] * n_a
     h = [None] * n_a
     y = np.zeros((n_a, d))
+    slices = _ExpertSlices(W1, W3, W2, offs)
     for a in range(n_a):
         if not D["kept"][a]:
             continue
         t, e = a // k, int(idx[a // k, a % k])
-        o0, o1 = offs[e], offs[e + 1]
-        s[a] = xg[t] @ W1[:, o0:o1]
-        s3[a] = xg[t] @ W3[:, o0:o1]
+        W1e, W3e, W2e = slices[e]
+        s[a] = xg[t] @ W1e
+        s3[a] = xg[t] @ W3e
         h[a] = O.silu(r[t] * s[a]) * (r[t] * s3[a])
-        y[a] = h[a] @ W2[o0:o1, :]
+        y[a] = h[a] @ W2e
     out = np.zeros((T, d))
     for t in range(T):
         for j in range(k):
             a = t * k + j
             if D["kept"][a]:
                 out[t] += gate[t, j] * y[a]
-    return {"x": x, "gamma": gamma, "Wr": Wr, "W1": W1, "W3": W3, "W2": W2,
+    return {"x": x, "gamma": gamma, "Wr": Wr, "W1": W1, "W3": W3, "W2": W2, "slices": slices,
             "r": r, "xg": xg, "z": z, "logits": logits, "p": p, "q": q,
             "idx": idx, "gate": gate, "kept": D["kept"], "offs": offs,
             "s": s, "s3": s3, "h": h, "y": y, "out": out, "k": k,
@@ -153,21 +171,27 @@ def swiglu_backward(dh: np.ndarray, u: np.ndarray, v: np.ndarray):
 # --------------------------------------------------------------------------
 # the whole backward
 # --------------------------------------------------------------------------
-def layer_backward(f: Dict[str, object], g) -> Dict[str, np.ndarray]:
+def layer_backward(f: Dict[str, object], g, weight_grads: bool = True) -> Dict[str, np.ndarray]:
     """Gradients of L = <g, out> w.r.t. x, gamma, Wr, bias, W1, W3, W2.
 
     ``f`` is ``layer_forward``'s result.  Also returns the per-assignment
     dgate and the per-token dr (split into its expert and router parts) so
     that each stage of another implementation can be checked on its own.
+    ``weight_grads=False`` skips dW1, dW3, dW2 (returned as None): the other
+    gradients of a token then depend on that token alone (without a capacity
+    limit), so a subset of tokens can be checked at full size.
     """
     g = _f64(g)
     x, gamma, Wr = f["x"], f["gamma"], f["Wr"]
-    W1, W3, W2 = f["W1"], f["W3"], f["W2"]
+    slices = f["slices"]
     r, xg, z, p, q = f["r"], f["xg"], f["z"], f["p"], f["q"]
     idx, gate, kept, offs, k = f["idx"], f["gate"], f["kept"], f["offs"], f["k"]
     T, d = x.shape
     E = Wr.shape[1]
-    dW1, dW3, dW2 = np.zeros_like(W1), np.zeros_like(W3), np.zeros_like(W2)
+    F = int(offs[-1])
+    dW1 = np.zeros((d, F)) if weight_grads else None
+    dW3 = np.zeros((d, F)) if weight_grads else None
+    dW2 = np.zeros((F, d)) if weight_grads else None
     dxg = np.zeros((T, d))
     dr_exp = np.zeros(T)
     dgate = np.zeros((T, k))
@@ -177,16 +201,18 @@ def layer_backward(f: Dict[str, object], g) -> Dict[str, np.ndarray]:
         t, j = a // k, a % k
         e = int(idx[t, j])
         o0, o1 = offs[e], offs[e + 1]
+        W1e, W3e, W2e = slices[e]
         dgate[t, j] = g[t] @ f["y"][a]
         dy = gate[t, j] * g[t]
-        dh = W2[o0:o1, :] @ dy
-        dW2[o0:o1, :] += np.outer(f["h"][a], dy)
+        dh = W2e @ dy
         u, v = r[t] * f["s"][a], r[t] * f["s3"][a]
         du, dv = swiglu_backward(dh, u, v)
         dS, dS3 = r[t] * du, r[t] * dv
-        dW1[:, o0:o1] += np.outer(xg[t], dS)
-        dW3[:, o0:o1] += np.outer(xg[t], dS3)
-        dxg[t] += W1[:, o0:o1] @ dS + W3[:, o0:o1] @ dS3
+        if weight_grads:
+            dW2[o0:o1, :] += np.outer(f["h"][a], dy)
+            dW1[:, o0:o1] += np.outer(xg[t], dS)
+            dW3[:, o0:o1] += np.outer(xg[t], dS3)
+        dxg[t] += W1e @ dS + W3e @ dS3
         dr_exp[t] += du @ f["s"][a] + dv @ f["s3"][a]
     # router: gates -> q -> p (scattered to the chosen experts) -> logits
     dq = gate_backward(dgate, q, f["renormalize"])

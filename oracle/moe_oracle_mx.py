@@ -105,12 +105,38 @@ def quantized_weights(W1_bits, W3_bits, W2_bits) -> Dict[str, np.ndarray]:
             "W2": mx_value(O.as_f64(W2_bits), axis=0)}
 
 
+class LazyExpertWeights:
+    """MX values of one expert's weight slices, quantised when first used:
+    W1/W3 columns o_e..o_e+1 blocked along d, W2 rows o_e..o_e+1 blocked along
+    F.  Blocks never cross an expert (every width is a multiple of 128), so a
+    slice's MX value equals the slice of the whole matrix's."""
+
+    def __init__(self, W1_bits, W3_bits, W2_bits, offs):
+        self.W, self.offs, self.cache = (W1_bits, W3_bits, W2_bits), offs, {}
+
+    def expert(self, e):
+        if e not in self.cache:
+            W1, W3, W2 = self.W
+            o0, o1 = int(self.offs[e]), int(self.offs[e + 1])
+            self.cache[e] = (mx_value(O.as_f64(W1[:, o0:o1]), axis=0), mx_value(O.as_f64(W3[:, o0:o1]), axis=0),
+                             mx_value(O.as_f64(W2[o0:o1, :]), axis=0))
+        return self.cache[e]
+
+
+def _expert_mx(Wq, offs, e):
+    if isinstance(Wq, LazyExpertWeights):
+        return Wq.expert(e)
+    o0, o1 = int(offs[e]), int(offs[e + 1])
+    return Wq["W1"][:, o0:o1], Wq["W3"][:, o0:o1], Wq["W2"][o0:o1, :]
+
+
 def experts_forward_mx(x_rows: np.ndarray, gamma: np.ndarray, r: np.ndarray, idx: np.ndarray,
                        kept: np.ndarray, Wq: Dict[str, np.ndarray], offs: Sequence[int],
                        tokens: np.ndarray) -> np.ndarray:
     """y [T*k, d] for the kept assignments of ``tokens`` (rows of x_rows in
     that order): u = r (MX(x*gamma) MX(W1_e)), v likewise with W3, h = silu(u) v,
-    y = MX(h) MX(W2_e), the MX blocks of h running along the expert width."""
+    y = MX(h) MX(W2_e), the MX blocks of h running along the expert width.
+    ``Wq``: ``quantized_weights``' dict or a ``LazyExpertWeights``."""
     idx = np.asarray(idx, dtype=np.int64)
     T, k = idx.shape
     d = x_rows.shape[1]
@@ -125,12 +151,12 @@ def experts_forward_mx(x_rows: np.ndarray, gamma: np.ndarray, r: np.ndarray, idx
         if not m.any():
             continue
         sel, rows = a_all[m], row_all[m]
-        o0, o1 = int(offs[e]), int(offs[e + 1])
+        W1e, W3e, W2e = _expert_mx(Wq, offs, e)
         rr = np.asarray(r, dtype=np.float64)[sel // k][:, None]
-        u = rr * (xq[rows] @ Wq["W1"][:, o0:o1])
-        v = rr * (xq[rows] @ Wq["W3"][:, o0:o1])
+        u = rr * (xq[rows] @ W1e)
+        v = rr * (xq[rows] @ W3e)
         h = O.silu(u) * v
-        y[sel] = mx_value(h, axis=1) @ Wq["W2"][o0:o1, :]
+        y[sel] = mx_value(h, axis=1) @ W2e
     return y
 
 

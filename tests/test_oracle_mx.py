@@ -141,3 +141,16 @@ def test_planted_rounding_mistakes_are_caught(mutant, monkeypatch):
         except AssertionError:
             failures += 1
     assert failures > 0, mutant
+
+
+def test_lazy_per_expert_quantisation_equals_the_whole_matrix():
+    w = mw.WORKLOADS["variable_size"]
+    widths = O.expert_widths(w.expert_sizes)
+    W1, W3, W2 = mw.gen_expert_weights(w, widths, experts=[0, 3])
+    full = M.quantized_weights(W1, W3, W2)
+    offs = O.expert_offsets(widths)
+    lazy = M.LazyExpertWeights(W1, W3, W2, offs)
+    for e in (0, 3):
+        o0, o1 = offs[e], offs[e + 1]
+        for got, ref in zip(lazy.expert(e), (full["W1"][:, o0:o1], full["W3"][:, o0:o1], full["W2"][o0:o1, :])):
+            np.testing.assert_array_equal(got, ref)
