@@ -259,7 +259,7 @@ MOE_API moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x,
  * cudaHostAlloc, lets the copies overlap; pageable memory works but does not
  * overlap).  Without a capacity limit a token's output depends only on that
  * token, so the batch is cut into n_chunks chunks (sizes in the ratio
- * 1 : 2 : ... : 2 : 1, since only the first copy in and the last copy out are
+ * 1 : 4 : ... : 4 : 1, since only the first copy in and the last copy out are
  * exposed) and the copy of chunk i+1 in and of chunk i-1 out run on the library's own
  * copy streams while the layer runs on chunk i: out is bit-identical to
  * moe_layer_fwd on the whole batch.  With a capacity limit (capacity_factor >

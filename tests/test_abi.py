@@ -209,7 +209,7 @@ def test_host_pipeline_chunking(lib):
     assert moe.moe_host_chunks(cap, 4) == 1
     for c, n in ((mix, 4), (small, 4), (cap, 4)):
         m = moe.moe_host_chunks(c, n)
-        w = [1] * m if m <= 2 else [1] + [2] * (m - 2) + [1]
+        w = [1] * m if m <= 2 else [1] + [4] * (m - 2) + [1]
         bounds = [c.T * sum(w[:i]) // sum(w) for i in range(m + 1)]
         for i in range(1, m):
             bounds[i] = min(max(bounds[i], bounds[i - 1] + 1), c.T - (m - i))
