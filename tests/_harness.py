@@ -12,7 +12,12 @@ import moe_workloads as mw
 import sparse_mixture_experts_rms_b200 as moe
 from oracle import moe_oracle as O
 
-# tolerances
+# Tolerances.  Gates and logits come from fp32 logits on both sides (the GPU
+# sums exact bf16 products in fp64 chunks and rounds once), so they agree to
+# a few fp32 ulps; tokens whose k-th and (k+1)-th oracle logits are closer
+# than TIE_MARGIN may take the other expert and are left out of the routing
+# comparison.  The layer output passes through bf16 operands and a bf16 H on
+# the GPU, so it is compared normwise per token and by its mean absolute error.
 GATE_ATOL = 1e-5          # gates: absolute
 LOGIT_ATOL = 1e-5         # router logits: absolute (also the near-tie margin)
 TIE_MARGIN = 1e-5         # k-th vs (k+1)-th oracle fp32 logit
