@@ -84,3 +84,75 @@ def test_pair_tile_boundaries(rows):
                           p.W2, O.expert_offsets(p.widths))
     ref = O.combine(y, gate.cpu().numpy().astype(np.float64), D["kept"])
     H.check_rows(H.bf16_dev_to_f64(o["out"]), ref, "out")
+
+
+def test_training_step_and_mx_forward_capture_into_cuda_graphs():
+    """The training forward + backward and the MXFP8 forward are stream-ordered
+    too: captured once, replayed, they reproduce the eager results bit for bit."""
+    w = mw.WORKLOADS["variable_size"].with_tokens(700, name="var_graph_train")
+    p = H.make_problem(w)
+    cfg = H.make_cfg(p)
+    d = H.Dev(p, cfg)
+    T, dm, E, F = cfg.T, cfg.d_model, cfg.E, cfg.F
+    dout = torch.randn((T, dm), generator=torch.Generator().manual_seed(3)).to(torch.bfloat16).cuda()
+    f32 = dict(dtype=torch.float32, device="cuda")
+
+    def grads():
+        return [torch.zeros((T, dm), **f32), torch.zeros((dm,), **f32), torch.zeros((dm, E), **f32),
+                torch.zeros((E,), **f32), torch.zeros((dm, F), **f32), torch.zeros((dm, F), **f32),
+                torch.zeros((F, dm), **f32)]
+
+    tws = moe.alloc_train_workspace(cfg)
+    out_e, G_e = torch.empty((T, dm), dtype=torch.bfloat16, device="cuda"), grads()
+    moe.moe_layer_fwd_train(cfg, d.x, d.gamma, d.Wr, d.bias, d.W1, d.W3, d.W2, out_e, tws)
+    moe.moe_layer_bwd(cfg, d.x, d.gamma, d.Wr, d.bias, d.W1, d.W3, d.W2, dout, *G_e, tws)
+    wq = moe.alloc_mx_weights(cfg, d.W1, d.W3, d.W2)
+    mws = moe.alloc_mx_workspace(cfg)
+    mx_e = torch.empty((T, dm), dtype=torch.bfloat16, device="cuda")
+    moe.moe_layer_fwd_mx(cfg, d.x, d.gamma, d.Wr, d.bias, wq, mx_e, mws)
+    torch.cuda.synchronize()
+    out_g, G_g = torch.zeros_like(out_e), grads()
+    mx_g = torch.zeros_like(mx_e)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.moe_layer_fwd_train(cfg, d.x, d.gamma, d.Wr, d.bias, d.W1, d.W3, d.W2, out_g, tws)
+        moe.moe_layer_bwd(cfg, d.x, d.gamma, d.Wr, d.bias, d.W1, d.W3, d.W2, dout, *G_g, tws)
+        moe.moe_layer_fwd_mx(cfg, d.x, d.gamma, d.Wr, d.bias, wq, mx_g, mws)
+    for _ in range(2):
+        for t in [out_g, mx_g] + G_g:
+            t.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out_g, out_e) and torch.equal(mx_g, mx_e)
+        for a, b in zip(G_g, G_e):
+            assert torch.equal(a, b)
+    assert moe.moe_get_device_error(tws, raise_on_error=False) == 0
+    assert moe.moe_get_device_error(mws, raise_on_error=False) == 0
+    del g
+
+
+def test_empty_batch_for_training_mx_and_host_calls():
+    """T = 0: nothing is launched except the zeroing of every parameter
+    gradient; the MX and host-buffer calls are no-ops."""
+    w = mw.WORKLOADS["tiny"].with_tokens(0, name="tiny0")
+    widths = moe.ffn_offsets_from_sizes(w.expert_sizes)
+    cfg = moe.MoEConfig(T=0, d_model=w.d_model, E=w.E, k=w.k, ffn_offsets=widths, eps=w.eps)
+    dm, E, F = cfg.d_model, cfg.E, cfg.F
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    x = torch.empty((0, dm), **bf)
+    gamma, Wr = torch.ones((dm,), **bf), torch.zeros((dm, E), **bf)
+    W1, W3, W2 = torch.zeros((dm, F), **bf), torch.zeros((dm, F), **bf), torch.zeros((F, dm), **bf)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    G = [torch.empty((0, dm), **f32), torch.full((dm,), 7.0, **f32), torch.full((dm, E), 7.0, **f32),
+         torch.full((E,), 7.0, **f32), torch.full((dm, F), 7.0, **f32), torch.full((dm, F), 7.0, **f32),
+         torch.full((F, dm), 7.0, **f32)]
+    tws = moe.alloc_train_workspace(cfg)
+    moe.moe_layer_fwd_train(cfg, x, gamma, Wr, None, W1, W3, W2, torch.empty((0, dm), **bf), tws)
+    moe.moe_layer_bwd(cfg, x, gamma, Wr, None, W1, W3, W2, torch.empty((0, dm), **bf), *G, tws)
+    wq = moe.alloc_mx_weights(cfg, W1, W3, W2)
+    moe.moe_layer_fwd_mx(cfg, x, gamma, Wr, None, wq, torch.empty((0, dm), **bf), moe.alloc_mx_workspace(cfg))
+    moe.moe_layer_fwd_host(cfg, torch.empty((0, dm), dtype=torch.bfloat16), gamma, Wr, None, W1, W3, W2,
+                           torch.empty((0, dm), dtype=torch.bfloat16), moe.alloc_host_workspace(cfg))
+    torch.cuda.synchronize()
+    for t in G[1:]:
+        assert int(torch.count_nonzero(t).item()) == 0
