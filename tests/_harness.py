@@ -2,6 +2,7 @@
 the C ABI (staged or fused), and the comparisons against the CPU oracle."""
 from __future__ import annotations
 
+import dataclasses
 from dataclasses import dataclass
 from typing import Dict, Optional
 
@@ -66,6 +67,22 @@ def make_problem(w: mw.Workload) -> Problem:
     W1, W3, W2 = mw.gen_expert_weights(w, widths)
     return Problem(w, widths, mw.gen_x(w), mw.gen_gamma(w), mw.gen_router_weight(w),
                    mw.gen_router_bias(w), W1, W3, W2)
+
+
+def degenerate_problem(w: mw.Workload) -> Problem:
+    """The workload's problem with rows 0-15 of x zero, rows 16-31 scaled by
+    2^12 and rows 32-47 by 2^-12 (exact in bf16), and router column 5 a copy
+    of column 3 (needs T >= 48, E >= 6)."""
+    p = make_problem(w)
+    xf = O.widen_bf16(p.x).astype(np.float32)
+    xf[0:16] = 0.0
+    xf[16:32] *= np.float32(2.0 ** 12)
+    xf[32:48] *= np.float32(2.0 ** -12)
+    Wr = p.Wr.copy()
+    Wr[:, 5] = Wr[:, 3]
+    x = mw.f32_to_bf16_bits(xf)
+    assert np.array_equal(O.widen_bf16(x).astype(np.float32), xf)
+    return dataclasses.replace(p, x=x, Wr=Wr)
 
 
 def make_cfg(p: Problem, renormalize: bool = False) -> moe.MoEConfig:

@@ -39,8 +39,8 @@ def _rel(a, b):
     return float(np.linalg.norm(a - b)) / (n if n > 0 else 1.0)
 
 
-def run_case(w, renormalize=False, bias_override=None):
-    p = H.make_problem(w)
+def run_case(w, renormalize=False, bias_override=None, problem=None):
+    p = H.make_problem(w) if problem is None else problem
     if bias_override is not None:
         p.bias = np.asarray(bias_override, dtype=np.float32)
     cfg = H.make_cfg(p, renormalize=renormalize)
@@ -150,3 +150,13 @@ def test_fine_grained_backward():
     E <= 64 variant of the norm backward and the router backward over 8 slots."""
     w = mw.Workload("bwd_fine", T=300, d_model=256, E=64, k=8, expert_sizes=((64, 128),), bias="normal")
     run_case(w, renormalize=True)
+
+
+def test_degenerate_rows_backward():
+    """Zero rows (r = 1/sqrt(eps), all logits tied at 0), rows scaled by 2^12 and
+    2^-12, and two identical router columns: every gradient within the bar.
+    A zero row has U = V = 0, so H, y, dS, dS3, dgate and the router gradient
+    of that token vanish, and its dx is exactly zero."""
+    w = mw.Workload("bwd_degenerate", T=256, d_model=256, E=8, k=2, expert_sizes=((8, 128),))
+    _, _, G = run_case(w, problem=H.degenerate_problem(w))
+    assert torch.count_nonzero(G["dx"][0:16]).item() == 0

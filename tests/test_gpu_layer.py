@@ -201,3 +201,30 @@ def test_zero_tokens_is_a_no_op():
                       counts=counts)
     assert moe.moe_get_device_error(ws, raise_on_error=False) == 0
     assert counts.cpu().tolist() == [0, 0, 0, 0]
+
+
+def test_degenerate_rows_and_tied_router_columns():
+    """Inputs the method has special cases for:
+    - all-zero rows: r = 1/sqrt(eps), every logit is exactly 0, so the tie rule
+      picks experts 0..k-1 with gates 1/E, and the output row is exactly zero;
+    - rows scaled by 2^12 and by 2^-12 (for the latter eps dominates the mean
+      square, so r is close to 1/sqrt(eps) rather than the row's own scale);
+    - two identical router columns (3 and 5): their logits tie bit-exactly for
+      every token, and expert 5 is never taken ahead of expert 3.
+    """
+    w = W("degenerate", T=256, d_model=256, E=8, k=2, expert_sizes=((8, 128),))
+    p = H.degenerate_problem(w)
+    o, R, D = _full_check(p)
+    idx, gate = o["idx"].cpu().numpy(), o["gate"].cpu().numpy()
+    logits = o["logits"].cpu().numpy()
+    assert np.array_equal(idx[0:16], np.tile([0, 1], (16, 1)))
+    assert np.all(np.abs(gate[0:16] - 1.0 / w.E) <= 1e-7)
+    assert np.all(logits[0:16] == 0.0)
+    assert int(o["out"][0:16].abs().max().item()) == 0
+    assert np.array_equal(logits[:, 3].view(np.uint32), logits[:, 5].view(np.uint32))
+    has3, has5 = np.any(idx == 3, axis=1), np.any(idx == 5, axis=1)
+    assert not np.any(has5 & ~has3), "expert 5 chosen over the tied expert 3"
+    both = has3 & has5
+    assert both.any() and np.all(np.argmax(idx[both] == 3, axis=1) < np.argmax(idx[both] == 5, axis=1))
+    eps_rows = O.rms_stat(O.widen_bf16(p.x[32:48]), w.eps)
+    assert np.all(eps_rows > 0.5 / np.sqrt(w.eps))  # the eps term dominates these rows' statistic

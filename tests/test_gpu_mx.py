@@ -37,8 +37,8 @@ def sf_offset(r, k, K):
     return ((r // 128) * (K // 128) + k // 128) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + (k % 128) // 32
 
 
-def run_mx(w, bias=None):
-    p = H.make_problem(w)
+def run_mx(w, bias=None, problem=None):
+    p = H.make_problem(w) if problem is None else problem
     if bias is not None:
         p.bias = np.asarray(bias, dtype=np.float32)
     cfg = H.make_cfg(p)
@@ -54,6 +54,7 @@ def run_mx(w, bias=None):
 
 SMALL = mw.Workload("mx_var", T=700, d_model=256, E=4, k=2,
                     expert_sizes=((1, 128), (1, 384), (1, 256), (1, 512)))
+SMALL8 = mw.Workload("mx_degenerate", T=300, d_model=256, E=8, k=2, expert_sizes=((8, 128),))
 
 
 def test_weight_codes_and_scales_are_bit_exact():
@@ -76,8 +77,10 @@ def test_weight_codes_and_scales_are_bit_exact():
     np.testing.assert_array_equal(sf2[sf_offset(c, f, F)], s2.T)
 
 
-def test_activation_codes_and_scales_are_bit_exact():
-    p, cfg, d, wq, ws, out = run_mx(SMALL)
+@pytest.mark.parametrize("degenerate", [False, True], ids=["random", "degenerate_rows"])
+def test_activation_codes_and_scales_are_bit_exact(degenerate):
+    """With degenerate rows, zero blocks get scale byte 0 (2^-127) and zero codes."""
+    p, cfg, d, wq, ws, out = run_mx(SMALL8, problem=H.degenerate_problem(SMALL8)) if degenerate else run_mx(SMALL)
     perm = moe.mx_part_view(cfg, wq, ws, "PERM").cpu().numpy()
     offs = moe.mx_part_view(cfg, wq, ws, "OFFSETS").cpu().numpy()
     assert np.all(offs % 128 == 0)
@@ -132,3 +135,11 @@ def test_layer_every_expert_chosen():
     """k = E: every token visits every expert."""
     w = mw.Workload("mx_kE", T=200, d_model=128, E=4, k=4, expert_sizes=((4, 256),))
     _check_layer(*run_mx(w))
+
+
+def test_layer_degenerate_rows():
+    """Zero rows, rows scaled by 2^12 and 2^-12, tied router columns: the layer
+    against the MX oracle, zero rows exactly zero."""
+    p, cfg, d, wq, ws, out = run_mx(SMALL8, problem=H.degenerate_problem(SMALL8))
+    _check_layer(p, cfg, d, wq, ws, out)
+    assert int(out[0:16].abs().max().item()) == 0
