@@ -54,11 +54,15 @@ moe_status_t device_ready(int* sms);
 int gemm_grid_of_current_device();
 moe_status_t cuda_status(cudaError_t e);
 
-// 2-D tensor maps with 128-byte swizzle: bf16 (make_map) or bytes
-// (make_map_u8), `inner` contiguous elements per row, `outer` rows; and the
-// MX scale blocks as a [nblocks, 128] array of 32-bit words (make_map_sf).
+// 2-D tensor maps with 128-byte swizzle (make_map: 64-byte when asked): bf16
+// (make_map), fp32 (make_map_f32) or bytes (make_map_u8), `inner` contiguous
+// elements per row,
+// `outer` rows; and the MX scale blocks as a [nblocks, 128] array of 32-bit
+// words (make_map_sf).
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_elems,
-              uint32_t box_inner, uint32_t box_outer);
+              uint32_t box_inner, uint32_t box_outer, bool swizzle64 = false);
+bool make_map_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_elems,
+                  uint32_t box_inner, uint32_t box_outer);
 bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                  uint32_t box_inner, uint32_t box_outer);
 bool make_map_sf(CUtensorMap* m, const void* base, uint64_t nblocks);

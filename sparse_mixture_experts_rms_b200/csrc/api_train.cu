@@ -85,9 +85,14 @@ moe_status_t run_backward(const moe_config_t& c, const Layout& L, void* ws, cons
     g.out_ds3 = static_cast<__nv_bfloat16*>(dS3);
     g.drp = at<float>(ws, L.drp);
     g.ld_drp = L.ld_drp;
-    if (!make_map(&mA0, dY, d, rows, d, 64, 128) || !make_map(&mB0, W2, d, F, d, 64, bn_h / 2))
+    EpiMaps em{};
+    if (!make_map(&mA0, dY, d, rows, d, 64, 128) || !make_map(&mB0, W2, d, F, d, 64, bn_h / 2) ||
+        !make_map(&em.m[0], g.in_u, ldh, rows, ldh, 32, 32, true) ||
+        !make_map(&em.m[1], g.in_v, ldh, rows, ldh, 32, 32, true) ||
+        !make_map(&em.m[2], dS, ldh, rows, ldh, 32, 32, true) ||
+        !make_map(&em.m[3], dS3, ldh, rows, ldh, 32, 32, true))
       return MOE_ERR_CUDA;
-    if ((st = cuda_status(launch_grouped_gemm(g, mA0, mA0, mB0, mB0, grid, s))) != MOE_OK) return st;
+    if ((st = cuda_status(launch_grouped_gemm(g, mA0, mA0, mB0, mB0, grid, s, &em))) != MOE_OK) return st;
   }
   {  // dX per kept row: [dS | dS3] x [W1 | W3]^T (W rows, K-major)
     GemmArgs g{};
@@ -96,10 +101,12 @@ moe_status_t run_backward(const moe_config_t& c, const Layout& L, void* ws, cons
     g.bn = bn_d;
     g.out_f0 = at<float>(ws, L.dXp);
     g.ld_f = c.d_model;
+    EpiMaps em{};
     if (!make_map(&mA0, dS, ldh, rows, ldh, 64, 128) || !make_map(&mA1, dS3, ldh, rows, ldh, 64, 128) ||
-        !make_map(&mB0, W1, F, d, F, 64, bn_d / 2) || !make_map(&mB1, W3, F, d, F, 64, bn_d / 2))
+        !make_map(&mB0, W1, F, d, F, 64, bn_d / 2) || !make_map(&mB1, W3, F, d, F, 64, bn_d / 2) ||
+        !make_map_f32(&em.m[0], g.out_f0, d, rows, d, 32, 32))
       return MOE_ERR_CUDA;
-    if ((st = cuda_status(launch_grouped_gemm(g, mA0, mA1, mB0, mB1, grid, s))) != MOE_OK) return st;
+    if ((st = cuda_status(launch_grouped_gemm(g, mA0, mA1, mB0, mB1, grid, s, &em))) != MOE_OK) return st;
   }
   {  // dW1 | dW3 = x_perm^T [dS | dS3]  (both operands MN-major, K = rows)
     GemmArgs g{};
@@ -109,10 +116,12 @@ moe_status_t run_backward(const moe_config_t& c, const Layout& L, void* ws, cons
     g.out_f0 = dW1;
     g.out_f1 = dW3;
     g.ld_f = static_cast<int>(F);
+    EpiMaps em{};
     if (!make_map(&mA0, at<void>(ws, L.x_perm), d, rows, d, 64, 64) ||
-        !make_map(&mB0, dS, ldh, rows, ldh, 64, 64) || !make_map(&mB1, dS3, ldh, rows, ldh, 64, 64))
+        !make_map(&mB0, dS, ldh, rows, ldh, 64, 64) || !make_map(&mB1, dS3, ldh, rows, ldh, 64, 64) ||
+        !make_map_f32(&em.m[0], dW1, F, d, F, 32, 32) || !make_map_f32(&em.m[1], dW3, F, d, F, 32, 32))
       return MOE_ERR_CUDA;
-    if ((st = cuda_status(launch_grouped_gemm(g, mA0, mA0, mB0, mB1, grid, s))) != MOE_OK) return st;
+    if ((st = cuda_status(launch_grouped_gemm(g, mA0, mA0, mB0, mB1, grid, s, &em))) != MOE_OK) return st;
   }
   {  // dW2 = H^T dY
     GemmArgs g{};
@@ -121,9 +130,11 @@ moe_status_t run_backward(const moe_config_t& c, const Layout& L, void* ws, cons
     g.bn = bn_d;
     g.out_f0 = dW2;
     g.ld_f = c.d_model;
-    if (!make_map(&mA0, at<void>(ws, L.H), ldh, rows, ldh, 64, 64) || !make_map(&mB0, dY, d, rows, d, 64, 64))
+    EpiMaps em{};
+    if (!make_map(&mA0, at<void>(ws, L.H), ldh, rows, ldh, 64, 64) || !make_map(&mB0, dY, d, rows, d, 64, 64) ||
+        !make_map_f32(&em.m[0], dW2, d, F, d, 32, 32))
       return MOE_ERR_CUDA;
-    if ((st = cuda_status(launch_grouped_gemm(g, mA0, mA0, mB0, mB0, grid, s))) != MOE_OK) return st;
+    if ((st = cuda_status(launch_grouped_gemm(g, mA0, mA0, mB0, mB0, grid, s, &em))) != MOE_OK) return st;
   }
   if ((st = cuda_status(launch_bwd_route(b, s))) != MOE_OK) return st;
   if ((st = cuda_status(launch_bwd_norm(b, s))) != MOE_OK) return st;

@@ -47,13 +47,24 @@
 //
 // Warp roles (192 threads per CTA): warp 0 = TMA producer, warp 1 = MMA issuer
 // (leader only) and TMEM owner, warps 2..5 = epilogue (TMEM -> registers ->
-// global), one per TMEM lane quarter.  (Eight epilogue warps, two per quarter
-// on column halves, measured 5% faster on the dS GEMM and 2.5-5% slower on
-// every other mode: the extra warps share sub-partitions with the producer
-// and MMA warps.)  Ring of 6 stages x (A 16 KB + B 16 KB) per CTA; two TMEM
-// accumulators of 256 fp32 columns, so the epilogue of tile i overlaps the
-// mainloop of tile i+1.  Every wait is bounded (4 s) and sets a device error
-// bit instead of hanging.
+// shared -> TMA store), one per TMEM lane quarter.  (Eight epilogue warps, two
+// per quarter on column halves, measured 5% faster on the dS GEMM and 2.5-5%
+// slower on every other mode: the extra warps share sub-partitions with the
+// producer and MMA warps.)  Ring of 6 stages x (A 16 KB + B 16 KB) per CTA;
+// two TMEM accumulators of 256 fp32 columns, so the epilogue of tile i
+// overlaps the mainloop of tile i+1.
+//
+// Epilogue output: a thread holds one accumulator row, so storing rows
+// directly makes every warp-wide store touch 32 rows in 16-byte pieces, which
+// costs the load/store path 8x the wavefronts of whole-row segments and slows
+// the MMAs sharing it (measured 5-7% on the training up, dS and weight-
+// gradient GEMMs).  Instead each epilogue warp writes its 32 rows of a
+// 32-column chunk into a swizzled 32 x 32 box in shared memory (conflict-free:
+// lane = row) and one lane stores the box by TMA; 8 KB of boxes per warp form
+// a ring.  The dS GEMM also loads its saved U, V chunks as boxes by TMA.  A
+// box is used when the warp's 32 rows all belong to the expert (always in the
+// 64-row-padded training layout); otherwise the threads store their rows.
+// Every wait is bounded (4 s) and sets a device error bit instead of hanging.
 #include "moe_internal.h"
 #include "ptx.cuh"
 
@@ -73,6 +84,11 @@ constexpr int kTmemCols = 512;
 constexpr int kAccCols = 256;                 // columns per accumulator buffer
 constexpr int kAtomBytes = BK * 64 * 2;       // one 64(mn) x 64(k) MN-major box: 8 KB
 constexpr long long kL2GroupBudget = 48ll << 20;  // A bytes of one raster group
+// Epilogue staging: per epilogue warp four 32-row x 32-column bf16 boxes
+// (2 KB each, 64-byte swizzle) through which up, down and bwd_h move their
+// rows by TMA
+constexpr int kEpiBoxBytes = 32 * 32 * 2;
+constexpr int kEpiBytes = kEpiWarps * 4 * kEpiBoxBytes;  // 32 KB
 
 struct __align__(8) GemmShared {
   uint64_t full[kStages];    // leader: both CTAs' loads of a stage landed
@@ -80,6 +96,7 @@ struct __align__(8) GemmShared {
   uint64_t tfull[2];         // each CTA: accumulator buffer ready
   uint64_t tempty[2];        // leader: both CTAs' epilogues drained the buffer
   uint64_t drain;
+  uint64_t ebar[kEpiWarps][2];  // bwd_h: an epilogue warp's U, V box pair landed
   uint32_t tmem_base;
   int abort_flag;
   int bad_segment;
@@ -93,7 +110,9 @@ struct __align__(8) GemmShared {
   int seg[kMaxExperts + 1];
 };
 
-constexpr size_t kSmemBytes = 1024 /* alignment slack */ + kStages * kStageBytes + sizeof(GemmShared);
+// [stages | bwd_h epilogue staging | GemmShared]
+constexpr size_t kSmemBytes = 1024 /* alignment slack */ + kStages * kStageBytes + kEpiBytes + sizeof(GemmShared);
+static_assert(kSmemBytes <= 232448, "shared memory above the per-block opt-in limit");
 
 struct TileCoord {
   int e, nt, mt;
@@ -136,12 +155,6 @@ __device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const uint32_
   uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
   for (int j = 0; j < 4; ++j) d4[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-}
-
-__device__ __forceinline__ void store_zero_bf16(__nv_bfloat16* dst) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) d4[j] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 __device__ __forceinline__ void store_row_f32(float* dst, const uint32_t (&u)[32], bool zero) {
@@ -236,151 +249,274 @@ __device__ __forceinline__ void issue_loads(const Maps& m, const TileCoord& c, i
 }
 
 // ---- epilogues: one thread per accumulator row (TMEM lane), 32 columns per load
+// Byte offset of 16-byte unit `unit` (0..3) of row `row` in a box of 64-byte
+// rows under TMA's 64-byte swizzle (unit bits [4,6) ^= address bits [7,9)).
+__device__ __forceinline__ uint32_t sw64(int row, int unit) {
+  return static_cast<uint32_t>(row * 64 + ((unit ^ ((row >> 1) & 3)) << 4));
+}
+
+// One lane's row (32 bf16 = 16 words) into a staged 32 x 32 box.
+__device__ __forceinline__ void box_put_row(uint8_t* box, int lane, const uint32_t (&o)[16]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4*>(box + sw64(lane, j)) = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+}
+
+// One lane's row (32 fp32) into a staged 32 x 32 fp32 box of 128-byte rows
+// under TMA's 128-byte swizzle (unit bits [4,7) ^= address bits [7,10)).
+__device__ __forceinline__ void box_put_row_f32(uint8_t* box, int lane, const uint32_t (&u)[32], bool zero) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+        zero ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(u[4 * j], u[4 * j + 1], u[4 * j + 2], u[4 * j + 3]);
+}
+
+// Staged output of a warp: `nbox` boxes per 32-column chunk in a ring of
+// 4 / nbox slots (the warp's 8 KB).  Before a slot is rewritten, lane 0 waits
+// until at most (slots - 1) of its bulk-store groups -- one per chunk -- are
+// still reading shared memory.
+__device__ __forceinline__ uint8_t* box_slot_acquire(uint8_t* boxes, int nbox, uint32_t n, int lane) {
+  const int slots = 4 / nbox;
+  if (lane == 0) bulk_wait_group_read_allow(slots - 1);
+  __syncwarp();
+  return boxes + (n % static_cast<uint32_t>(slots)) * nbox * kEpiBoxBytes;
+}
+
+// After every lane wrote its rows of the slot's boxes: lane 0 stores box b
+// with map m[b] at (x, p0), one bulk group for the chunk.
+__device__ __forceinline__ void box_slot_store(const EpiMaps& em, uint8_t* slot, int nbox, int x, int p0,
+                                               int lane) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    for (int b = 0; b < nbox; ++b) tma_store_2d(&em.m[b], slot + b * kEpiBoxBytes, x, p0);
+    bulk_commit_group();
+  }
+}
+
+// Row-tile epilogues (up, down, bwd_x); one thread per accumulator row
+// (TMEM lane), 32-column chunks.  The outputs leave through shared memory by
+// TMA when the warp's 32 rows all belong to the expert (`staged`); otherwise
+// each thread stores its own row.  Padding rows of the training layout
+// (perm = -1) get zeros.
 template <int MODE>
-__device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShared& sh, const TileCoord& c,
-                                              uint32_t taddr, int row_in_cta, uint32_t rank) {
-  const int p = sh.seg[c.e] + c.mt * BM + static_cast<int>(rank) * BM_CTA + row_in_cta;
+__device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShared& sh, const EpiMaps& em,
+                                              const TileCoord& c, uint32_t taddr, int q, int lane,
+                                              uint32_t rank, uint8_t* boxes, uint32_t& n) {
+  const int p0 = sh.seg[c.e] + c.mt * BM + static_cast<int>(rank) * BM_CTA + q * 32;
+  const int p = p0 + lane;
   const bool valid = p < sh.seg[c.e + 1];
+  const bool staged = a.staged != 0 && p0 + 32 <= sh.seg[c.e + 1];
   const int asg = valid ? a.perm[p] : -1;
-  const bool pad = valid && asg < 0;  // padding row of the training layout: zeros out
+  const bool pad = valid && asg < 0;
   const size_t prow = static_cast<size_t>(valid ? p : 0);
   if (MODE == kGemmUp) {
     const float scale = asg >= 0 ? a.scale[asg / a.k] : 0.f;
     const size_t off = prow * a.ld_out + c.nt * kBlockN;
+    const bool keep_uv = a.out_u != nullptr;
+    const int nbox = keep_uv ? 3 : 1;
 #pragma unroll 1
     for (int cc = 0; cc < kBlockN; cc += 32) {
       uint32_t u[32], v[32];
       tmem_ld_32x32b_x32(taddr + cc, u);
       tmem_ld_32x32b_x32(taddr + kBlockN + cc, v);
       tmem_ld_wait();
-      if (!valid) continue;
-      if (pad) {
-        store_zero_bf16(a.out + off + cc);
-        if (a.out_u != nullptr) {
-          store_zero_bf16(a.out_u + off + cc);
-          store_zero_bf16(a.out_v + off + cc);
-        }
-        continue;
-      }
+      if (!valid) continue;  // never taken when staged
       uint32_t o[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float h0 = silu(scale * __uint_as_float(u[2 * j])) * (scale * __uint_as_float(v[2 * j]));
         const float h1 = silu(scale * __uint_as_float(u[2 * j + 1])) * (scale * __uint_as_float(v[2 * j + 1]));
-        o[j] = pack_bf16(h0, h1);
+        o[j] = pad ? 0u : pack_bf16(h0, h1);
       }
-      store_row_bf16(a.out + off + cc, o);
-      if (a.out_u != nullptr) {
+      uint8_t* slot = nullptr;
+      if (staged) {
+        slot = box_slot_acquire(boxes, nbox, n++, lane);
+        box_put_row(slot, lane, o);
+      } else {
+        store_row_bf16(a.out + off + cc, o);
+      }
+      if (keep_uv) {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-          o[j] = pack_bf16(scale * __uint_as_float(u[2 * j]), scale * __uint_as_float(u[2 * j + 1]));
-        store_row_bf16(a.out_u + off + cc, o);
+          o[j] = pad ? 0u : pack_bf16(scale * __uint_as_float(u[2 * j]), scale * __uint_as_float(u[2 * j + 1]));
+        if (staged) box_put_row(slot + kEpiBoxBytes, lane, o);
+        else store_row_bf16(a.out_u + off + cc, o);
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-          o[j] = pack_bf16(scale * __uint_as_float(v[2 * j]), scale * __uint_as_float(v[2 * j + 1]));
-        store_row_bf16(a.out_v + off + cc, o);
+          o[j] = pad ? 0u : pack_bf16(scale * __uint_as_float(v[2 * j]), scale * __uint_as_float(v[2 * j + 1]));
+        if (staged) box_put_row(slot + 2 * kEpiBoxBytes, lane, o);
+        else store_row_bf16(a.out_v + off + cc, o);
       }
+      if (staged) box_slot_store(em, slot, nbox, c.nt * kBlockN + cc, p0, lane);
     }
   } else if (MODE == kGemmDown) {
     const float scale = asg >= 0 ? a.scale[asg] : 0.f;
     const size_t off = prow * a.ld_out + c.nt * a.bn;
+    const bool keep_yu = a.out_yu != nullptr;
+    const int nbox = keep_yu ? 2 : 1;
 #pragma unroll 1
     for (int cc = 0; cc < a.bn; cc += 32) {
       uint32_t u[32];
       tmem_ld_32x32b_x32(taddr + cc, u);
       tmem_ld_wait();
-      if (!valid) continue;
-      if (pad) {
-        store_zero_bf16(a.out + off + cc);
-        if (a.out_yu != nullptr) store_zero_bf16(a.out_yu + off + cc);
-        continue;
-      }
+      if (!valid) continue;  // never taken when staged
       uint32_t o[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        o[j] = pack_bf16(scale * __uint_as_float(u[2 * j]), scale * __uint_as_float(u[2 * j + 1]));
-      store_row_bf16(a.out + off + cc, o);
-      if (a.out_yu != nullptr) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) o[j] = pack_bf16(__uint_as_float(u[2 * j]), __uint_as_float(u[2 * j + 1]));
-        store_row_bf16(a.out_yu + off + cc, o);
+        o[j] = pad ? 0u : pack_bf16(scale * __uint_as_float(u[2 * j]), scale * __uint_as_float(u[2 * j + 1]));
+      uint8_t* slot = nullptr;
+      if (staged) {
+        slot = box_slot_acquire(boxes, nbox, n++, lane);
+        box_put_row(slot, lane, o);
+      } else {
+        store_row_bf16(a.out + off + cc, o);
       }
+      if (keep_yu) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          o[j] = pad ? 0u : pack_bf16(__uint_as_float(u[2 * j]), __uint_as_float(u[2 * j + 1]));
+        if (staged) box_put_row(slot + kEpiBoxBytes, lane, o);
+        else store_row_bf16(a.out_yu + off + cc, o);
+      }
+      if (staged) box_slot_store(em, slot, nbox, c.nt * a.bn + cc, p0, lane);
     }
-  } else if (MODE == kGemmBwdH) {
-    const float r = asg >= 0 ? a.scale[asg / a.k] : 0.f;
-    const size_t off = prow * a.ld_out + c.nt * a.bn;
-    float dr = 0.f;
-#pragma unroll 1
-    for (int cc = 0; cc < a.bn; cc += 32) {
-      // the saved U, V of this chunk are fetched while the accumulator is read
-      uint4 ur[4], vr[4];
-      if (valid && !pad) {
-        const uint4* u4 = reinterpret_cast<const uint4*>(a.in_u + off + cc);
-        const uint4* v4 = reinterpret_cast<const uint4*>(a.in_v + off + cc);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          ur[j] = u4[j];
-          vr[j] = v4[j];
-        }
-      }
-      uint32_t g[32];
-      tmem_ld_32x32b_x32(taddr + cc, g);
-      tmem_ld_wait();
-      if (!valid) continue;
-      if (pad) {
-        store_zero_bf16(a.out_ds + off + cc);
-        store_zero_bf16(a.out_ds3 + off + cc);
-        continue;
-      }
-      uint32_t uw[16], vw[16];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uw[4 * j] = ur[j].x; uw[4 * j + 1] = ur[j].y; uw[4 * j + 2] = ur[j].z; uw[4 * j + 3] = ur[j].w;
-        vw[4 * j] = vr[j].x; vw[4 * j + 1] = vr[j].y; vw[4 * j + 2] = vr[j].z; vw[4 * j + 3] = vr[j].w;
-      }
-      uint32_t o1[16], o3[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        float du[2], dv[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float uu = h ? bf16_hi(uw[j]) : bf16_lo(uw[j]);
-          const float vv = h ? bf16_hi(vw[j]) : bf16_lo(vw[j]);
-          const float gg = __uint_as_float(g[2 * j + h]);
-          const float sg = sigmoid(uu);
-          du[h] = gg * vv * (sg * (1.0f + uu * (1.0f - sg)));
-          dv[h] = gg * (uu * sg);
-          dr += du[h] * uu + dv[h] * vv;
-        }
-        o1[j] = pack_bf16(r * du[0], r * du[1]);
-        o3[j] = pack_bf16(r * dv[0], r * dv[1]);
-      }
-      store_row_bf16(a.out_ds + off + cc, o1);
-      store_row_bf16(a.out_ds3 + off + cc, o3);
-    }
-    if (valid) a.drp[prow * a.ld_drp + c.nt] = pad ? 0.f : dr / r;
-  } else {  // kGemmBwdX
+  } else {  // kGemmBwdX: fp32 rows, staged as 32 x 32 fp32 boxes (128-byte swizzle, two per warp)
     float* dst = a.out_f0 + prow * a.ld_f + c.nt * a.bn;
 #pragma unroll 1
     for (int cc = 0; cc < a.bn; cc += 32) {
       uint32_t u[32];
       tmem_ld_32x32b_x32(taddr + cc, u);
       tmem_ld_wait();
-      if (valid) store_row_f32(dst + cc, u, pad);
+      if (!valid) continue;  // never taken when staged
+      if (staged) {
+        uint8_t* box = boxes + (n++ & 1u) * 2 * kEpiBoxBytes;
+        if (lane == 0) bulk_wait_group_read_allow(1);
+        __syncwarp();
+        box_put_row_f32(box, lane, u, pad);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&em.m[0], box, c.nt * a.bn + cc, p0);
+          bulk_commit_group();
+        }
+      } else {
+        store_row_f32(dst + cc, u, pad);
+      }
     }
   }
 }
 
+// bwd_h epilogue of one warp: its 32 accumulator rows (TMEM lane quarter q)
+// in 32-column chunks.  The saved U, V chunks come in and dS, dS3 go out as
+// whole 32 x 32 boxes through shared memory by TMA, so global memory sees
+// contiguous row segments; each lane reads and writes its own row of the
+// boxes, conflict-free under the swizzle.  Two box pairs per warp form a
+// ring: chunk n reads U, V from pair n % 2, overwrites them with dS, dS3 and
+// stores them from there, while chunk n + 1's U, V load into the other pair
+// (once that pair's previous store has read it out).  The training layout
+// pads every expert segment to a multiple of 64 rows, so a box lies entirely
+// inside or entirely past the expert's rows.  `n` counts this warp's chunks
+// across tiles.  Returns false when a wait gave up.
+__device__ __forceinline__ bool epilogue_dsh(const GemmArgs& a, const GemmShared& sh, const EpiMaps& em,
+                                             const TileCoord& c, uint32_t taddr, int q, int lane, uint32_t rank,
+                                             uint8_t* boxes, uint64_t* bars, uint32_t& n, volatile int* abort_flag) {
+  const int p0 = sh.seg[c.e] + c.mt * BM + static_cast<int>(rank) * BM_CTA + q * 32;
+  if (p0 >= sh.seg[c.e + 1]) return true;
+  const int p = p0 + lane;
+  const int asg = a.perm[p];
+  const bool pad = asg < 0;  // padding row: zeros out
+  const float r = pad ? 0.f : a.scale[asg / a.k];
+  const int col0 = c.nt * a.bn;
+  auto load_uv = [&](uint32_t slot, int col) {  // lane 0
+    uint8_t* bx = boxes + slot * 2 * kEpiBoxBytes;
+    bulk_wait_group_read0();  // the slot's previous store has read it
+    mbar_arrive_expect_tx(&bars[slot], 2 * kEpiBoxBytes);
+    tma_load_2d(bx, &em.m[0], &bars[slot], col, p0);
+    tma_load_2d(bx + kEpiBoxBytes, &em.m[1], &bars[slot], col, p0);
+  };
+  if (lane == 0) load_uv(n & 1u, col0);
+  float dr = 0.f;
+#pragma unroll 1
+  for (int cc = 0; cc < a.bn; cc += 32, ++n) {
+    const uint32_t slot = n & 1u;
+    uint8_t* s_u = boxes + slot * 2 * kEpiBoxBytes;
+    uint8_t* s_v = s_u + kEpiBoxBytes;
+    uint32_t g[32];
+    tmem_ld_32x32b_x32(taddr + cc, g);
+    if (lane == 0 && cc + 32 < a.bn) load_uv(slot ^ 1u, col0 + cc + 32);
+    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars[slot], (n >> 1) & 1u, abort_flag, a.err,
+                                                     MOE_DEVERR_TIMEOUT, kWaitTimeoutNs));
+    tmem_ld_wait();
+    if (!ok) {
+      if (lane == 0) {  // let the loads in flight land (bounded) before giving up
+        volatile int no_abort = 0;
+        mbar_wait(&bars[slot], (n >> 1) & 1u, &no_abort, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs);
+        if (cc + 32 < a.bn)
+          mbar_wait(&bars[slot ^ 1u], ((n + 1) >> 1) & 1u, &no_abort, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs);
+      }
+      return false;
+    }
+    uint32_t uw[16], vw[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 u4 = *reinterpret_cast<const uint4*>(s_u + sw64(lane, j));
+      const uint4 v4 = *reinterpret_cast<const uint4*>(s_v + sw64(lane, j));
+      uw[4 * j] = u4.x; uw[4 * j + 1] = u4.y; uw[4 * j + 2] = u4.z; uw[4 * j + 3] = u4.w;
+      vw[4 * j] = v4.x; vw[4 * j + 1] = v4.y; vw[4 * j + 2] = v4.z; vw[4 * j + 3] = v4.w;
+    }
+    uint32_t o1[16], o3[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      float du[2], dv[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float uu = h ? bf16_hi(uw[j]) : bf16_lo(uw[j]);
+        const float vv = h ? bf16_hi(vw[j]) : bf16_lo(vw[j]);
+        const float gg = __uint_as_float(g[2 * j + h]);
+        const float sg = sigmoid(uu);
+        du[h] = gg * vv * (sg * (1.0f + uu * (1.0f - sg)));
+        dv[h] = gg * (uu * sg);
+        dr += du[h] * uu + dv[h] * vv;
+      }
+      o1[j] = pad ? 0u : pack_bf16(r * du[0], r * du[1]);
+      o3[j] = pad ? 0u : pack_bf16(r * dv[0], r * dv[1]);
+    }
+    // each lane overwrites only its own row of the boxes it has just read
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      *reinterpret_cast<uint4*>(s_u + sw64(lane, j)) = make_uint4(o1[4 * j], o1[4 * j + 1], o1[4 * j + 2], o1[4 * j + 3]);
+      *reinterpret_cast<uint4*>(s_v + sw64(lane, j)) = make_uint4(o3[4 * j], o3[4 * j + 1], o3[4 * j + 2], o3[4 * j + 3]);
+    }
+    fence_proxy_async_smem();  // the boxes' writes are visible to the TMA stores
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(&em.m[2], s_u, col0 + cc, p0);
+      tma_store_2d(&em.m[3], s_v, col0 + cc, p0);
+      bulk_commit_group();
+    }
+  }
+  a.drp[static_cast<size_t>(p) * a.ld_drp + c.nt] = pad ? 0.f : dr / r;
+  return true;
+}
+
 // Weight gradients: the accumulator row is an output row of dW (a column of
-// x_perm or H); an expert with no rows gets zeros.
+// x_perm or H); an expert with no rows gets zeros.  The fp32 rows leave
+// through shared memory by TMA (32 x 32 fp32 boxes, 128-byte swizzle, a ring
+// of two per warp) when tensor maps were given; every box is whole, since d
+// and the expert widths are multiples of 128.
 template <int MODE>
-__device__ __forceinline__ void epilogue_wgrad(const GemmArgs& a, const GemmShared& sh, const TileCoord& c,
-                                               uint32_t taddr, int row_in_cta, uint32_t rank) {
+__device__ __forceinline__ void epilogue_wgrad(const GemmArgs& a, const GemmShared& sh, const EpiMaps& em,
+                                               const TileCoord& c, uint32_t taddr, int q, int lane,
+                                               uint32_t rank, uint8_t* boxes, uint32_t& n) {
   const int o_e = a.ffn.off[c.e];
   const int f = a.ffn.off[c.e + 1] - o_e;
-  const int m = c.mt * BM + static_cast<int>(rank) * BM_CTA + row_in_cta;
+  const int m0 = c.mt * BM + static_cast<int>(rank) * BM_CTA + q * 32;
+  const int m = m0 + lane;
   const bool zero = sh.k_blocks[c.e] == 0;
-  const bool valid = m < (MODE == kGemmWgradX ? a.d : f);
+  const int m_end = MODE == kGemmWgradX ? a.d : f;
+  const bool valid = m < m_end;
+  const bool staged = a.staged != 0 && m0 + 32 <= m_end;
 #pragma unroll 1
   for (int cc = 0; cc < a.bn; cc += 32) {
     uint32_t u[32];
@@ -388,14 +524,30 @@ __device__ __forceinline__ void epilogue_wgrad(const GemmArgs& a, const GemmShar
       tmem_ld_32x32b_x32(taddr + cc, u);
       tmem_ld_wait();
     }
-    if (!valid) continue;
-    const int n = c.nt * a.bn + cc;
+    if (!valid) continue;  // never taken when staged
+    const int nn = c.nt * a.bn + cc;
+    if (staged) {
+      uint8_t* box = boxes + (n++ & 1u) * 2 * kEpiBoxBytes;  // 4 KB fp32 box
+      if (lane == 0) bulk_wait_group_read_allow(1);
+      __syncwarp();
+      box_put_row_f32(box, lane, u, zero);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (MODE == kGemmWgradX)
+          tma_store_2d(&em.m[nn < f ? 0 : 1], box, o_e + (nn < f ? nn : nn - f), m0);
+        else
+          tma_store_2d(&em.m[0], box, nn, o_e + m0);
+        bulk_commit_group();
+      }
+      continue;
+    }
     float* dst;
     if (MODE == kGemmWgradX)
-      dst = (n < f ? a.out_f0 + static_cast<size_t>(m) * a.ld_f + o_e + n
-                   : a.out_f1 + static_cast<size_t>(m) * a.ld_f + o_e + (n - f));
+      dst = (nn < f ? a.out_f0 + static_cast<size_t>(m) * a.ld_f + o_e + nn
+                    : a.out_f1 + static_cast<size_t>(m) * a.ld_f + o_e + (nn - f));
     else
-      dst = a.out_f0 + static_cast<size_t>(o_e + m) * a.ld_f + n;
+      dst = a.out_f0 + static_cast<size_t>(o_e + m) * a.ld_f + nn;
     store_row_f32(dst, u, zero);
   }
 }
@@ -404,10 +556,11 @@ template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                         const __grid_constant__ CUtensorMap mapB0, const __grid_constant__ CUtensorMap mapB1,
-                        const __grid_constant__ GemmArgs a) {
+                        const __grid_constant__ GemmArgs a, const __grid_constant__ EpiMaps em) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  GemmShared& sh = *reinterpret_cast<GemmShared*>(smem + kStages * kStageBytes);
+  uint8_t* epi_boxes = smem + kStages * kStageBytes;
+  GemmShared& sh = *reinterpret_cast<GemmShared*>(epi_boxes + kEpiBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = a.E;
   const uint32_t rank = cluster_ctarank();      // 0 = leader, 1 = peer
@@ -425,6 +578,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&sh.tempty[b], 2 * kEpiWarps);
     }
     mbar_init(&sh.drain, 1);
+    for (int w = 0; w < kEpiWarps; ++w) {
+      mbar_init(&sh.ebar[w][0], 1);
+      mbar_init(&sh.ebar[w][1], 1);
+    }
     sh.abort_flag = 0;
     sh.bad_segment = 0;
     fence_mbar_init();
@@ -434,6 +591,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tma_prefetch_map(&mapB0);
     if (MODE == kGemmBwdX) tma_prefetch_map(&mapA1);
     if (MODE == kGemmUp || MODE == kGemmBwdX || MODE == kGemmWgradX) tma_prefetch_map(&mapB1);
+    if (MODE == kGemmBwdH)
+      for (int i = 0; i < 4; ++i) tma_prefetch_map(&em.m[i]);
   }
   if (warp == 1) {
     tmem_alloc_pair(&sh.tmem_base, kTmemCols);
@@ -448,6 +607,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     geometry<MODE>(rows, f, a.d, a.bn, mext, nt, kb);
     // K of the weight gradients is a row segment: it must be whole K blocks
     if (!Traits<MODE>::row_tiles && (rows < 0 || rows % BK != 0)) sh.bad_segment = 1;
+    // bwd_h moves 32-row boxes: segments must start and end on 32-row boundaries
+    if (MODE == kGemmBwdH && (sh.seg[tid] % 32 != 0 || rows < 0 || rows % 32 != 0)) sh.bad_segment = 1;
     const int mt = (mext + BM - 1) / BM;
     const long long a_panel = static_cast<long long>(BM) * kb * BK * 2;  // one M tile's A over all K
     const long long b_panel = static_cast<long long>(a.bn) * kb * BK * 2;  // one N tile's B over all K
@@ -570,9 +731,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else {
     // ================= epilogue (warps 2..5): a warp reads TMEM lane quarter warp % 4
     const int q = warp & 3;
-    const int row_in_cta = q * 32 + lane;
     const uint32_t tempty_leader0 = map_to_cta(smem_addr(&sh.tempty[0]), 0);
-    uint32_t tcount = 0;
+    uint32_t tcount = 0, eit = 0;
     for (int tile = pair; tile < total; tile += npairs, ++tcount) {
       const TileCoord c = decode_tile(sh, E, tile);
       const uint32_t buf = tcount & 1u;
@@ -584,14 +744,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kAccCols;
-      if (Traits<MODE>::row_tiles)
-        epilogue_rows<MODE>(a, sh, c, taddr, row_in_cta, rank);
+      if (MODE == kGemmBwdH)
+        ok = epilogue_dsh(a, sh, em, c, taddr, q, lane, rank, epi_boxes + (warp - 2) * 4 * kEpiBoxBytes,
+                          sh.ebar[warp - 2], eit, abort_flag);
+      else if (Traits<MODE>::row_tiles)
+        epilogue_rows<MODE>(a, sh, em, c, taddr, q, lane, rank, epi_boxes + (warp - 2) * 4 * kEpiBoxBytes, eit);
       else
-        epilogue_wgrad<MODE>(a, sh, c, taddr, row_in_cta, rank);
+        epilogue_wgrad<MODE>(a, sh, em, c, taddr, q, lane, rank, epi_boxes + (warp - 2) * 4 * kEpiBoxBytes, eit);
       tc_fence_before();
       __syncwarp();
+      if (!ok) break;
       if (lane == 0) mbar_arrive_cluster(tempty_leader0 + buf * 8u);
     }
+    // the staged stores have completed before the CTA's shared memory goes away
+    if (lane == 0) bulk_wait_group0();
   }
 
   // ---- teardown: neither CTA leaves while its pair may still touch its memory
@@ -640,26 +806,31 @@ int grouped_gemm_max_grid(int num_sms) {
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA0, const CUtensorMap& mapA1,
                                 const CUtensorMap& mapB0, const CUtensorMap& mapB1, int grid,
-                                cudaStream_t s) {
+                                cudaStream_t s, const EpiMaps* em_opt) {
   if (a.bn != 128 && a.bn != 256) return cudaErrorInvalidValue;
+  if (a.mode == kGemmBwdH && em_opt == nullptr) return cudaErrorInvalidValue;
+  static const EpiMaps kNoMaps{};
+  const EpiMaps& em = em_opt != nullptr ? *em_opt : kNoMaps;
+  GemmArgs ga = a;
+  ga.staged = em_opt != nullptr ? 1 : 0;
   switch (a.mode) {
     case kGemmUp:
-      grouped_gemm_kernel<kGemmUp><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, a);
+      grouped_gemm_kernel<kGemmUp><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmDown:
-      grouped_gemm_kernel<kGemmDown><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, a);
+      grouped_gemm_kernel<kGemmDown><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmBwdH:
-      grouped_gemm_kernel<kGemmBwdH><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, a);
+      grouped_gemm_kernel<kGemmBwdH><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmBwdX:
-      grouped_gemm_kernel<kGemmBwdX><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, a);
+      grouped_gemm_kernel<kGemmBwdX><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmWgradX:
-      grouped_gemm_kernel<kGemmWgradX><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, a);
+      grouped_gemm_kernel<kGemmWgradX><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmWgradH:
-      grouped_gemm_kernel<kGemmWgradH><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, a);
+      grouped_gemm_kernel<kGemmWgradH><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     default:
       return cudaErrorInvalidValue;

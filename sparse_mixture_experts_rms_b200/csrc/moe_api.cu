@@ -200,14 +200,27 @@ int gemm_grid_of_current_device() {
 // 2-D bf16 tensor map with 128-byte swizzle: `inner` contiguous elements per
 // row, `outer` rows, `row_elems` elements between rows; box inner x outer.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_elems,
-              uint32_t box_inner, uint32_t box_outer) {
+              uint32_t box_inner, uint32_t box_outer, bool swizzle64) {
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_elems * 2};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D fp32 tensor map, 128-byte swizzle, box inner x outer.
+bool make_map_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_elems,
+                  uint32_t box_inner, uint32_t box_outer) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_elems * 4};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 2-D E4M3 (byte) tensor map, 128-byte swizzle, box inner x outer.
@@ -345,8 +358,14 @@ moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_
   g.ld_out = L.ldh;
   g.out_u = reinterpret_cast<__nv_bfloat16*>(U);
   g.out_v = reinterpret_cast<__nv_bfloat16*>(V);
+  const uint64_t ldh = static_cast<uint64_t>(L.ldh);
+  EpiMaps em{};
+  if (!make_map(&em.m[0], g.out, ldh, rows, ldh, 32, 32, true) ||
+      (U != nullptr && (!make_map(&em.m[1], U, ldh, rows, ldh, 32, 32, true) ||
+                        !make_map(&em.m[2], V, ldh, rows, ldh, 32, 32, true))))
+    return MOE_ERR_CUDA;
   (void)sms;
-  return cuda_status(launch_grouped_gemm(g, mA, mA, mB0, mB1, gemm_grid_of_current_device(), s));
+  return cuda_status(launch_grouped_gemm(g, mA, mA, mB0, mB1, gemm_grid_of_current_device(), s, &em));
 }
 
 // GEMM 2: H [rows, f_e] (workspace) x W2 [F, d] -> y [rows, d], gate in the epilogue
@@ -370,8 +389,12 @@ moe_status_t run_down(const moe_config_t& c, const Layout& L, void* ws, const fl
   g.out = reinterpret_cast<__nv_bfloat16*>(y);
   g.ld_out = c.d_model;
   g.out_yu = reinterpret_cast<__nv_bfloat16*>(yu);
+  EpiMaps em{};
+  if (!make_map(&em.m[0], y, d, rows, d, 32, 32, true) ||
+      (yu != nullptr && !make_map(&em.m[1], yu, d, rows, d, 32, 32, true)))
+    return MOE_ERR_CUDA;
   (void)sms;
-  return cuda_status(launch_grouped_gemm(g, mA, mA, mB, mB, gemm_grid_of_current_device(), s));
+  return cuda_status(launch_grouped_gemm(g, mA, mA, mB, mB, gemm_grid_of_current_device(), s, &em));
 }
 
 moe_status_t run_experts(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x_perm,

@@ -141,6 +141,7 @@ struct GemmArgs {
   int ld_f;
   uint32_t* err;
   ExpertTable ffn;
+  int staged;               // set by the launcher: epilogue tensor maps were given
 };
 
 struct CombineArgs {
@@ -197,11 +198,24 @@ constexpr int kBwdNormCols = 128;     // columns per bwd_norm CTA
 // Launchers (return the launch error, if any).
 cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchArgs& a, int num_sms, cudaStream_t s);
+// Tensor maps of the epilogues that move their bf16 rows through shared
+// memory by TMA (64-byte swizzle, 32 x 32 boxes over [rows, columns]):
+//   up:    m[0] = H, m[1] = U, m[2] = V (U, V when kept)   [rows, ld_out]
+//   down:  m[0] = y, m[1] = ungated y (when kept)          [rows, d]
+//   bwd_h: m[0] = U, m[1] = V (loaded), m[2] = dS, m[3] = dS3 (stored)
+//   bwd_x: m[0] = dX rows [rows, d];  wgrad_x: m[0] = dW1, m[1] = dW3 [d, F];
+//   wgrad_h: m[0] = dW2 [F, d]  (these three fp32, 128-byte swizzle)
+// Required by bwd_h; without them the other modes store row by row.
+struct EpiMaps {
+  CUtensorMap m[4];
+};
+
 // mapA1 is the second A operand (bwd_x: dS3); mapB1 the second B operand
-// (up: W3; bwd_x: W3; wgrad_x: dS3).  Unused maps may repeat another.
+// (up: W3; bwd_x: W3; wgrad_x: dS3).  Unused maps may repeat another.  `em`:
+// see EpiMaps.
 cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA0, const CUtensorMap& mapA1,
                                 const CUtensorMap& mapB0, const CUtensorMap& mapB1, int grid,
-                                cudaStream_t s);
+                                cudaStream_t s, const EpiMaps* em = nullptr);
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);
 // stats[4] = {E*sum_e f_e*P_e, CV^2(P), CV^2(counts), dropped fraction}
 cudaError_t launch_router_stats(const float* prob_mean, const int32_t* counts, const int32_t* offsets,

@@ -125,6 +125,44 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// 2-D tiled bulk tensor store from this CTA's shared memory (bulk-group
+// completion; c0 innermost, in elements, non-negative).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_addr(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// The bulk stores committed so far have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// At most `allow` (0..3) of the bulk-store groups committed so far are still
+// reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read_allow(int allow) {
+  if (allow >= 3)
+    asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory");
+  else if (allow == 2)
+    asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory");
+  else if (allow == 1)
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+  else
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// The bulk stores committed so far have completed.
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Orders this thread's generic-proxy shared-memory accesses before later
+// async-proxy (TMA) accesses of the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Same load, issued by either CTA of a 2-CTA pair: the data lands in this CTA's
 // shared memory and the byte count completes on the mbarrier at `bar_cluster`
 // (a shared::cluster address, here the pair leader's barrier).
