@@ -149,20 +149,33 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const DispatchArgs a)
     const int t = asg / a.k;
     const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d);
     uint4* dst = reinterpret_cast<uint4*>(a.x_perm + static_cast<size_t>(p) * a.d);
-    for (int c = lane; c < chunks; c += 32) {
-      const uint4 xv = __ldg(src + c);
-      const uint4 gv = __ldg(g4 + c);
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-      uint32_t o[4];
+    // four 16-byte loads per lane in flight before any store
+    for (int c0 = lane; c0 < chunks; c0 += 128) {
+      uint4 xv[4], gv[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float lo = __uint_as_float(xw[i] << 16) * __uint_as_float(gw[i] << 16);
-        const float hi = __uint_as_float(xw[i] & 0xFFFF0000u) * __uint_as_float(gw[i] & 0xFFFF0000u);
-        const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-        o[i] = *reinterpret_cast<const uint32_t*>(&h);
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < chunks) {
+          xv[u] = __ldg(src + c);
+          gv[u] = __ldg(g4 + c);
+        }
       }
-      dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 32 * u;
+        if (c >= chunks) break;
+        const uint32_t xw[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+        const uint32_t gw[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float lo = __uint_as_float(xw[i] << 16) * __uint_as_float(gw[i] << 16);
+          const float hi = __uint_as_float(xw[i] & 0xFFFF0000u) * __uint_as_float(gw[i] & 0xFFFF0000u);
+          const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+          o[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
   }
 }
