@@ -47,12 +47,16 @@
 //
 // Warp roles (192 threads per CTA): warp 0 = TMA producer, warp 1 = MMA issuer
 // (leader only) and TMEM owner, warps 2..5 = epilogue (TMEM -> registers ->
-// shared -> TMA store), one per TMEM lane quarter.  (Eight epilogue warps, two
-// per quarter on column halves, measured 5% faster on the dS GEMM and 2.5-5%
-// slower on every other mode: the extra warps share sub-partitions with the
-// producer and MMA warps.)  Ring of 6 stages x (A 16 KB + B 16 KB) per CTA;
-// two TMEM accumulators of 256 fp32 columns, so the epilogue of tile i
-// overlaps the mainloop of tile i+1.
+// shared -> TMA store), one per TMEM lane quarter.  Ring of 6 stages x (A 16
+// KB + B 16 KB) per CTA; two TMEM accumulators of 256 fp32 columns, so the
+// epilogue of tile i overlaps the mainloop of tile i+1 -- as long as it is
+// shorter.  With a reduction of at most 1024 (up: d, down: the widest
+// expert) a tile's MMAs take about as long as its epilogue, so up and down
+// then run 8 epilogue warps (320 threads), two per lane quarter on the two
+// halves of the tile's columns: measured -17 % (up, d = 1024), -27 % (up, d =
+// 768), -14 % (down, f = 512).  At d = 2048 and above the extra warps cost
+// 1-2 %, as they did (2.5-5 %) on every mode of the Mixtral shape: they share
+// sub-partitions with the producer and MMA warps.
 //
 // Epilogue output: a thread holds one accumulator row, so storing rows
 // directly makes every warp-wide store touch 32 rows in 16-byte pieces, which
@@ -80,6 +84,9 @@ constexpr int kBBytes = BK * 128 * 2;         // 16 KB: this CTA's half of BN <=
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kEpiWarps = 4;                  // one per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue
+// up and down with a short reduction may run 8 epilogue warps, two per TMEM
+// lane quarter on the two halves of the tile's columns
+__host__ __device__ constexpr int threads_of(int epi) { return 64 + 32 * epi; }
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = 256;                 // columns per accumulator buffer
 constexpr int kAtomBytes = BK * 64 * 2;       // one 64(mn) x 64(k) MN-major box: 8 KB
@@ -272,11 +279,11 @@ __device__ __forceinline__ void box_put_row_f32(uint8_t* box, int lane, const ui
 }
 
 // Staged output of a warp: `nbox` boxes per 32-column chunk in a ring of
-// 4 / nbox slots (the warp's 8 KB).  Before a slot is rewritten, lane 0 waits
-// until at most (slots - 1) of its bulk-store groups -- one per chunk -- are
-// still reading shared memory.
-__device__ __forceinline__ uint8_t* box_slot_acquire(uint8_t* boxes, int nbox, uint32_t n, int lane) {
-  const int slots = 4 / nbox;
+// bpw / nbox slots (the warp's bpw boxes).  Before a slot is rewritten, lane 0
+// waits until at most (slots - 1) of its bulk-store groups -- one per chunk --
+// are still reading shared memory.
+__device__ __forceinline__ uint8_t* box_slot_acquire(uint8_t* boxes, int nbox, uint32_t n, int lane, int bpw) {
+  const int slots = bpw / nbox;
   if (lane == 0) bulk_wait_group_read_allow(slots - 1);
   __syncwarp();
   return boxes + (n % static_cast<uint32_t>(slots)) * nbox * kEpiBoxBytes;
@@ -302,11 +309,13 @@ __device__ __forceinline__ void box_slot_store(const EpiMaps& em, uint8_t* slot,
 template <int MODE>
 __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShared& sh, const EpiMaps& em,
                                               const TileCoord& c, uint32_t taddr, int q, int lane,
-                                              uint32_t rank, uint8_t* boxes, uint32_t& n) {
+                                              uint32_t rank, uint8_t* boxes, int bpw, uint32_t& n, int c_lo,
+                                              int c_hi) {
   const int p0 = sh.seg[c.e] + c.mt * BM + static_cast<int>(rank) * BM_CTA + q * 32;
   const int p = p0 + lane;
   const bool valid = p < sh.seg[c.e + 1];
-  const bool staged = a.staged != 0 && p0 + 32 <= sh.seg[c.e + 1];
+  const int nbox_max = MODE == kGemmUp ? (a.out_u != nullptr ? 3 : 1) : (MODE == kGemmDown && a.out_yu != nullptr ? 2 : 1);
+  const bool staged = a.staged != 0 && nbox_max <= bpw && p0 + 32 <= sh.seg[c.e + 1];
   const int asg = valid ? a.perm[p] : -1;
   const bool pad = valid && asg < 0;
   const size_t prow = static_cast<size_t>(valid ? p : 0);
@@ -316,7 +325,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
     const bool keep_uv = a.out_u != nullptr;
     const int nbox = keep_uv ? 3 : 1;
 #pragma unroll 1
-    for (int cc = 0; cc < kBlockN; cc += 32) {
+    for (int cc = c_lo; cc < c_hi; cc += 32) {
       uint32_t u[32], v[32];
       tmem_ld_32x32b_x32(taddr + cc, u);
       tmem_ld_32x32b_x32(taddr + kBlockN + cc, v);
@@ -331,7 +340,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
       }
       uint8_t* slot = nullptr;
       if (staged) {
-        slot = box_slot_acquire(boxes, nbox, n++, lane);
+        slot = box_slot_acquire(boxes, nbox, n++, lane, bpw);
         box_put_row(slot, lane, o);
       } else {
         store_row_bf16(a.out + off + cc, o);
@@ -356,7 +365,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
     const bool keep_yu = a.out_yu != nullptr;
     const int nbox = keep_yu ? 2 : 1;
 #pragma unroll 1
-    for (int cc = 0; cc < a.bn; cc += 32) {
+    for (int cc = c_lo; cc < c_hi; cc += 32) {
       uint32_t u[32];
       tmem_ld_32x32b_x32(taddr + cc, u);
       tmem_ld_wait();
@@ -367,7 +376,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
         o[j] = pad ? 0u : pack_bf16(scale * __uint_as_float(u[2 * j]), scale * __uint_as_float(u[2 * j + 1]));
       uint8_t* slot = nullptr;
       if (staged) {
-        slot = box_slot_acquire(boxes, nbox, n++, lane);
+        slot = box_slot_acquire(boxes, nbox, n++, lane, bpw);
         box_put_row(slot, lane, o);
       } else {
         store_row_bf16(a.out + off + cc, o);
@@ -552,8 +561,8 @@ __device__ __forceinline__ void epilogue_wgrad(const GemmArgs& a, const GemmShar
   }
 }
 
-template <int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <int MODE, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                         const __grid_constant__ CUtensorMap mapB0, const __grid_constant__ CUtensorMap mapB1,
                         const __grid_constant__ GemmArgs a, const __grid_constant__ EpiMaps em) {
@@ -575,7 +584,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.tfull[b], 1);
-      mbar_init(&sh.tempty[b], 2 * kEpiWarps);
+      mbar_init(&sh.tempty[b], 2 * EPI);
     }
     mbar_init(&sh.drain, 1);
     for (int w = 0; w < kEpiWarps; ++w) {
@@ -729,8 +738,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_wait(&sh.drain, 0, &no_abort, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs);
     }
   } else {
-    // ================= epilogue (warps 2..5): a warp reads TMEM lane quarter warp % 4
+    // ================= epilogue (warps 2 .. 1 + EPI): a warp reads TMEM lane quarter
+    // warp % 4; with 8 warps the second four take the second half of the columns
+    static_assert(EPI == 4 || MODE == kGemmUp || MODE == kGemmDown, "8 epilogue warps: up and down only");
     const int q = warp & 3;
+    const int w = warp - 2;
+    const int bpw = kEpiBytes / EPI / kEpiBoxBytes;  // staging boxes of this warp
+    uint8_t* my_boxes = epi_boxes + w * (kEpiBytes / EPI);
+    int c_lo = 0, c_hi = MODE == kGemmUp ? kBlockN : a.bn;
+    if (EPI == 8) {
+      const int span = c_hi / 2;
+      c_lo = (w >> 2) * span;
+      c_hi = c_lo + span;
+    }
     const uint32_t tempty_leader0 = map_to_cta(smem_addr(&sh.tempty[0]), 0);
     uint32_t tcount = 0, eit = 0;
     for (int tile = pair; tile < total; tile += npairs, ++tcount) {
@@ -745,12 +765,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kAccCols;
       if (MODE == kGemmBwdH)
-        ok = epilogue_dsh(a, sh, em, c, taddr, q, lane, rank, epi_boxes + (warp - 2) * 4 * kEpiBoxBytes,
-                          sh.ebar[warp - 2], eit, abort_flag);
+        ok = epilogue_dsh(a, sh, em, c, taddr, q, lane, rank, my_boxes, sh.ebar[w], eit, abort_flag);
       else if (Traits<MODE>::row_tiles)
-        epilogue_rows<MODE>(a, sh, em, c, taddr, q, lane, rank, epi_boxes + (warp - 2) * 4 * kEpiBoxBytes, eit);
+        epilogue_rows<MODE>(a, sh, em, c, taddr, q, lane, rank, my_boxes, bpw, eit, c_lo, c_hi);
       else
-        epilogue_wgrad<MODE>(a, sh, em, c, taddr, q, lane, rank, epi_boxes + (warp - 2) * 4 * kEpiBoxBytes, eit);
+        epilogue_wgrad<MODE>(a, sh, em, c, taddr, q, lane, rank, my_boxes, eit);
       tc_fence_before();
       __syncwarp();
       if (!ok) break;
@@ -767,9 +786,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
 }
 
-template <int MODE>
+template <int MODE, int EPI = 4>
 cudaError_t set_smem_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(grouped_gemm_kernel<MODE, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(kSmemBytes));
 }
 
@@ -784,6 +803,8 @@ cudaError_t prepare_grouped_gemm() {
   if (e == cudaSuccess) e = set_smem_attr<kGemmBwdX>();
   if (e == cudaSuccess) e = set_smem_attr<kGemmWgradX>();
   if (e == cudaSuccess) e = set_smem_attr<kGemmWgradH>();
+  if (e == cudaSuccess) e = set_smem_attr<kGemmUp, 8>();
+  if (e == cudaSuccess) e = set_smem_attr<kGemmDown, 8>();
   return e;
 }
 
@@ -795,7 +816,7 @@ int grouped_gemm_max_grid(int num_sms) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<kGemmUp>, &cfg) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<kGemmUp, 4>, &cfg) != cudaSuccess ||
       clusters <= 0) {
     cudaGetLastError();
     return num_sms & ~1;
@@ -811,26 +832,33 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA0, con
   if (a.mode == kGemmBwdH && em_opt == nullptr) return cudaErrorInvalidValue;
   static const EpiMaps kNoMaps{};
   const EpiMaps& em = em_opt != nullptr ? *em_opt : kNoMaps;
+  if (a.epi8 && a.mode != kGemmUp && a.mode != kGemmDown) return cudaErrorInvalidValue;
   GemmArgs ga = a;
   ga.staged = em_opt != nullptr ? 1 : 0;
   switch (a.mode) {
     case kGemmUp:
-      grouped_gemm_kernel<kGemmUp><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+      if (ga.epi8)
+        grouped_gemm_kernel<kGemmUp, 8><<<grid, threads_of(8), kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+      else
+        grouped_gemm_kernel<kGemmUp, 4><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmDown:
-      grouped_gemm_kernel<kGemmDown><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+      if (ga.epi8)
+        grouped_gemm_kernel<kGemmDown, 8><<<grid, threads_of(8), kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+      else
+        grouped_gemm_kernel<kGemmDown, 4><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmBwdH:
-      grouped_gemm_kernel<kGemmBwdH><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+      grouped_gemm_kernel<kGemmBwdH, 4><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmBwdX:
-      grouped_gemm_kernel<kGemmBwdX><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+      grouped_gemm_kernel<kGemmBwdX, 4><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmWgradX:
-      grouped_gemm_kernel<kGemmWgradX><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+      grouped_gemm_kernel<kGemmWgradX, 4><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmWgradH:
-      grouped_gemm_kernel<kGemmWgradH><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+      grouped_gemm_kernel<kGemmWgradH, 4><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     default:
       return cudaErrorInvalidValue;

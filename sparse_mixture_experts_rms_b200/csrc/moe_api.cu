@@ -358,6 +358,9 @@ moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_
   g.ld_out = L.ldh;
   g.out_u = reinterpret_cast<__nv_bfloat16*>(U);
   g.out_v = reinterpret_cast<__nv_bfloat16*>(V);
+  // short reduction: a tile's MMAs take about as long as its epilogue, so run 8 epilogue
+  // warps (the training up keeps 4: its three output boxes per chunk need a warp's 8 KB)
+  g.epi8 = (c.d_model <= kEpi8MaxK && U == nullptr) ? 1 : 0;
   const uint64_t ldh = static_cast<uint64_t>(L.ldh);
   EpiMaps em{};
   if (!make_map(&em.m[0], g.out, ldh, rows, ldh, 32, 32, true) ||
@@ -389,6 +392,7 @@ moe_status_t run_down(const moe_config_t& c, const Layout& L, void* ws, const fl
   g.out = reinterpret_cast<__nv_bfloat16*>(y);
   g.ld_out = c.d_model;
   g.out_yu = reinterpret_cast<__nv_bfloat16*>(yu);
+  g.epi8 = L.ldh <= kEpi8MaxK ? 1 : 0;  // the down GEMM reduces over the expert width
   EpiMaps em{};
   if (!make_map(&em.m[0], y, d, rows, d, 32, 32, true) ||
       (yu != nullptr && !make_map(&em.m[1], yu, d, rows, d, 32, 32, true)))

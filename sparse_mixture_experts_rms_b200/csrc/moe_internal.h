@@ -142,6 +142,7 @@ struct GemmArgs {
   uint32_t* err;
   ExpertTable ffn;
   int staged;               // set by the launcher: epilogue tensor maps were given
+  int epi8;                 // up / down: 8 epilogue warps (short reductions)
 };
 
 struct CombineArgs {
@@ -194,6 +195,8 @@ cudaError_t launch_bwd_norm(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_reduce(const BwdArgs& a, cudaStream_t s);
 constexpr int kBwdRouteTokens = 64;   // tokens per bwd_route CTA (8 warps x 8)
 constexpr int kBwdNormCols = 128;     // columns per bwd_norm CTA
+// Up / down GEMMs whose reduction is at most this long run 8 epilogue warps.
+constexpr int kEpi8MaxK = 1024;
 
 // Launchers (return the launch error, if any).
 cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, cudaStream_t s);
