@@ -24,8 +24,9 @@
 // ldmatrix reads it conflict-free) plus the chunk's B fragments of hi/lo
 // (precomputed once per call into the workspace, in the per-lane order the
 // MMA wants, and fetched with one bulk copy).  The sum of squares for r comes
-// from the same A fragments.  Logits meet in shared memory, where one thread
-// per token does the softmax and the top-k.
+// from the same A fragments.  Logits meet in shared memory (rows padded to an
+// odd word stride, so the per-token threads read them without bank conflicts),
+// where one thread per token does the softmax and the top-k.
 #include "moe_internal.h"
 #include "ptx.cuh"
 
@@ -211,7 +212,9 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__
 
   // logits of the CTA's 64 tokens meet in shared memory (the ring is idle now)
   float* lg = reinterpret_cast<float*>(ring);
-  float* rr = lg + kTok * EP;
+  constexpr int LS = EP + 1;  // logit row stride in words: odd, so one token per bank
+  static_assert((kTok * LS + kTok) * 4 <= Cfg::kRing * Cfg::kStageBytes, "logits exceed the idle ring");
+  float* rr = lg + kTok * LS;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -220,7 +223,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__
       const int row = (i < 2) ? row_g : row_g8;
       const double rv = (i < 2) ? r_g : r_g8;
       const double b = (a.bias != nullptr && e < a.E) ? static_cast<double>(a.bias[e]) : 0.0;
-      lg[row * EP + e] = e < a.E ? static_cast<float>(fma(rv, acc[nt][i], b)) : -INFINITY;
+      lg[row * LS + e] = e < a.E ? static_cast<float>(fma(rv, acc[nt][i], b)) : -INFINITY;
     }
   }
   if (tq == 0) {
@@ -229,9 +232,9 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__
   }
   __syncthreads();
   const int t = t0 + tid;
-  if (tid < kTok && t < a.T) route_token<EP>(a, lg + tid * EP, rr[tid], t, a.prob_mean != nullptr);
+  if (tid < kTok && t < a.T) route_token<EP>(a, lg + tid * LS, rr[tid], t, a.prob_mean != nullptr);
   else if (tid < kTok && a.prob_mean != nullptr)
-    for (int e = 0; e < EP; ++e) lg[tid * EP + e] = 0.f;  // rows past T add nothing
+    for (int e = 0; e < EP; ++e) lg[tid * LS + e] = 0.f;  // rows past T add nothing
   if (a.prob_mean == nullptr) return;
 
   // Router metric in the epilogue: this CTA's probability sums, then the last
@@ -240,7 +243,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__
   __syncthreads();
   if (tid < a.E) {
     float sum = 0.f;
-    for (int i = 0; i < kTok; ++i) sum += lg[i * EP + tid];
+    for (int i = 0; i < kTok; ++i) sum += lg[i * LS + tid];
     a.prob_partial[static_cast<size_t>(blockIdx.x) * a.E + tid] = sum;
   }
   __threadfence();
