@@ -64,3 +64,19 @@ def test_reference_arm_other_ranks_exit_silently():
     r = _run_reference(1, 2)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_l2_flush_rule_follows_the_layer_footprint():
+    """Layers touching less than twice the L2 per step are timed with an L2
+    flush between steps, and their config says so; the Mixtral-shaped layer
+    (weights alone 2.8 GB) is not."""
+    import moe_workloads as mw
+    W = mw.WORKLOADS
+    # weights 3 * d * F * 2 bytes are part of the footprint
+    m = W["mixtral"]
+    assert bench.layer_footprint(m) > 3 * m.d_model * 8 * 14336 * 2
+    assert not bench.flushes_l2(m)
+    assert bench.flushes_l2(W["tiny"]) and bench.flushes_l2(W["variable_size"])
+    assert not bench.flushes_l2(W["fine_grained"])
+    assert "flushed" in bench.workload_config(W["tiny"], 1)["l2"]
+    assert "no flush" in bench.workload_config(m, 1)["l2"]
