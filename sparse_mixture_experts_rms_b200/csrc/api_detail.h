@@ -66,6 +66,7 @@ bool make_map_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t out
 bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                  uint32_t box_inner, uint32_t box_outer);
 bool make_map_sf(CUtensorMap* m, const void* base, uint64_t nblocks);
+bool make_map_sfp(CUtensorMap* m, const void* base, uint64_t nregions);
 
 // The layer's stages on one stream (cfg validated, pointers checked).
 moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf16_t* gamma,

@@ -38,7 +38,7 @@ moe_status_t run_layer_mx(const moe_config_t& c, const Layout& L, void* ws, cons
   g.err = at<uint32_t>(ws, L.err);
   for (int e = 0; e <= c.E; ++e) g.ffn.off[e] = c.ffn_offsets[e];
   const int grid = gemm_grid_of_current_device();
-  CUtensorMap mA, mB0, mB1, mSA, mSB0, mSB1;
+  CUtensorMap mA, mB0, mB1, mSA, mSB0;
   g.up = 1;
   g.bn = 256;
   g.scale = r;
@@ -47,9 +47,9 @@ moe_status_t run_layer_mx(const moe_config_t& c, const Layout& L, void* ws, cons
   if (!make_map_u8(&mA, at<void>(ws, L.x8), d, rows, d, 128, 128) || !make_map_u8(&mB0, q.w1, d, F, d, 128, 128) ||
       !make_map_u8(&mB1, q.w3, d, F, d, 128, 128) ||
       !make_map_sf(&mSA, at<void>(ws, L.xsf), (rows / 128) * (d / 128)) ||
-      !make_map_sf(&mSB0, q.sf1, (F / 128) * (d / 128)) || !make_map_sf(&mSB1, q.sf3, (F / 128) * (d / 128)))
+      !make_map_sfp(&mSB0, q.sfp13, (F / 128) * (d / 128)))
     return MOE_ERR_CUDA;
-  if ((st = cuda_status(launch_grouped_gemm_mx(g, mA, mB0, mB1, mSA, mSB0, mSB1, grid, s))) != MOE_OK) return st;
+  if ((st = cuda_status(launch_grouped_gemm_mx(g, mA, mB0, mB1, mSA, mSB0, mSB0, grid, s))) != MOE_OK) return st;
   g.up = 0;
   g.bn = (c.d_model % 256 == 0) ? 256 : 128;
   g.scale = gate;
@@ -57,7 +57,7 @@ moe_status_t run_layer_mx(const moe_config_t& c, const Layout& L, void* ws, cons
   if (!make_map_u8(&mA, at<void>(ws, L.h8), ldh, rows, ldh, 128, 128) ||
       !make_map_u8(&mB0, q.w2, F, d, F, 128, static_cast<uint32_t>(g.bn / 2)) ||
       !make_map_sf(&mSA, at<void>(ws, L.hsf), (rows / 128) * (ldh / 128)) ||
-      !make_map_sf(&mSB0, q.sf2, (d / 128) * (F / 128)))
+      !make_map_sfp(&mSB0, q.sfp2, ((d / 128 + 1) / 2) * (F / 128)))
     return MOE_ERR_CUDA;
   if ((st = cuda_status(launch_grouped_gemm_mx(g, mA, mB0, mB0, mSA, mSB0, mSB0, grid, s))) != MOE_OK) return st;
   return run_combine(c, y, inv_perm, out, sms, s);

@@ -16,9 +16,14 @@
 //         (128 when d is not a multiple of 256)
 //
 // Per pipeline stage each CTA holds 128 rows x 128 K of A (16 KB), its 128
-// rows of B (16 KB), and the scale blocks of its A rows (512 B) and of all
-// 256 B columns (two 512-B blocks, the layout tcgen05.cp takes).  The MMA
-// thread copies the scale blocks into TMEM (columns 480..491) and then issues
+// rows of B (16 KB), the scale block of its A rows (512 B, the layout
+// tcgen05.cp.32x128b.warpx4 replicates into the four TMEM lane quarters) and
+// the scales of all 256 B columns as one 4 KB paired region (both 512-B
+// blocks, each stored four times over by the weight quantiser), which a
+// single tcgen05.cp.128x256b turns into the same TMEM image: each copy
+// instruction costs the MMA thread about as much as the next, so one copy of
+// the region beats two of the blocks (measured -2.5 % up, -3 % down).  The
+// MMA thread copies the scales into TMEM (columns 480..491) and then issues
 // the stage's four K=32 MMAs, naming the scale byte of each; tcgen05
 // operations of one thread run in order, so the next stage's copy cannot
 // overtake them.  Row segments are padded to 128 rows, so a CTA's 128 rows
@@ -46,7 +51,8 @@ constexpr int kStages = 6;
 constexpr int kABytes = BM_CTA * BK;             // 16 KB
 constexpr int kBBytes = (BN / 2) * BK;           // 16 KB
 constexpr int kSfBytes = 512;                    // one scale block: 128 rows x 4 scales
-constexpr int kLoadBytes = kABytes + kBBytes + 3 * kSfBytes;   // A, B, SFA, 2 x SFB
+// stage: [B scales: one 4 KB paired region | A 16 KB | B 16 KB | A scales 512 B]
+constexpr int kLoadBytes = kMxPairRegion + kABytes + kBBytes + kSfBytes;
 constexpr int kStageBytes = (kLoadBytes + 1023) / 1024 * 1024;  // 1024-byte aligned stages
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
@@ -76,6 +82,7 @@ struct __align__(8) MxShared {
 };
 
 constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + sizeof(MxShared);
+static_assert(kSmemBytes <= 232448, "shared memory above the per-block opt-in limit");
 
 struct TileCoord {
   int e, nt, mt;
@@ -107,27 +114,26 @@ __device__ __forceinline__ void issue_loads(const MxGemmArgs& a, const CUtensorM
                                             const CUtensorMap* mSFB0, const CUtensorMap* mSFB1, const TileCoord& c,
                                             int kb, uint8_t* stage, uint32_t bar, int seg_e, int o_e,
                                             uint32_t rank, int bn) {
-  uint8_t* sA = stage;
-  uint8_t* sB = stage + kABytes;
+  uint8_t* sSFB = stage;
+  uint8_t* sA = stage + kMxPairRegion;
+  uint8_t* sB = sA + kABytes;
   uint8_t* sSFA = sB + kBBytes;
-  uint8_t* sSFB = sSFA + kSfBytes;
   const int row0 = seg_e + c.mt * BM + static_cast<int>(rank) * BM_CTA;  // a multiple of 128
   const int KA = a.up ? a.d : a.ldh;                                      // A's reduction length
   tma_load_2d_pair(sA, mA, bar, kb * BK, row0);
   tma_load_2d_pair(sSFA, mSFA, bar, 0, (row0 >> 7) * (KA >> 7) + kb);
+  // B scales: one paired region (a box of 4 rows of 1 KB)
   if (a.up) {
-    // leader: 128 columns of W1 (w1 rows), peer: the same 128 of W3
+    // leader: 128 columns of W1 (w1 rows), peer: the same 128 of W3; the region
+    // holds both blocks of scales
     const int n0 = o_e + c.nt * 128;
     tma_load_2d_pair(sB, rank == 0 ? mB0 : mB1, bar, kb * BK, n0);
-    const int blk = (n0 >> 7) * (a.d >> 7) + kb;
-    tma_load_2d_pair(sSFB, mSFB0, bar, 0, blk);              // W1 columns' scales
-    tma_load_2d_pair(sSFB + kSfBytes, mSFB1, bar, 0, blk);   // W3 columns' scales
+    tma_load_2d_pair(sSFB, mSFB0, bar, 0, 4 * ((n0 >> 7) * (a.d >> 7) + kb));
   } else {
+    // the region of column blocks (2q, 2q + 1) holding this tile's n0
     const int n0 = c.nt * bn;
     tma_load_2d_pair(sB, mB0, bar, o_e + kb * BK, n0 + static_cast<int>(rank) * (bn / 2));
-    const int kblk = (o_e >> 7) + kb;
-    tma_load_2d_pair(sSFB, mSFB0, bar, 0, (n0 >> 7) * (a.F >> 7) + kblk);
-    if (bn == 256) tma_load_2d_pair(sSFB + kSfBytes, mSFB0, bar, 0, ((n0 >> 7) + 1) * (a.F >> 7) + kblk);
+    tma_load_2d_pair(sSFB, mSFB0, bar, 0, 4 * ((n0 >> 8) * (a.F >> 7) + (o_e >> 7) + kb));
   }
 }
 
@@ -278,9 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ================= TMA producer (one lane per CTA)
     if (lane == 0) {
       const uint32_t full_leader0 = map_to_cta(smem_addr(&sh.full[0]), 0);
-      const int sfb_blocks = (a.up || a.bn == 256) ? 2 : 1;
-      const uint32_t tx_pair =
-          2u * static_cast<uint32_t>(kABytes + (a.bn / 2) * BK + kSfBytes + sfb_blocks * kSfBytes);
+      const uint32_t tx_pair = 2u * static_cast<uint32_t>(kABytes + (a.bn / 2) * BK + kSfBytes + kMxPairRegion);
       uint32_t it = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < total; tile += npairs) {
@@ -311,7 +315,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ================= MMA issuer (leader CTA, one lane)
     if (rank == 0 && lane == 0) {
       const uint32_t sfa_t = tmem_base + kSfaCol, sfb_t = tmem_base + kSfbCol;
-      const bool two_sfb = a.up || a.bn == 256;
       const uint32_t idesc_n = static_cast<uint32_t>(a.bn);
       uint32_t it = 0, tcount = 0;
       bool ok = true;
@@ -333,6 +336,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf_col(buf);
+        // a 128-column down tile of an odd column block reads the region's second half
+        const uint32_t sfb_k = sfb_t + ((!a.up && a.bn == 128 && (c.nt & 1)) ? 4u : 0u);
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1u;
@@ -341,20 +346,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t aA = smem_addr(smem + s * kStageBytes);
+          const uint32_t aSFB = smem_addr(smem + s * kStageBytes);
+          const uint32_t aA = aSFB + kMxPairRegion;
           const uint32_t aB = aA + kABytes;
-          const uint32_t aSFA = aB + kBBytes, aSFB = aSFA + kSfBytes;
-          // scale blocks: 32 lines x 16 bytes = four 8 x 16-byte core matrices, 128 bytes apart
+          const uint32_t aSFA = aB + kBBytes;
+          // A scale block: 32 lines x 16 bytes = four 8 x 16-byte core matrices, 128 bytes
+          // apart; B: the paired region, 128 rows of 2 x 16 bytes, halves 2 KB apart
           tmem_cp_pair_32x128b_warpx4(sfa_t, smem_desc_noswz(aSFA, 0, 128));
-          tmem_cp_pair_32x128b_warpx4(sfb_t, smem_desc_noswz(aSFB, 0, 128));
-          if (two_sfb) tmem_cp_pair_32x128b_warpx4(sfb_t + 4, smem_desc_noswz(aSFB + kSfBytes, 0, 128));
+          tmem_cp_pair_128x256b(sfb_t, smem_desc_noswz(aSFB, kMxPairRegion / 2, 128));
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
             const uint64_t adesc = smem_desc_sw128(aA + kk * 32, 16, 1024);
             const uint64_t bdesc = smem_desc_sw128(aB + kk * 32, 16, 1024);
             const uint32_t idesc = umma_idesc_mxf8(BM, idesc_n, kk, kk);
             umma_mxf8_pair(d_tmem, adesc, bdesc, idesc, sfa_t | (static_cast<uint32_t>(kk) << 30),
-                           sfb_t | (static_cast<uint32_t>(kk) << 30), (kb | kk) != 0 ? 1u : 0u);
+                           sfb_k | (static_cast<uint32_t>(kk) << 30), (kb | kk) != 0 ? 1u : 0u);
           }
           umma_commit_pair_mc(&sh.empty[s], 0x3);
         }

@@ -246,6 +246,18 @@ bool make_map_sf(CUtensorMap* m, const void* base, uint64_t nblocks) {
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The MX weights' paired scale regions (4 KB each) as a [4 * nregions, 256]
+// array of 32-bit words; one region (4 rows) per box.
+bool make_map_sfp(CUtensorMap* m, const void* base, uint64_t nregions) {
+  const cuuint64_t dims[2] = {256, 4 * nregions};
+  const cuuint64_t strides[1] = {1024};
+  const cuuint32_t box[2] = {256, 4};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 moe_status_t cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return MOE_OK;
   cudaGetLastError();

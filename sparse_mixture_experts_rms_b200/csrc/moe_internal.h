@@ -77,9 +77,17 @@ __host__ __device__ inline size_t mx_sf_offset(int64_t r, int64_t k, int64_t K) 
 // Quantised expert weights: K-major E4M3 copies and their scale blocks.
 //   w1, w3 [F, d]   (row n = column n of W1 / W3)      w2 [d, F] (row c = column c of W2)
 //   sf1, sf3, sf2: the standard scale blocks of those [rows, K] operands
+// sf1 / sf3 / sf2: the weights' scales in the standard blocks (mx_sf_offset).
+// sfp13 / sfp2: the same scales as the MX GEMM loads them for its B operand:
+// 4 KB regions of two 2 KB halves, each half one 512-byte block written four
+// times over, which one tcgen05.cp.128x256b copies into the TMEM image of two
+// 32x128b.warpx4 copies.  sfp13 region (nb, kb) = [W1 block | W3 block] of
+// column block nb and K block kb (index nb * d/128 + kb); sfp2 region (q, kb)
+// = [W2 column block 2q | 2q + 1] (index q * F/128 + kb).
 struct MxWeights {
-  uint8_t *w1, *w3, *w2, *sf1, *sf3, *sf2;
+  uint8_t *w1, *w3, *w2, *sf1, *sf3, *sf2, *sfp13, *sfp2;
 };
+constexpr int kMxPairRegion = 4096;
 size_t mx_weights_bytes(int d, int F);
 MxWeights mx_weights_at(void* base, int d, int F);
 cudaError_t launch_quantize_weights_mx(const __nv_bfloat16* W1, const __nv_bfloat16* W3,

@@ -274,6 +274,12 @@ __device__ __forceinline__ void umma_mxf8_pair(uint32_t d_tmem, uint64_t a_desc,
 // Pair copy shared memory -> TMEM of a 32-row x 128-bit block, replicated to
 // the four lane quarters (each CTA copies its own shared memory into its own
 // TMEM); issued by the leader CTA, ordered with its later MMAs.
+// 128 lanes x 256 bits (8 columns) from a K-major no-swizzle shared matrix:
+// lane r gets row r's two 16-byte halves (lbo bytes apart in the descriptor).
+__device__ __forceinline__ void tmem_cp_pair_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 __device__ __forceinline__ void tmem_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
