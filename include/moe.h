@@ -296,7 +296,10 @@ MOE_API moe_status_t moe_layer_fwd_host(const moe_config_t* cfg, const moe_bf16_
  * rows are padded to a multiple of 128 in the workspace. */
 
 /* Bytes of the quantised weights for cfg (0 if invalid): K-major E4M3 copies
- * of W1, W3 ([F, d]) and W2 ([d, F]) and their scale blocks. */
+ * of W1, W3 ([F, d]) and W2 ([d, F]), their scale blocks (the layout
+ * moe_mx_part describes), and the same scales once more in the form the MX
+ * GEMM loads them: each 512-byte block stored four times, two blocks per
+ * 4 KB region (about 4x the scale bytes; internal, not a part). */
 MOE_API size_t moe_mx_weights_size(const moe_config_t* cfg);
 /* Quantise W1, W3 [d, F] and W2 [F, d] (bf16, device) into wq (device,
  * 256-byte aligned, moe_mx_weights_size bytes, caller-owned). */
