@@ -220,3 +220,30 @@ def test_host_pipeline_chunking(lib):
         sub.T = T_c
         staging = 4 * T_c * c.d_model * 2
         assert moe.moe_host_workspace_size(c, n) >= moe.moe_workspace_size(sub) + staging
+
+
+@pytest.mark.parametrize("name", ["mixtral", "variable_size", "fine_grained"])
+def test_mx_weights_layout(lib, name):
+    """The MX weights buffer holds the K-major E4M3 copies, the standard scale
+    blocks (the parts moe_mx_part names, in order, none overlapping) and one
+    more copy of the scales, four times over, that the GEMM loads: at least
+    4x the scale bytes of W1 + W3 + W2 beyond the parts.  Pure host
+    arithmetic: the part pointers are offsets from a fake base."""
+    import ctypes
+    w = mw.WORKLOADS[name]
+    cfg = moe.MoEConfig(T=w.T, d_model=w.d_model, E=w.E, k=w.k,
+                        ffn_offsets=moe.ffn_offsets_from_sizes(w.expert_sizes))
+    d, F = cfg.d_model, cfg.F
+    total = moe.moe_mx_weights_size(cfg)
+    base = 1 << 40
+    out = ctypes.c_void_p()
+    sizes = {"W1": d * F, "W3": d * F, "W2": d * F, "SF1": d * F // 32, "SF3": d * F // 32, "SF2": d * F // 32}
+    end = 0
+    for part in ("W1", "W3", "W2", "SF1", "SF3", "SF2"):
+        st = lib.moe_mx_part(ctypes.byref(cfg.c()), ctypes.c_void_p(base), ctypes.c_void_p(0), ctypes.c_size_t(0),
+                             moe.MOE_MX[part], ctypes.byref(out))
+        assert st == 0
+        off = out.value - base
+        assert off >= end and off % 256 == 0, part
+        end = off + sizes[part]
+    assert total - end >= 4 * 3 * d * F // 32
