@@ -192,7 +192,10 @@ MOE_API moe_status_t moe_dispatch(const moe_config_t* cfg, const int32_t* expert
  *    return MOE_ERR_UNSUPPORTED before anything is enqueued.
  *  - The first call on a device looks up the array's device address (once per
  *    device, with that device current); make that first call before any
- *    stream capture.
+ *    stream capture.  The address is kept for the life of the process: after
+ *    cudaDeviceReset() on a device the library's module is loaded anew there
+ *    and the kept address is stale, so do not use this entry point on a
+ *    device after resetting it.
  *  - Every call on a device shares the one array, which keeps the last call's
  *    contents; the call clears what must start at zero.  Calls that overlap on
  *    the GPU (e.g. on two streams at once) race on the array: serialise them.

@@ -212,3 +212,91 @@ def check_rows(g_out: np.ndarray, ref: np.ndarray, what: str = "out"):
     assert worst <= ROW_REL, f"{what}: max row relative error {worst:.3e} > {ROW_REL}"
     assert mae <= bound, f"{what}: mean abs error {mae:.3e} > {bound:.3e}"
     return worst, mae
+
+
+# ---- gradients (training path), compared element by element
+#
+# GRAD_REL is the forward's per-row normwise bar.  Mean absolute error:
+# the forward's 1e-3 sits at 0.5-2 % of its workloads' mean output magnitude
+# (0.05-0.21); gradients have no fixed scale, so their bar is relative:
+# mean|err| <= GRAD_MEAN_REL * mean|ref| (measured normwise errors ~3.5e-3).
+# Quantities that are sums whose terms may cancel (dbias over tokens, dgamma
+# over tokens, dr and dgate over a dot product) are compared element by
+# element against GRAD_REL * (|ref| + rss), rss = the root-sum-square of the
+# sum's terms: the GPU's bf16 roundings of the terms' operands are
+# independent from term to term, so their effect on the sum grows with the
+# terms' rss, not with the (possibly cancelled) value of the sum.
+GRAD_REL = 2e-2
+GRAD_MEAN_REL = 1e-2
+
+
+def check_grad_rows(got: np.ndarray, ref: np.ndarray, what: str):
+    """Per-row normwise relative error <= GRAD_REL (rows whose reference is
+    exactly zero must be exactly zero) and mean|err| <= GRAD_MEAN_REL *
+    mean|ref|.  Returns (worst row error, relative mean absolute error)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    err = got - ref
+    nref = np.linalg.norm(ref, axis=1)
+    nerr = np.linalg.norm(err, axis=1)
+    zero = nref == 0
+    assert np.all(nerr[zero] == 0), f"{what}: rows that must be exactly zero are not"
+    rel = nerr[~zero] / nref[~zero]
+    worst = float(rel.max()) if rel.size else 0.0
+    mref = float(np.abs(ref).mean()) if ref.size else 0.0
+    mae = float(np.abs(err).mean()) if err.size else 0.0
+    rmae = mae / mref if mref > 0 else 0.0
+    assert worst <= GRAD_REL, f"{what}: row {int(np.argmax(rel))} relative error {worst:.3e} > {GRAD_REL}"
+    assert mae <= GRAD_MEAN_REL * mref, f"{what}: mean abs error {mae:.3e} > {GRAD_MEAN_REL} x {mref:.3e}"
+    return worst, rmae
+
+
+def check_sum_elems(got: np.ndarray, ref: np.ndarray, rss: np.ndarray, what: str):
+    """|got - ref| <= GRAD_REL * (|ref| + rss) element by element, for sums
+    whose terms have root-sum-square rss.  Returns the worst ratio of the
+    error to its bound."""
+    got = np.asarray(got, dtype=np.float64).reshape(-1)
+    ref = np.asarray(ref, dtype=np.float64).reshape(-1)
+    rss = np.asarray(rss, dtype=np.float64).reshape(-1)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    bound = GRAD_REL * (np.abs(ref) + rss)
+    err = np.abs(got - ref)
+    bad = np.nonzero(err > bound)[0]
+    assert bad.size == 0, (f"{what}: {bad.size} elements outside the bound, first {bad[:5]}: "
+                           f"got {got[bad[:3]]}, ref {ref[bad[:3]]}, bound {bound[bad[:3]]}")
+    nz = bound > 0
+    return float((err[nz] / bound[nz]).max()) if nz.any() else 0.0
+
+
+def grad_term_rss(f: Dict[str, object], g: np.ndarray, ref: Dict[str, np.ndarray]) -> Dict[str, np.ndarray]:
+    """Root-sum-square of the terms of the backward's reductions, from the
+    oracle's forward state ``f`` (moe_oracle_bwd.layer_forward), the upstream
+    gradient g and the oracle's gradients ``ref``:
+      dgamma_i = sum_t dxg_ti x_ti          dbias_e = sum_t dl_te
+      dgate_a  = sum_i g_ti y_ai            dr_t = sum_a <du_a, s_a> + <dv_a, s3_a> + <dl_t, z_t>
+    (du, dv from the SwiGLU backward of the kept assignment a, as the oracle
+    forms them)."""
+    from oracle import moe_oracle_bwd as B
+    g = np.asarray(g, dtype=np.float64)
+    x, r, idx, gate, kept, k = f["x"], f["r"], f["idx"], f["gate"], f["kept"], f["k"]
+    T = x.shape[0]
+    out = {"dgamma": np.sqrt(((ref["dxg"] * x) ** 2).sum(axis=0)),
+           "dbias": np.sqrt((ref["dl"] ** 2).sum(axis=0))}
+    dgate = np.zeros(T * k)
+    dr2 = (ref["dl"] * f["z"]) ** 2
+    dr2 = dr2.sum(axis=1)
+    for a in range(T * k):
+        if not kept[a]:
+            continue
+        t, j = a // k, a % k
+        e = int(idx[t, j])
+        W1e, W3e, W2e = f["slices"][e]
+        dgate[a] = np.sqrt(((g[t] * f["y"][a]) ** 2).sum())
+        dh = W2e @ (gate[t, j] * g[t])
+        du, dv = B.swiglu_backward(dh, r[t] * f["s"][a], r[t] * f["s3"][a])
+        dr2[t] += ((du * f["s"][a]) ** 2).sum() + ((dv * f["s3"][a]) ** 2).sum()
+    out["dgate"] = dgate
+    out["dr"] = np.sqrt(dr2)
+    return out
