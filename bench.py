@@ -40,13 +40,12 @@ METRIC = "MoE layer fwd tokens/s & TFLOP/s, % of B200 bf16 peak / HBM roofline"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) per launch of the up GEMM on the default
-# workload, from one ncu capture at full size (dram__bytes_read.sum +
-# dram__bytes_write.sum, a 1-pass metric; summary and command in
-# profiles/grouped_gemm_traffic_mixtral_T16384.md).  Reported only while the
-# kernel sources still hash to `digest`; after any change it is null until
-# re-measured.
+# workload, from one ncu capture of two GEMM launches at full size
+# (dram__bytes_read.sum + dram__bytes_write.sum, 1-pass metrics).  Reported
+# only while the kernel sources still hash to `digest`; after any change it
+# is null until re-measured.
 MEASURED_TRAFFIC = {"workload": "mixtral", "T": 16384, "digest": "14e7f9a5e1f6889d",
-                    "bytes": 7.055e9 + 0.928e9}   # dram read + write of the up launch (median of 12)
+                    "bytes": 7.055e9 + 0.928e9}   # dram read + write of the up launch
 
 
 def kernel_digest() -> str:
@@ -58,7 +57,11 @@ def kernel_digest() -> str:
     return h.hexdigest()[:16]
 
 
-KERNELS_PER_STEP = 8  # router weights, route, dispatch count/scatter/permute, GEMM up, GEMM down, combine
+def kernels_per_step(k: int) -> int:
+    """Launches of this library's kernels per layer step: router weights, route,
+    dispatch (count + look-back scan + scatter), permute, GEMM up, GEMM down and,
+    for k > 1, combine (k = 1: the down GEMM writes the output rows itself)."""
+    return 7 if k > 1 else 6
 
 
 def parse_args():
@@ -77,6 +80,9 @@ def parse_args():
                     help="skip the MXFP8 leg (the layer with block-scaled E4M3 expert GEMMs)")
     ap.add_argument("--no-train", action="store_true",
                     help="skip the training leg (forward with saved state + backward)")
+    ap.add_argument("--no-others", action="store_true",
+                    help="skip the other workload configurations (tiny, switch_capacity, variable_size, "
+                         "fine_grained) timed after the main line")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's token count (profiling of smaller cases)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -226,6 +232,133 @@ def replica_throughput(world: int, tokens_per_rank: int, steps: int, ms_total_ma
     return world * tokens_per_rank * steps / (ms_total_max * 1e-3)
 
 
+def layer_work(w: mw.Workload, widths, kept):
+    """Algorithmic FLOPs and bytes of one layer step from the kept rows per
+    expert: F = 2 T d E (router) + 6 d sum_e n_e f_e; B = x in + out + gamma +
+    Wr + the weights of experts that received rows + the routing metadata.
+    Returns (F, B, sum_e n_e f_e, kept rows)."""
+    d, E, T, k = w.d_model, w.E, w.T, w.k
+    kept = np.asarray(kept, dtype=np.int64)
+    nf = float(np.sum(kept * np.array(widths, dtype=np.int64)))
+    F_alg = 2.0 * T * d * E + 6.0 * d * nf
+    w_bytes = float(sum(3 * d * f * 2 for f, n in zip(widths, kept) if n > 0))
+    B_alg = 2.0 * T * d * 2 + d * 2 + d * E * 2 + w_bytes + T * k * 8 + T * 4
+    return F_alg, B_alg, nf, int(kept.sum())
+
+
+def dispatch_scale_leg(moe, steps: int = 20):
+    """The dispatch alone at its largest supported scan, 2^20 assignments
+    (T = 131072, top-8 of 64 experts, d = 128 so that the permuted copy is
+    small): moe_dispatch and moe_dispatch_noalloc, CUDA events, mean of
+    ``steps`` calls after warm-up."""
+    import torch
+    T, E, k, d = 131072, 64, 8, 128
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    idx = torch.rand((T, E), generator=g, device="cuda").topk(k, dim=1).indices.to(torch.int32).contiguous()
+    x = torch.randn((T, d), generator=g, device="cuda").to(torch.bfloat16)
+    gamma = torch.ones(d, dtype=torch.bfloat16, device="cuda")
+    cfg = moe.MoEConfig(T=T, d_model=d, E=E, k=k, ffn_offsets=[128 * i for i in range(E + 1)])
+    ws = moe.alloc_workspace(cfg)
+    o = {"counts": torch.empty(E, dtype=torch.int32, device="cuda"),
+         "offsets": torch.empty(E + 1, dtype=torch.int32, device="cuda"),
+         "perm": torch.empty(T * k, dtype=torch.int32, device="cuda"),
+         "inv_perm": torch.empty(T * k, dtype=torch.int32, device="cuda"),
+         "x_perm": torch.empty((T * k, d), dtype=torch.bfloat16, device="cuda")}
+    res = {"assignments": T * k, "E": E, "d": d}
+    for name, fn in (("moe_dispatch", lambda: moe.moe_dispatch(cfg, idx, x, gamma, o["counts"], o["offsets"],
+                                                                o["perm"], o["inv_perm"], o["x_perm"], ws)),
+                     ("moe_dispatch_noalloc", lambda: moe.moe_dispatch_noalloc(
+                         cfg, idx, x, gamma, o["counts"], o["offsets"], o["perm"], o["inv_perm"], o["x_perm"]))):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        e1.synchronize()
+        res[name + "_ms"] = e0.elapsed_time(e1) / steps
+    res["device_error"] = moe.moe_get_device_error(ws, raise_on_error=False)
+    res["counts_sum_ok"] = int(o["counts"].sum().item()) == T * k
+    del ws, o, idx, x
+    torch.cuda.empty_cache()
+    return res
+
+
+def layer_leg(moe, w: mw.Workload, steps: int, warmup: int, sampler, barrier, world: int):
+    """moe_layer_fwd on workload ``w`` alone: inputs resident in HBM, the same
+    timing rules as the main line (CUDA events on the launching stream; an L2
+    flush between steps, outside the event pairs, for layers that fit in L2).
+    Returns its step time, tokens/s and layer roofline fractions."""
+    import torch
+    widths = widths_of(w)
+    dev = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+    x, gamma, Wr = dev(mw.gen_x(w)), dev(mw.gen_gamma(w)), dev(mw.gen_router_weight(w))
+    b = mw.gen_router_bias(w)
+    bias = None if b is None else torch.from_numpy(b).cuda()
+    W1b, W3b, W2b = mw.gen_expert_weights(w, widths)
+    W1, W3, W2 = dev(W1b), dev(W3b), dev(W2b)
+    del W1b, W3b, W2b
+    cfg = moe.MoEConfig(T=w.T, d_model=w.d_model, E=w.E, k=w.k,
+                        ffn_offsets=moe.ffn_offsets_from_sizes(w.expert_sizes),
+                        capacity_factor=w.capacity_factor, eps=w.eps)
+    stream = torch.cuda.Stream()
+    ws = moe.alloc_workspace(cfg)
+    out = torch.empty((w.T, w.d_model), dtype=torch.bfloat16, device="cuda")
+    counts = torch.zeros(w.E, dtype=torch.int32, device="cuda")
+
+    def step():
+        moe.moe_layer_fwd(cfg, x, gamma, Wr, bias, W1, W3, W2, out, ws, counts=counts, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(warmup, 3)):
+            step()
+    stream.synchronize()
+    flush = flushes_l2(w)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda") if flush else None
+    barrier()
+    torch.cuda.synchronize()
+    tw0 = time.time()
+    with torch.cuda.stream(stream):
+        if flush:
+            for a_ev, b_ev in evs:
+                flush_buf.fill_(1.0)
+                a_ev.record(stream)
+                step()
+                b_ev.record(stream)
+        else:
+            evs[0][0].record(stream)
+            for _ in range(steps):
+                step()
+            evs[0][1].record(stream)
+    stream.synchronize()
+    sampler.window(tw0, time.time())
+    barrier()
+    local = (sum(a.elapsed_time(b_) for a, b_ in evs) if flush else evs[0][0].elapsed_time(evs[0][1]))
+    ms = max_over_ranks(local, world, "cuda") / steps
+    counts_h = counts.cpu().numpy().astype(np.int64)
+    C = moe.moe_capacity(cfg)
+    kept = np.minimum(counts_h, C) if C >= 0 else counts_h
+    F_alg, B_alg, nf, n_kept = layer_work(w, widths, kept)
+    peaks = load_peaks()
+    t_burst = max(F_alg / (peaks["bf16_tflops"] * 1e12), B_alg / (peaks["hbm_gbs"] * 1e9))
+    code = moe.moe_get_device_error(ws, stream=stream, raise_on_error=False)
+    res = {"workload": f"{w.name}: {w.description}", "ms_per_step": ms,
+           "tokens_per_s": world * w.T / (ms * 1e-3), "tflops": F_alg / (ms * 1e-3) / 1e12,
+           "bound": "tensor" if F_alg / (peaks["bf16_tflops"] * 1e12) >= B_alg / (peaks["hbm_gbs"] * 1e9)
+           else "hbm",
+           "t_roof_ms": t_burst * 1e3, "frac_of_burst_peak": t_burst / (ms * 1e-3),
+           "flops": F_alg, "bytes": B_alg, "kept_rows": n_kept,
+           "l2": "flushed between steps" if flush else "inputs larger than L2", "steps": steps,
+           "device_error": code}
+    del x, W1, W3, W2, ws, out, flush_buf
+    torch.cuda.empty_cache()
+    return res
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local):
     import torch
@@ -368,14 +501,9 @@ def run_ours(args, rank, world, local):
     offs_h = st["offsets"].cpu().numpy().astype(np.int64)
     kept = np.diff(offs_h)
     d, E, T, k = w.d_model, w.E, w.T, w.k
-    nf = float(np.sum(kept * np.array(widths, dtype=np.int64)))
-    fl_router = 2.0 * T * d * E
+    F_alg, B_alg, nf, n_kept = layer_work(w, widths, kept)
     fl_up = 4.0 * d * nf
     fl_down = 2.0 * d * nf
-    F_alg = fl_router + fl_up + fl_down
-    n_kept = int(kept.sum())
-    w_bytes = float(sum(3 * d * f * 2 for f, n in zip(widths, kept) if n > 0))
-    B_alg = 2.0 * T * d * 2 + d * 2 + d * E * 2 + w_bytes + T * k * 8 + T * 4
     peaks = load_peaks()
     pk_tc = peaks["bf16_tflops_sustained"] * 1e12
     pk_tc_burst = peaks["bf16_tflops"] * 1e12
@@ -444,6 +572,18 @@ def run_ours(args, rank, world, local):
         train = train_leg(moe, cfg, w, x, gamma, Wr, bias, W1, W3, W2, stream, args.steps, nf, sampler,
                           barrier, world)
 
+    # ---- the other workload configurations, each timed alone after the main line
+    others = None
+    if not args.no_others and args.tokens == 0:
+        others = {}
+        for name in mw.WORKLOAD_ORDER:
+            if name == w.name:
+                continue
+            others[name] = layer_leg(moe, mw.WORKLOADS[name], max(min(args.steps, 50), 5), args.warmup,
+                                     sampler, barrier, world)
+
+    dscale = dispatch_scale_leg(moe) if (not args.no_others and args.tokens == 0) else None
+
     clocks = sampler.stop()
     code = moe.moe_get_device_error(ws, stream=stream, raise_on_error=False)
 
@@ -471,8 +611,8 @@ def run_ours(args, rank, world, local):
         },
         "roofline": {
             "kernel": "grouped_gemm_kernel (up: x_perm x [W1|W3], SwiGLU epilogue)",
-            "bound": "tensor", "achieved": achieved_up, "peak": peaks["bf16_tflops_sustained"],
-            "unit": "TFLOP/s", "frac": achieved_up / peaks["bf16_tflops_sustained"],
+            "bound": "tensor", "achieved": achieved_up, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": achieved_up / peaks["bf16_tflops"],
             "traffic": (MEASURED_TRAFFIC["bytes"]
                         if (MEASURED_TRAFFIC["digest"] == kernel_digest()
                             and w.name == MEASURED_TRAFFIC["workload"] and w.T == MEASURED_TRAFFIC["T"])
@@ -480,14 +620,17 @@ def run_ours(args, rank, world, local):
             # W1|W3 of the experts that received rows + x_perm read + H written
             "traffic_algorithmic": (float(sum(2 * d * f * 2 for f, n in zip(widths, kept) if n > 0))
                                     + n_kept * d * 2.0 + nf * 2.0),
-            "peak_note": f"{peaks['source']} sustained cuBLAS bf16 (kernel timed inside long steps)",
+            "peak_note": f"{peaks['source']} burst cuBLAS bf16 (the up launch is timed by CUDA events around "
+                         f"the staged call, in a timed region well under a second); sustained: "
+                         f"{achieved_up / peaks['bf16_tflops_sustained']:.3f} of "
+                         f"{peaks['bf16_tflops_sustained']:.0f}",
             "flops_per_launch": fl_up,
         },
         "stages": stage_report,
         "staged_ms_per_step": staged_step_ms,
         "kept_rows": n_kept,
         "counts": counts_h.tolist(),
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": kernels_per_step(w.k) * args.steps,
         "clocks": clocks,
         "device_error": code,
     }
@@ -497,6 +640,10 @@ def run_ours(args, rank, world, local):
         result["train"] = train
     if mx is not None:
         result["mx"] = mx
+    if others is not None:
+        result["other_workloads"] = others
+    if dscale is not None:
+        result["dispatch_2e20"] = dscale
     if world > 1:
         dist.barrier()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

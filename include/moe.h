@@ -121,6 +121,19 @@ MOE_API moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream)
  * Returns MOE_ERR_DEVICE if the word was non-zero, MOE_OK otherwise. */
 MOE_API moe_status_t moe_get_device_error(void* ws, size_t ws_bytes, void* stream, uint32_t* code);
 
+/* Limit of the bounded pipeline waits of the kernels that later run on this
+ * workspace (any workspace of this library: forward, training, MXFP8 or
+ * host-buffer), written into its header in stream order.  limit_ns = 0
+ * restores the default of 4 s.  Every wait inside the router, the dispatch's
+ * scan and the expert GEMMs that does not complete within the limit sets
+ * MOE_DEVERR_TIMEOUT, stops its kernel's CTAs (both CTAs of a tensor-core
+ * pair), lets every copy and matrix operation already in flight finish, and
+ * returns; the layer's outputs
+ * are then undefined, and later calls with the default limit are unaffected.
+ * Normal use never needs this: it exists to exercise that path (a limit of a
+ * few ns makes nearly every wait run out).  moe_workspace_init resets it. */
+MOE_API moe_status_t moe_set_wait_limit(void* ws, size_t ws_bytes, uint32_t limit_ns, void* stream);
+
 /* Route: RMS statistic, router GEMM with the statistic applied after the GEMM
  * and before the top-k (CODA thread), softmax and top-k gating (MoE glossary,
  * "Top-k Gating" / "Switch Routing").
@@ -182,14 +195,15 @@ MOE_API moe_status_t moe_dispatch(const moe_config_t* cfg, const int32_t* expert
  * its input and output buffers, a runtime that forbids cudaMalloc after start-up
  * (it synchronises the device and can fail under memory pressure), or code that
  * runs inside another library's memory pool.  Such callers cannot provide the
- * workspace moe_dispatch needs for its per-tile count vectors, so this variant
- * keeps that scratch in a fixed array inside the library (a file-scope
- * __device__ array of 256 KiB + 256 B, held by every GPU that loads the
- * library until the process exits).  It allocates nothing and takes no
- * workspace; arguments and results are those of moe_dispatch.
- *  - Limit: T*k <= 1048576 assignments (the array holds the count vectors of
- *    1024 tiles of 1024 assignments for up to 64 experts); larger problems
- *    return MOE_ERR_UNSUPPORTED before anything is enqueued.
+ * workspace moe_dispatch needs for the scratch of its scan (a status word and
+ * two count vectors per tile of 1024 assignments), so this variant keeps that
+ * scratch in a fixed array inside the library (a file-scope __device__ array
+ * of 516 KiB + 256 B, held by every GPU that loads the library until the
+ * process exits).  It allocates nothing and takes no workspace; arguments and
+ * results are those of moe_dispatch.
+ *  - Limit: T*k <= 1048576 assignments (the array holds the scan of 1024
+ *    tiles of 1024 assignments for up to 64 experts); larger problems return
+ *    MOE_ERR_UNSUPPORTED before anything is enqueued.
  *  - The first call on a device looks up the array's device address (once per
  *    device, with that device current); make that first call before any
  *    stream capture.  The address is kept for the life of the process: after
@@ -201,7 +215,8 @@ MOE_API moe_status_t moe_dispatch(const moe_config_t* cfg, const int32_t* expert
  *    the GPU (e.g. on two streams at once) race on the array: serialise them.
  *  - The device error word also lives in the array and is not readable through
  *    moe_get_device_error: an expert id outside [0, E) is dropped
- *    (inv_perm = -1) and left out of counts, so sum(counts) < T*k reveals it. */
+ *    (inv_perm = -1) and left out of counts, so sum(counts) < T*k reveals it.
+ *    The scan's waits use the default limit of 4 s. */
 MOE_API moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const int32_t* expert_idx,
                                           const moe_bf16_t* x, const moe_bf16_t* gamma,
                                           int32_t* counts, int32_t* expert_offsets, int32_t* perm,

@@ -38,7 +38,7 @@ MOE_DEVERR_TIMEOUT = 0x2
 MOE_DEVERR_TILE_TABLE = 0x4
 
 EXPORTED = ["moe_status_string", "moe_capacity", "moe_max_kept", "moe_workspace_size",
-            "moe_workspace_init", "moe_get_device_error", "moe_route", "moe_dispatch",
+            "moe_workspace_init", "moe_get_device_error", "moe_set_wait_limit", "moe_route", "moe_dispatch",
             "moe_dispatch_noalloc",
             "moe_experts_fwd", "moe_experts_up", "moe_experts_down", "moe_combine",
             "moe_layer_fwd", "moe_router_stats", "moe_train_workspace_size", "moe_train_rows",
@@ -104,6 +104,8 @@ def _lib():
         lib.moe_workspace_init.argtypes = [P, SZ, P]
         lib.moe_get_device_error.restype = ctypes.c_int
         lib.moe_get_device_error.argtypes = [P, SZ, P, ctypes.POINTER(ctypes.c_uint32)]
+        lib.moe_set_wait_limit.restype = ctypes.c_int
+        lib.moe_set_wait_limit.argtypes = [P, SZ, ctypes.c_uint32, P]
         lib.moe_route.restype = ctypes.c_int
         lib.moe_route.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, SZ, P]
         lib.moe_router_stats.restype = ctypes.c_int
@@ -271,6 +273,13 @@ def moe_get_device_error(ws: torch.Tensor, stream=None, raise_on_error: bool = T
         return int(code.value)
     _check(st, "moe_get_device_error")
     return int(code.value)
+
+
+def moe_set_wait_limit(ws: torch.Tensor, limit_ns: int, stream=None) -> None:
+    """Limit (ns) of the bounded pipeline waits of the kernels that later run on
+    ``ws``; 0 restores the default (4 s).  For tests of the timeout path."""
+    _check(_lib().moe_set_wait_limit(_ptr(ws, "ws", torch.uint8), ws.numel(), int(limit_ns), _stream(stream)),
+           "moe_set_wait_limit")
 
 
 def moe_route(cfg: MoEConfig, x, gamma, Wr, bias, expert_idx, gate, r, logits,

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 
 SOURCES = ["moe_api.cu", "route.cu", "dispatch.cu", "grouped_gemm.cu", "combine.cu", "backward.cu", "quantize.cu", "grouped_gemm_mx.cu", "api_train.cu", "api_mx.cu",
            "api_host.cu"]
-HEADERS = ["moe_internal.h", "api_detail.h", "ptx.cuh", "mx.cuh"]
+HEADERS = ["moe_internal.h", "api_detail.h", "ptx.cuh", "mx.cuh", "pair_pipe.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -16,7 +16,7 @@ constexpr int kMaxDevices = 64;
 constexpr size_t kHeaderBytes = 256;  // workspace header: the device error word, the ticket
 
 struct Layout {
-  size_t err, ticket, rw, prob_partial, prob_mean, tile_counts, r, idx, gate, counts, offsets, perm,
+  size_t err, ticket, rw, prob_partial, prob_mean, scan, r, idx, gate, counts, offsets, perm,
       inv_perm, x_perm, H, y, total;
   // training workspace only
   size_t logits, U, V, yu, dY, dS, dS3, drp, dXp, dgate, rdl, dr, dbias_part, dgamma_part, dWr_part;
@@ -76,7 +76,7 @@ moe_status_t run_dispatch(const moe_config_t& c, const Layout& L, void* ws, cons
                           const moe_bf16_t* x, const moe_bf16_t* gamma, int32_t* counts,
                           int32_t* offsets, int32_t* perm, int32_t* inv_perm, moe_bf16_t* x_perm,
                           int sms, cudaStream_t s, int row_align = 1, uint8_t* x8 = nullptr,
-                          uint8_t* xsf = nullptr);
+                          uint8_t* xsf = nullptr, moe_bf16_t* zero_out = nullptr);
 void fill_gemm_common(GemmArgs& g, const moe_config_t& c, const Layout& L, void* ws,
                       const int32_t* perm, const int32_t* offsets);
 moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x_perm,
@@ -85,7 +85,8 @@ moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_
                     moe_bf16_t* U = nullptr, moe_bf16_t* V = nullptr);
 moe_status_t run_down(const moe_config_t& c, const Layout& L, void* ws, const float* gate,
                       const int32_t* perm, const int32_t* offsets, const moe_bf16_t* W2,
-                      moe_bf16_t* y, int sms, cudaStream_t s, moe_bf16_t* yu = nullptr);
+                      moe_bf16_t* y, int sms, cudaStream_t s, moe_bf16_t* yu = nullptr,
+                      bool to_token = false);
 moe_status_t run_experts(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x_perm,
                          const float* r, const float* gate, const int32_t* perm,
                          const int32_t* offsets, const moe_bf16_t* W1, const moe_bf16_t* W3,

@@ -36,6 +36,7 @@ moe_status_t run_layer_mx(const moe_config_t& c, const Layout& L, void* ws, cons
   g.offsets = offsets;
   g.perm = perm;
   g.err = at<uint32_t>(ws, L.err);
+  g.wait_ctl = at<uint32_t>(ws, kWaitCtlOffset);
   for (int e = 0; e <= c.E; ++e) g.ffn.off[e] = c.ffn_offsets[e];
   const int grid = gemm_grid_of_current_device();
   CUtensorMap mA, mB0, mB1, mSA, mSB0;

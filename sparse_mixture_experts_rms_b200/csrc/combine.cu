@@ -55,6 +55,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
 
 }  // namespace
 
+__global__ void set_words_kernel(uint32_t* dst, uint32_t w0, uint32_t w1) {
+  dst[0] = w0;
+  dst[1] = w1;
+}
+
+cudaError_t launch_set_words(uint32_t* dst, uint32_t w0, uint32_t w1, cudaStream_t s) {
+  set_words_kernel<<<1, 1, 0, s>>>(dst, w0, w1);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
   int grid = (a.T + 7) / 8;

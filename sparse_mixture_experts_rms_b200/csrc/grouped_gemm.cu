@@ -20,7 +20,8 @@
 //          acc3 = x_perm[p] . W3[:, o_e+n].  One 256 x 256 x 16 pair MMA covers 128 columns
 //          of W1 and the same 128 of W3.  Training also stores U = r*acc1, V = r*acc3.
 //   down   y[p, n] = bf16( gate[perm[p]] * (H[p, :f_e] . W2[o_e + :, n]) ); training also
-//          stores the ungated bf16(acc).
+//          stores the ungated bf16(acc).  With k = 1 the layer has nothing to sum, so
+//          the row goes straight to its token's row of the layer output (to_token).
 //   bwd_h  G = dY[p] . W2[o_e + n, :]  (dY = gate * dout of the row's token), then
 //          du = G * v * silu'(u), dv = G * silu(u) from the saved U, V, and
 //          dS = bf16(r_t du), dS3 = bf16(r_t dv), plus the dr partial sum_n (du u + dv v) / r_t
@@ -68,8 +69,12 @@
 // a ring.  The dS GEMM also loads its saved U, V chunks as boxes by TMA.  A
 // box is used when the warp's 32 rows all belong to the expert (always in the
 // 64-row-padded training layout); otherwise the threads store their rows.
-// Every wait is bounded (4 s) and sets a device error bit instead of hanging.
+// Every wait is bounded (4 s by default; the workspace header can set another
+// limit) and sets a device error bit instead of hanging; a wait that gives up
+// stops both CTAs of the pair, which still let every copy and MMA in flight
+// finish before they exit (pair_pipe.cuh).
 #include "moe_internal.h"
+#include "pair_pipe.cuh"
 #include "ptx.cuh"
 
 namespace moe {
@@ -104,6 +109,7 @@ struct __align__(8) GemmShared {
   uint64_t tempty[2];        // leader: both CTAs' epilogues drained the buffer
   uint64_t drain;
   uint64_t ebar[kEpiWarps][2];  // bwd_h: an epilogue warp's U, V box pair landed
+  PairDrain pd;                 // the producers' end-of-pipeline handshake
   uint32_t tmem_base;
   int abort_flag;
   int bad_segment;
@@ -315,7 +321,8 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
   const int p = p0 + lane;
   const bool valid = p < sh.seg[c.e + 1];
   const int nbox_max = MODE == kGemmUp ? (a.out_u != nullptr ? 3 : 1) : (MODE == kGemmDown && a.out_yu != nullptr ? 2 : 1);
-  const bool staged = a.staged != 0 && nbox_max <= bpw && p0 + 32 <= sh.seg[c.e + 1];
+  // rows sent to their tokens (down, k = 1) are not contiguous: no boxes
+  const bool staged = a.staged != 0 && a.to_token == 0 && nbox_max <= bpw && p0 + 32 <= sh.seg[c.e + 1];
   const int asg = valid ? a.perm[p] : -1;
   const bool pad = valid && asg < 0;
   const size_t prow = static_cast<size_t>(valid ? p : 0);
@@ -361,7 +368,8 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
     }
   } else if (MODE == kGemmDown) {
     const float scale = asg >= 0 ? a.scale[asg] : 0.f;
-    const size_t off = prow * a.ld_out + c.nt * a.bn;
+    const size_t orow = a.to_token ? static_cast<size_t>(asg >= 0 ? asg : 0) : prow;
+    const size_t off = orow * a.ld_out + c.nt * a.bn;
     const bool keep_yu = a.out_yu != nullptr;
     const int nbox = keep_yu ? 2 : 1;
 #pragma unroll 1
@@ -369,7 +377,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
       uint32_t u[32];
       tmem_ld_32x32b_x32(taddr + cc, u);
       tmem_ld_wait();
-      if (!valid) continue;  // never taken when staged
+      if (!valid || (a.to_token && asg < 0)) continue;  // never taken when staged
       uint32_t o[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j)
@@ -429,7 +437,8 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
 // across tiles.  Returns false when a wait gave up.
 __device__ __forceinline__ bool epilogue_dsh(const GemmArgs& a, const GemmShared& sh, const EpiMaps& em,
                                              const TileCoord& c, uint32_t taddr, int q, int lane, uint32_t rank,
-                                             uint8_t* boxes, uint64_t* bars, uint32_t& n, volatile int* abort_flag) {
+                                             uint8_t* boxes, uint64_t* bars, uint32_t& n, volatile int* abort_flag,
+                                             uint64_t wait_ns, uint32_t peer_abort) {
   const int p0 = sh.seg[c.e] + c.mt * BM + static_cast<int>(rank) * BM_CTA + q * 32;
   if (p0 >= sh.seg[c.e + 1]) return true;
   const int p = p0 + lane;
@@ -455,7 +464,7 @@ __device__ __forceinline__ bool epilogue_dsh(const GemmArgs& a, const GemmShared
     tmem_ld_32x32b_x32(taddr + cc, g);
     if (lane == 0 && cc + 32 < a.bn) load_uv(slot ^ 1u, col0 + cc + 32);
     const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars[slot], (n >> 1) & 1u, abort_flag, a.err,
-                                                     MOE_DEVERR_TIMEOUT, kWaitTimeoutNs));
+                                                     MOE_DEVERR_TIMEOUT, wait_ns, false, peer_abort));
     tmem_ld_wait();
     if (!ok) {
       if (lane == 0) {  // let the loads in flight land (bounded) before giving up
@@ -591,6 +600,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
       mbar_init(&sh.ebar[w][0], 1);
       mbar_init(&sh.ebar[w][1], 1);
     }
+    pair_drain_init(sh.pd);
     sh.abort_flag = 0;
     sh.bad_segment = 0;
     fence_mbar_init();
@@ -656,6 +666,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
   const int total = sh.total_tiles;
   volatile int* abort_flag = &sh.abort_flag;
   const Maps maps{&mapA0, &mapA1, &mapB0, &mapB1};
+  // main-loop waits: the workspace's limit; a wait that gives up also stops the other CTA
+  const uint64_t wait_ns = wait_limit_ns(a.wait_ctl);
+  const uint32_t peer_abort = map_to_cta(smem_addr(&sh.abort_flag), rank ^ 1u);
 
   if (warp == 0) {
     // ================= TMA producer (one lane per CTA)
@@ -672,7 +685,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1u;
-          if (!mbar_wait(&sh.empty[s], ph ^ 1u, abort_flag, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs)) {
+          if (!mbar_wait(&sh.empty[s], ph ^ 1u, abort_flag, a.err, MOE_DEVERR_TIMEOUT, wait_ns, false,
+                         peer_abort)) {
             ok = false;
             break;
           }
@@ -682,14 +696,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
           issue_loads<MODE>(maps, c, kb, sA, sA + kABytes, bar, sh.seg[c.e], o_e, f, rank, a.bn);
         }
       }
-      // Drain: the last stages issued are released by the MMA (normally already
-      // true), so no copy into this CTA is in flight when it exits.
-      const uint32_t n_issued = it;
-      for (uint32_t j = (n_issued > kStages ? n_issued - kStages : 0); j < n_issued; ++j) {
-        volatile int no_abort = 0;
-        mbar_wait(&sh.empty[j % kStages], (j / kStages) & 1u, &no_abort, a.err, MOE_DEVERR_TIMEOUT,
-                  kWaitTimeoutNs);
-      }
+      // no copy into either CTA is in flight when it exits, whatever stopped the loop
+      pair_producer_drain<kStages>(sh.pd, sh.full, it, rank, tx_pair / 2u, a.err);
     }
   } else if (warp == 1) {
     // ================= MMA issuer (leader CTA, one lane)
@@ -703,8 +711,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
         const uint32_t buf = tcount & 1u;
         const uint32_t aph = (tcount >> 1) & 1u;
         // both CTAs' epilogues release the buffer (the peer's arrival is remote)
-        if (!mbar_wait(&sh.tempty[buf], aph ^ 1u, abort_flag, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs,
-                       true)) {
+        if (!mbar_wait(&sh.tempty[buf], aph ^ 1u, abort_flag, a.err, MOE_DEVERR_TIMEOUT, wait_ns, true,
+                       peer_abort)) {
           ok = false;
           break;
         }
@@ -713,7 +721,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1u;
-          if (!mbar_wait(&sh.full[s], ph, abort_flag, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs)) {
+          if (!mbar_wait(&sh.full[s], ph, abort_flag, a.err, MOE_DEVERR_TIMEOUT, wait_ns, false, peer_abort)) {
             ok = false;
             break;
           }
@@ -759,13 +767,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
       const uint32_t aph = (tcount >> 1) & 1u;
       bool ok = true;
       if (lane == 0)
-        ok = mbar_wait(&sh.tfull[buf], aph, abort_flag, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs);
+        ok = mbar_wait(&sh.tfull[buf], aph, abort_flag, a.err, MOE_DEVERR_TIMEOUT, wait_ns, false, peer_abort);
       ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kAccCols;
       if (MODE == kGemmBwdH)
-        ok = epilogue_dsh(a, sh, em, c, taddr, q, lane, rank, my_boxes, sh.ebar[w], eit, abort_flag);
+        ok = epilogue_dsh(a, sh, em, c, taddr, q, lane, rank, my_boxes, sh.ebar[w], eit, abort_flag, wait_ns,
+                          peer_abort);
       else if (Traits<MODE>::row_tiles)
         epilogue_rows<MODE>(a, sh, em, c, taddr, q, lane, rank, my_boxes, bpw, eit, c_lo, c_hi);
       else

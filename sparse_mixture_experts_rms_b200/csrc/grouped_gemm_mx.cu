@@ -38,6 +38,7 @@
 // and for the full drain of the tile before it in their own buffer.
 #include "moe_internal.h"
 #include "mx.cuh"
+#include "pair_pipe.cuh"
 #include "ptx.cuh"
 
 namespace moe {
@@ -69,6 +70,7 @@ struct __align__(8) MxShared {
   uint64_t tempty[2];
   uint64_t ovl[2];           // leader: both CTAs' epilogues read the buffer's overlap columns
   uint64_t drain;
+  PairDrain pd;              // the producers' end-of-pipeline handshake
   uint32_t tmem_base;
   int abort_flag;
   int bad_segment;
@@ -229,6 +231,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&sh.ovl[b], 2 * kEpiWarps);
     }
     mbar_init(&sh.drain, 1);
+    pair_drain_init(sh.pd);
     sh.abort_flag = 0;
     sh.bad_segment = 0;
     fence_mbar_init();
@@ -279,6 +282,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = sh.tmem_base;
   const int total = sh.total_tiles;
   volatile int* abort_flag = &sh.abort_flag;
+  // main-loop waits: the workspace's limit; a wait that gives up also stops the other CTA
+  const uint64_t wait_ns = wait_limit_ns(a.wait_ctl);
+  const uint32_t peer_abort = map_to_cta(smem_addr(&sh.abort_flag), rank ^ 1u);
 
   if (warp == 0) {
     // ================= TMA producer (one lane per CTA)
@@ -294,7 +300,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1u;
-          if (!mbar_wait(&sh.empty[s], ph ^ 1u, abort_flag, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs)) {
+          if (!mbar_wait(&sh.empty[s], ph ^ 1u, abort_flag, a.err, MOE_DEVERR_TIMEOUT, wait_ns, false,
+                         peer_abort)) {
             ok = false;
             break;
           }
@@ -304,12 +311,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                       sh.seg[c.e], o_e, rank, a.bn);
         }
       }
-      const uint32_t n_issued = it;
-      for (uint32_t j = (n_issued > kStages ? n_issued - kStages : 0); j < n_issued; ++j) {
-        volatile int no_abort = 0;
-        mbar_wait(&sh.empty[j % kStages], (j / kStages) & 1u, &no_abort, a.err, MOE_DEVERR_TIMEOUT,
-                  kWaitTimeoutNs);
-      }
+      // no copy into either CTA is in flight when it exits, whatever stopped the loop
+      pair_producer_drain<kStages>(sh.pd, sh.full, it, rank, tx_pair / 2u, a.err);
     }
   } else if (warp == 1) {
     // ================= MMA issuer (leader CTA, one lane)
@@ -323,14 +326,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int kblocks = sh.k_blocks[c.e];
         const uint32_t buf = tcount & 1u;
         const uint32_t aph = (tcount >> 1) & 1u;
-        if (!mbar_wait(&sh.tempty[buf], aph ^ 1u, abort_flag, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs,
-                       true)) {
+        if (!mbar_wait(&sh.tempty[buf], aph ^ 1u, abort_flag, a.err, MOE_DEVERR_TIMEOUT, wait_ns, true,
+                       peer_abort)) {
           ok = false;
           break;
         }
         // the previous tile's epilogues have read the columns both buffers share
         if (tcount >= 1 && !mbar_wait(&sh.ovl[buf ^ 1u], ((tcount - 1) >> 1) & 1u, abort_flag, a.err,
-                                      MOE_DEVERR_TIMEOUT, kWaitTimeoutNs, true)) {
+                                      MOE_DEVERR_TIMEOUT, wait_ns, true, peer_abort)) {
           ok = false;
           break;
         }
@@ -341,7 +344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1u;
-          if (!mbar_wait(&sh.full[s], ph, abort_flag, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs)) {
+          if (!mbar_wait(&sh.full[s], ph, abort_flag, a.err, MOE_DEVERR_TIMEOUT, wait_ns, false, peer_abort)) {
             ok = false;
             break;
           }
@@ -383,7 +386,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t buf = tcount & 1u;
       const uint32_t aph = (tcount >> 1) & 1u;
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(&sh.tfull[buf], aph, abort_flag, a.err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs);
+      if (lane == 0)
+        ok = mbar_wait(&sh.tfull[buf], aph, abort_flag, a.err, MOE_DEVERR_TIMEOUT, wait_ns, false, peer_abort);
       ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       tc_fence_after();

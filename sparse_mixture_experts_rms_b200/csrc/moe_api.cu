@@ -89,7 +89,7 @@ Layout layout_of(const moe_config_t& c, bool train, bool mx) {
   L.rw = take(static_cast<size_t>(c.d_model) * kRouterPadE * 4);
   L.prob_partial = take(static_cast<size_t>((c.T + kRouteTok - 1) / kRouteTok) * c.E * 4);
   L.prob_mean = take(static_cast<size_t>(c.E) * 4);
-  L.tile_counts = take(ntiles * c.E * 4);
+  L.scan = take(dispatch_scan_ints(static_cast<int>(ntiles), c.E) * 4);
   L.r = take(static_cast<size_t>(c.T) * 4);
   L.idx = take(tk * 4);
   L.gate = take(tk * 4);
@@ -272,6 +272,7 @@ moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf1
   RouteArgs a{};
   a.wprime = at<float>(ws, L.rw);
   a.err = at<uint32_t>(ws, L.err);
+  a.wait_ctl = at<uint32_t>(ws, kWaitCtlOffset);
   a.prob_mean = prob_mean;
   a.prob_partial = at<float>(ws, L.prob_partial);
   a.ticket = at<unsigned>(ws, L.ticket);
@@ -305,14 +306,16 @@ moe_status_t run_dispatch(const moe_config_t& c, const Layout& L, void* ws, cons
                           const moe_bf16_t* x, const moe_bf16_t* gamma, int32_t* counts,
                           int32_t* offsets, int32_t* perm, int32_t* inv_perm, moe_bf16_t* x_perm,
                           int sms, cudaStream_t s, int row_align, uint8_t* x8,
-                          uint8_t* xsf) {
+                          uint8_t* xsf, moe_bf16_t* zero_out) {
   DispatchArgs a{};
+  a.zero_out = c.k == 1 ? reinterpret_cast<__nv_bfloat16*>(zero_out) : nullptr;
   a.x8 = x8;
   a.xsf = xsf;
   a.idx = idx;
   a.x = reinterpret_cast<const __nv_bfloat16*>(x);
   a.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
-  a.tile_counts = at<int32_t>(ws, L.tile_counts);
+  a.scan = at<int32_t>(ws, L.scan);
+  a.wait_ctl = at<uint32_t>(ws, kWaitCtlOffset);
   a.counts = counts;
   a.offsets = offsets;
   a.perm = perm;
@@ -345,6 +348,7 @@ void fill_gemm_common(GemmArgs& g, const moe_config_t& c, const Layout& L, void*
   g.offsets = offsets;
   g.perm = perm;
   g.err = at<uint32_t>(ws, L.err);
+  g.wait_ctl = at<uint32_t>(ws, kWaitCtlOffset);
   for (int e = 0; e <= c.E; ++e) g.ffn.off[e] = c.ffn_offsets[e];
 }
 
@@ -383,10 +387,11 @@ moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_
   return cuda_status(launch_grouped_gemm(g, mA, mA, mB0, mB1, gemm_grid_of_current_device(), s, &em));
 }
 
-// GEMM 2: H [rows, f_e] (workspace) x W2 [F, d] -> y [rows, d], gate in the epilogue
+// GEMM 2: H [rows, f_e] (workspace) x W2 [F, d] -> y [rows, d], gate in the epilogue;
+// to_token (k = 1): y is the layer output [T, d] and row p goes to row perm[p]
 moe_status_t run_down(const moe_config_t& c, const Layout& L, void* ws, const float* gate,
                       const int32_t* perm, const int32_t* offsets, const moe_bf16_t* W2,
-                      moe_bf16_t* y, int sms, cudaStream_t s, moe_bf16_t* yu) {
+                      moe_bf16_t* y, int sms, cudaStream_t s, moe_bf16_t* yu, bool to_token) {
   if (L.max_kept == 0) return MOE_OK;
   const uint64_t rows = static_cast<uint64_t>(L.max_kept);
   const uint64_t d = static_cast<uint64_t>(c.d_model);
@@ -405,11 +410,15 @@ moe_status_t run_down(const moe_config_t& c, const Layout& L, void* ws, const fl
   g.ld_out = c.d_model;
   g.out_yu = reinterpret_cast<__nv_bfloat16*>(yu);
   g.epi8 = L.ldh <= kEpi8MaxK ? 1 : 0;  // the down GEMM reduces over the expert width
+  (void)sms;
+  if (to_token && c.k == 1 && yu == nullptr) {  // scattered rows: stored row by row
+    g.to_token = 1;
+    return cuda_status(launch_grouped_gemm(g, mA, mA, mB, mB, gemm_grid_of_current_device(), s, nullptr));
+  }
   EpiMaps em{};
   if (!make_map(&em.m[0], y, d, rows, d, 32, 32, true) ||
       (yu != nullptr && !make_map(&em.m[1], yu, d, rows, d, 32, 32, true)))
     return MOE_ERR_CUDA;
-  (void)sms;
   return cuda_status(launch_grouped_gemm(g, mA, mA, mB, mB, gemm_grid_of_current_device(), s, &em));
 }
 
@@ -437,9 +446,10 @@ moe_status_t run_combine(const moe_config_t& c, const moe_bf16_t* y, const int32
 // ---- scratch of moe_dispatch_noalloc: a fixed device array instead of a workspace
 constexpr int64_t kNoallocMaxAssignments = int64_t(1) << 20;
 constexpr size_t kNoallocHeaderInts = 64;  // 256 B: the error word, then padding
-constexpr size_t kNoallocCountInts =
-    static_cast<size_t>(kNoallocMaxAssignments / kDispatchTile) * kMaxExperts;  // 256 KiB
-static __device__ __align__(256) int32_t g_noalloc_scratch[kNoallocHeaderInts + kNoallocCountInts];
+// the look-back scan of 1024 tiles of 1024 assignments, up to 64 experts: 516 KiB
+constexpr size_t kNoallocScanInts =
+    dispatch_scan_ints(static_cast<int>(kNoallocMaxAssignments / kDispatchTile), kMaxExperts);
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoallocHeaderInts + kNoallocScanInts];
 
 static int32_t* g_noalloc_ptr[kMaxDevices] = {};
 
@@ -482,11 +492,16 @@ moe_status_t run_layer(const moe_config_t& c, const Layout& L, void* ws, const m
   moe_bf16_t* y = at<moe_bf16_t>(ws, L.y);
   float* pm = prob_mean ? prob_mean : (stats ? at<float>(ws, L.prob_mean) : nullptr);
   if ((st = run_route(c, x, gamma, Wr, bias, idx_, gate_, r_, nullptr, pm, L, ws, s)) != MOE_OK) return st;
-  if ((st = run_dispatch(c, L, ws, idx_, x, gamma, counts_, offsets, perm, inv_perm, x_perm, sms, s)) != MOE_OK)
+  // k = 1: nothing to sum per token -- the dispatch zeroes the rows of dropped
+  // tokens and the down GEMM writes each kept row straight to its token's row
+  const bool direct = c.k == 1;
+  if ((st = run_dispatch(c, L, ws, idx_, x, gamma, counts_, offsets, perm, inv_perm, x_perm, sms, s, 1, nullptr,
+                         nullptr, direct ? out : nullptr)) != MOE_OK)
     return st;
-  if ((st = run_experts(c, L, ws, x_perm, r_, gate_, perm, offsets, W1, W3, W2, y, sms, s)) != MOE_OK)
+  if ((st = run_up(c, L, ws, x_perm, r_, perm, offsets, W1, W3, sms, s)) != MOE_OK) return st;
+  if ((st = run_down(c, L, ws, gate_, perm, offsets, W2, direct ? out : y, sms, s, nullptr, direct)) != MOE_OK)
     return st;
-  if ((st = run_combine(c, y, inv_perm, out, sms, s)) != MOE_OK) return st;
+  if (!direct && (st = run_combine(c, y, inv_perm, out, sms, s)) != MOE_OK) return st;
   if (stats != nullptr)
     return cuda_status(launch_router_stats(pm, counts_, offsets, stats, c.T, c.E, c.k, s));
   return MOE_OK;
@@ -536,6 +551,16 @@ moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   moe_status_t st = device_ready(&sms);
   if (st != MOE_OK) return st;
   return cuda_status(cudaMemsetAsync(ws, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_set_wait_limit(void* ws, size_t ws_bytes, uint32_t limit_ns, void* stream) {
+  if (ws == nullptr || ws_bytes < kHeaderBytes) return MOE_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGNMENT;
+  int sms;
+  moe_status_t st = device_ready(&sms);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_set_words(at<uint32_t>(ws, kWaitCtlOffset), limit_ns != 0 ? kWaitCtlTag : 0u,
+                                      limit_ns, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_get_device_error(void* ws, size_t ws_bytes, void* stream, uint32_t* code) {
@@ -631,14 +656,15 @@ moe_status_t moe_dispatch_noalloc(const moe_config_t* cfg, const int32_t* expert
     if (e == cudaSuccess) e = cudaMemsetAsync(counts, 0, cfg->E * sizeof(int32_t), s);
     return cuda_status(e);
   }
-  // the error word must start at zero; the tile counts are fully rewritten
+  // the error word must start at zero (the dispatch clears its scan's status words itself;
+  // the scan's count vectors are written before they are read)
   cudaError_t e = cudaMemsetAsync(scratch, 0, kNoallocHeaderInts * sizeof(int32_t), s);
   if (e != cudaSuccess) return cuda_status(e);
   DispatchArgs a{};
   a.idx = expert_idx;
   a.x = reinterpret_cast<const __nv_bfloat16*>(x);
   a.gamma = reinterpret_cast<const __nv_bfloat16*>(gamma);
-  a.tile_counts = scratch + kNoallocHeaderInts;
+  a.scan = scratch + kNoallocHeaderInts;
   a.counts = counts;
   a.offsets = expert_offsets;
   a.perm = perm;

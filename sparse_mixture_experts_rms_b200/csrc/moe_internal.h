@@ -16,7 +16,22 @@ constexpr int kMaxExperts = 64;
 constexpr int kRouterPadE = 64;         // w' scratch is sized for the widest router variant
 constexpr int kBlockN = 128;            // expert width granule (and G1's N per projection)
 constexpr int kDispatchTile = 1024;     // assignments per dispatch CTA
-constexpr uint64_t kWaitTimeoutNs = 4000000000ull;  // bounded pipeline waits: 4 s
+constexpr uint64_t kWaitTimeoutNs = 4000000000ull;  // bounded pipeline waits: 4 s (default)
+
+// Workspace header (256 bytes at offset 0 of every workspace): word 0 = the
+// device error word, word 1 = a CTA ticket, words 2-3 = the wait-limit
+// control: the tag kWaitCtlTag and a limit in ns for the pipeline waits of
+// the kernels that run on this workspace (moe_set_wait_limit).  Any other
+// tag, or a zero limit, means the default kWaitTimeoutNs.
+constexpr size_t kWaitCtlOffset = 8;
+constexpr uint32_t kWaitCtlTag = 0x544D494Cu;
+__device__ __forceinline__ uint64_t wait_limit_ns(const uint32_t* ctl) {
+  if (ctl != nullptr) {
+    const uint32_t tag = ctl[0], ns = ctl[1];
+    if (tag == kWaitCtlTag && ns != 0) return ns;
+  }
+  return kWaitTimeoutNs;
+}
 
 // Expert widths passed by value to the GEMM kernels (no device copy needed).
 struct ExpertTable {
@@ -33,6 +48,7 @@ struct RouteArgs {
   float* r;
   float* logits;      // may be null
   uint32_t* err;      // device error word, may be null
+  const uint32_t* wait_ctl;  // wait-limit control of the workspace header, may be null
   float* wprime;      // [d, EP] fp32 scratch: gamma * Wr, zero-padded
   float* prob_mean;     // [E] out: mean softmax probability per expert, may be null
   float* prob_partial;  // scratch [gridDim, E]: per-CTA probability sums
@@ -46,7 +62,7 @@ struct DispatchArgs {
   const int32_t* idx;       // [T*k]
   const __nv_bfloat16* x;   // [T, d]
   const __nv_bfloat16* gamma;
-  int32_t* tile_counts;     // [ntiles, E] scratch
+  int32_t* scan;            // scratch of the look-back scan (dispatch_scan_ints)
   int32_t* counts;          // [E]
   int32_t* offsets;         // [E+1]
   int32_t* perm;            // [T*k]
@@ -60,7 +76,17 @@ struct DispatchArgs {
                             // padded to that multiple (perm = -1, zero rows there)
   uint8_t* x8;              // MX mode (x_perm == null): E4M3 codes [max_kept, d]
   uint8_t* xsf;             // MX mode: E8M0 scale blocks of x8 (see mx_sf_offset)
+  __nv_bfloat16* zero_out;  // k = 1 only, may be null: rows of dropped tokens set to zero [T, d]
+  const uint32_t* wait_ctl; // wait-limit control of the workspace header, may be null
 };
+
+// Scratch of the dispatch's look-back scan over tiles of kDispatchTile
+// assignments: per tile a status word, then its aggregate and its inclusive
+// prefix as E-wide count vectors.
+__host__ __device__ constexpr int dispatch_status_ints(int ntiles) { return (ntiles + 63) / 64 * 64; }
+__host__ __device__ constexpr size_t dispatch_scan_ints(int ntiles, int E) {
+  return static_cast<size_t>(dispatch_status_ints(ntiles)) + 2 * static_cast<size_t>(ntiles) * E;
+}
 
 // ---- MXFP8 (OCP MX: 32-element blocks along K, E4M3 codes, E8M0 scales)
 //
@@ -106,6 +132,7 @@ struct MxGemmArgs {
   uint8_t* hsf;             // up: scale blocks of h8 (K = ldh)
   __nv_bfloat16* y;         // down: [rows, d]
   uint32_t* err;
+  const uint32_t* wait_ctl;  // wait-limit control of the workspace header
   ExpertTable ffn;
 };
 // up: mapSFB0 / mapSFB1 = scales of W1 / W3; down: both the scales of W2.
@@ -148,7 +175,9 @@ struct GemmArgs {
   float* out_f1;            // wgrad_x: dW3 [d, F]
   int ld_f;
   uint32_t* err;
+  const uint32_t* wait_ctl;  // wait-limit control of the workspace header
   ExpertTable ffn;
+  int to_token;             // down, k = 1: row p goes to row perm[p] (its token) of out [T, d]
   int staged;               // set by the launcher: epilogue tensor maps were given
   int epi8;                 // up / down: 8 epilogue warps (short reductions)
 };
@@ -228,6 +257,8 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA0, con
                                 const CUtensorMap& mapB0, const CUtensorMap& mapB1, int grid,
                                 cudaStream_t s, const EpiMaps* em = nullptr);
 cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s);
+// dst[0] = w0, dst[1] = w1 on the device, in stream order (one thread).
+cudaError_t launch_set_words(uint32_t* dst, uint32_t w0, uint32_t w1, cudaStream_t s);
 // stats[4] = {E*sum_e f_e*P_e, CV^2(P), CV^2(counts), dropped fraction}
 cudaError_t launch_router_stats(const float* prob_mean, const int32_t* counts, const int32_t* offsets,
                                 float* stats, int T, int E, int k, cudaStream_t s);

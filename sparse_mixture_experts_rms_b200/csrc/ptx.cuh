@@ -62,28 +62,45 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   return done != 0;
 }
 
+// Store to a 32-bit shared variable given by its shared::cluster address
+// (this CTA's or another CTA's of the cluster).
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
 // Wait for the phase of `bar` with the given parity to complete, giving up
-// after `timeout_ns` or as soon as *abort is set.  On a timeout it sets
-// *abort and ORs `err_bit` into *err.  Returns false if it gave up.
-// With `cluster` set, the wait acquires at cluster scope (for barriers that
-// receive arrivals released by another CTA of the cluster).
+// after `timeout_ns` or as soon as *abort is set.  The clock is checked on the
+// first retry and then every 64 polls, so a wait that does not complete at
+// once under a limit of a few nanoseconds gives up.  On a timeout it sets
+// *abort (and, when `peer_abort` is a shared::cluster address, the same flag
+// of the other CTA of the pair) and ORs `err_bit` into *err.  Returns false
+// if it gave up.  With `cluster` set, the wait acquires at cluster scope (for
+// barriers that receive arrivals released by another CTA of the cluster).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint32_t* err, uint32_t err_bit, uint64_t timeout_ns,
-                                          bool cluster = false) {
+                                          bool cluster = false, uint32_t peer_abort = 0) {
   auto poll = [&]() { return cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
   if (poll()) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 1;; ++n) {
     if (poll()) return true;
-    if ((n & 63u) == 0) {
+    if ((n & 63u) == 1u) {
       if (*abort) return false;
       if (global_timer_ns() - t0 > timeout_ns) {
         *abort = 1;
+        if (peer_abort != 0) st_cluster_u32(peer_abort, 1u);
         atomicOr(err, err_bit);
         return false;
       }
     }
   }
+}
+
+// Decrement the pending transaction bytes of the current phase of `bar`
+// without a copy (for bytes that were expected but will never be sent).
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
 }
 
 // ---------------------------------------------------------------- clusters

@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__
   const int t0 = blockIdx.x * kTok;
   uint32_t* err = a.err ? a.err : dummy_err;
   const int nchunks = a.d / kChunk;
+  const uint64_t wait_ns = wait_limit_ns(a.wait_ctl);  // the stage waits' limit (workspace header)
   const uint8_t* frag_src = reinterpret_cast<const uint8_t*>(a.wprime);
 
   auto issue = [&](int c, int s) {
@@ -138,10 +139,11 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__
   const int lrow = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
   const int lpiece = lane >> 4;
 
+  int stop = nchunks;  // chunks consumed
   for (int c = 0; c < nchunks; ++c) {
     const int s = c % Cfg::kRing;
     const uint32_t ph = (c / Cfg::kRing) & 1u;
-    if (ok) ok = mbar_wait(&full[s], ph, abort_flag, err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs);
+    ok = mbar_wait(&full[s], ph, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns);
     if (ok) {
       const uint8_t* st = ring + s * Cfg::kStageBytes;
       const uint2* frag = reinterpret_cast<const uint2*>(st + kTileBytes);
@@ -185,13 +187,18 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__
     }
     // every warp is done with stage s; a wait that gave up anywhere stops the CTA
     ok = __syncthreads_and(ok) != 0;
-    if (tid == 0 && ok && c + Cfg::kRing < nchunks) issue(c + Cfg::kRing, s);
+    if (!ok) {
+      stop = c;
+      break;
+    }
+    if (tid == 0 && c + Cfg::kRing < nchunks) issue(c + Cfg::kRing, s);
   }
   if (!ok) {
-    // a stage never arrived: let the copies already issued land before exiting
+    // chunks [stop, stop + ring) were issued but not consumed: let them land
+    // (default limit: issued copies always finish) before exiting
     if (tid == 0) {
       volatile int no_abort = 0;
-      for (int c = (nchunks > Cfg::kRing ? nchunks - Cfg::kRing : 0); c < nchunks; ++c)
+      for (int c = stop; c < nchunks && c < stop + Cfg::kRing; ++c)
         mbar_wait(&full[c % Cfg::kRing], (c / Cfg::kRing) & 1u, &no_abort, err, MOE_DEVERR_TIMEOUT,
                   kWaitTimeoutNs);
     }

@@ -128,6 +128,13 @@ def test_valid_call_without_device_reports_no_device(lib):
     assert _call_layer(lib, c, good, 1 << 20, wsz) == moe.MOE_ERR_NO_DEVICE
 
 
+def test_wait_limit_rejects_bad_workspace_before_device_work(lib):
+    P = ctypes.c_void_p
+    assert lib.moe_set_wait_limit(P(0), 1 << 20, 5, P(0)) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_set_wait_limit(P(1 << 20), 255, 5, P(0)) == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_set_wait_limit(P((1 << 20) + 16), 1 << 20, 5, P(0)) == moe.MOE_ERR_ALIGNMENT
+
+
 def test_status_strings(lib):
     for s in range(8):
         assert moe.moe_status_string(s).startswith("MOE_")

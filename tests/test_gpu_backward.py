@@ -2,13 +2,14 @@
 the float64 backward oracle, on the GPU's own routing (replayed into the
 oracle, whose routing parity the forward tests establish).
 
-Every gradient is compared element by element, at the forward's bar
-(``tests/_harness.py``): dx per token row; dW1, dW3 per expert column slice
-and, inside it, per row (one input feature); dW2 per expert row slice and per
-row; dWr per expert column; dgamma, dbias, dgate and dr per element, within
-2e-2 of |ref| plus the root-sum-square of the terms they sum (those sums can
-cancel).  A mistake confined to one expert's slice therefore fails even when
-the other slices are right.  The GPU path rounds x*gamma, U, V, H, gate*dout,
+Every gradient is compared piece by piece, at the forward's bar
+(``tests/_harness.py``): dx per token row; dW1, dW3, dW2 per expert slice;
+dWr, dgamma, dbias and dr per element, within 2e-2 of |ref| plus the
+root-sum-square of the terms they sum (those sums can cancel); dgate
+per assignment against the dot product of dout with the GPU's own saved
+expert output (replay), and as a vector against the oracle.  A mistake
+confined to one expert's slice therefore fails even when the other slices
+are right.  The GPU path rounds x*gamma, U, V, H, gate*dout,
 dS and dS3 to bf16 (each 2^-9 relative) and accumulates in fp32; the
 measured errors are printed.
 """
@@ -77,25 +78,29 @@ def run_case(w, renormalize=False, bias_override=None, problem=None):
     errs["dx"] = H.check_grad_rows(got["dx"], ref["dx"], "dx per token")[0]
     offs = f["offs"]
     kept_e = np.bincount(idx.reshape(-1)[f["kept"]], minlength=E)
+    slices = (("dW1", lambda o0, o1: np.s_[:, o0:o1]), ("dW3", lambda o0, o1: np.s_[:, o0:o1]),
+              ("dW2", lambda o0, o1: np.s_[o0:o1, :]))
     for e in range(E):
         o0, o1 = offs[e], offs[e + 1]
-        if kept_e[e] == 0:  # an expert with no rows gets exactly zero weight gradients
-            for name, sl in (("dW1", np.s_[:, o0:o1]), ("dW3", np.s_[:, o0:o1]), ("dW2", np.s_[o0:o1, :])):
-                assert np.count_nonzero(got[name][sl]) == 0, (name, e)
-            continue
-        for name, sl in (("dW1", np.s_[:, o0:o1]), ("dW3", np.s_[:, o0:o1]), ("dW2", np.s_[o0:o1, :])):
-            g_sl, r_sl = got[name][sl], ref[name][sl]
-            rel = _rel(g_sl, r_sl)
-            assert rel <= H.GRAD_REL, (f"{name} expert {e} slice", rel)
-            H.check_grad_rows(g_sl, r_sl, f"{name} expert {e} rows")
-            errs[f"{name}[{e}]"] = rel
-    errs["dWr"] = H.check_grad_rows(got["dWr"].T, ref["dWr"].T, "dWr per expert column")[0]
+        for name, sl in slices:
+            if kept_e[e] == 0:  # an expert with no rows gets exactly zero weight gradients
+                assert np.count_nonzero(got[name][sl(o0, o1)]) == 0, (name, e)
+            else:
+                errs[f"{name}[{e}]"] = H.check_grad_slice(got[name][sl(o0, o1)], ref[name][sl(o0, o1)],
+                                                          f"{name} expert {e} slice")
     rss = H.grad_term_rss(f, O.widen_bf16(g_bits), ref)
+    errs["dWr"] = H.check_sum_elems(got["dWr"], ref["dWr"], rss["dWr"], "dWr")
     errs["dgamma"] = H.check_sum_elems(got["dgamma"], ref["dgamma"], rss["dgamma"], "dgamma")
     errs["dbias"] = H.check_sum_elems(got["dbias"], ref["dbias"], rss["dbias"], "dbias")
     kept = f["kept"]
     dg = moe.train_saved_view(cfg, tws, "dgate").cpu().numpy().astype(np.float64)
-    errs["dgate"] = H.check_sum_elems(dg[kept], ref["dgate"].reshape(-1)[kept], rss["dgate"][kept], "dgate")
+    # dgate: per assignment against the dot product with the GPU's own saved y (replay;
+    # fp32 accumulation of d products), and as a vector against the oracle (the chain)
+    rep, rep_rss = H.dgate_replay(cfg, tws, g_bits)
+    H.check_sum_elems(dg[kept], rep.reshape(-1)[kept], rep_rss.reshape(-1)[kept], "dgate replay",
+                      rel=H.DGATE_REPLAY_REL)
+    errs["dgate"] = _rel(dg[kept], ref["dgate"].reshape(-1)[kept])
+    assert errs["dgate"] <= H.GRAD_REL, ("dgate", errs["dgate"])
     dr = moe.train_saved_view(cfg, tws, "dr").cpu().numpy().astype(np.float64)
     errs["dr"] = H.check_sum_elems(dr, ref["dr"], rss["dr"], "dr")
     worst_slice = max((v for k_, v in errs.items() if "[" in k_), default=0.0)
