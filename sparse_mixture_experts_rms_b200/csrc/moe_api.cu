@@ -86,7 +86,7 @@ Layout layout_of(const moe_config_t& c, bool train, bool mx) {
   const size_t mk = static_cast<size_t>(L.max_kept);
   L.err = 0;
   L.ticket = 4;  // second word of the header
-  L.rw = take(static_cast<size_t>(c.d_model) * kRouterPadE * 4);
+  L.rw = take(static_cast<size_t>(c.d_model) * 2 * kRouterPadE * 2);  // router hi/lo B [2 EP, d] bf16
   L.prob_partial = take(static_cast<size_t>((c.T + kRouteTok - 1) / kRouteTok) * c.E * 4);
   L.prob_mean = take(static_cast<size_t>(c.E) * 4);
   L.scan = take(dispatch_scan_ints(static_cast<int>(ntiles), c.E) * 4);
@@ -270,7 +270,7 @@ moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf1
                        float* logits, float* prob_mean, const Layout& L, void* ws, cudaStream_t s) {
   if (c.T == 0) return MOE_OK;
   RouteArgs a{};
-  a.wprime = at<float>(ws, L.rw);
+  a.wprime = at<__nv_bfloat16>(ws, L.rw);
   a.err = at<uint32_t>(ws, L.err);
   a.wait_ctl = at<uint32_t>(ws, kWaitCtlOffset);
   a.prob_mean = prob_mean;
@@ -294,12 +294,14 @@ moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf1
   a.k = c.k;
   a.eps = c.eps;
   a.renormalize = c.renormalize ? 1 : 0;
-  CUtensorMap xmap;
-  // x [T, d]: tiles of 64 tokens x 64 elements
+  CUtensorMap xmap, wmap;
+  // x [T, d]: tiles of 128 tokens x 64 elements; the router's hi/lo B [2 EP, d]: 2 EP x 64
+  const uint32_t ep2 = static_cast<uint32_t>(2 * route_padded_experts(c.E));
   if (!make_map(&xmap, x, static_cast<uint64_t>(c.d_model), static_cast<uint64_t>(c.T),
-                static_cast<uint64_t>(c.d_model), 64, 64))
+                static_cast<uint64_t>(c.d_model), 64, kRouteTok) ||
+      !make_map(&wmap, a.wprime, static_cast<uint64_t>(c.d_model), ep2, static_cast<uint64_t>(c.d_model), 64, ep2))
     return MOE_ERR_CUDA;
-  return cuda_status(launch_route(a, xmap, s));
+  return cuda_status(launch_route(a, xmap, wmap, s));
 }
 
 moe_status_t run_dispatch(const moe_config_t& c, const Layout& L, void* ws, const int32_t* idx,

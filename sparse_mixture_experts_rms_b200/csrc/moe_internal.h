@@ -49,7 +49,7 @@ struct RouteArgs {
   float* logits;      // may be null
   uint32_t* err;      // device error word, may be null
   const uint32_t* wait_ctl;  // wait-limit control of the workspace header, may be null
-  float* wprime;      // [d, EP] fp32 scratch: gamma * Wr, zero-padded
+  __nv_bfloat16* wprime;  // [2 EP, d] scratch: (gamma * Wr)^T split into bf16 hi rows, then lo rows
   float* prob_mean;     // [E] out: mean softmax probability per expert, may be null
   float* prob_partial;  // scratch [gridDim, E]: per-CTA probability sums
   unsigned* ticket;     // scratch: CTAs done (zeroed before the launch)
@@ -236,7 +236,10 @@ constexpr int kBwdNormCols = 128;     // columns per bwd_norm CTA
 constexpr int kEpi8MaxK = 1024;
 
 // Launchers (return the launch error, if any).
-cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, cudaStream_t s);
+// xmap: x [T, d], boxes of 64 x 128 tokens; wmap: the [2 EP, d] hi/lo scratch,
+// boxes of 64 x 2 EP (both 128-byte swizzled).
+cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, const CUtensorMap& wmap, cudaStream_t s);
+int route_padded_experts(int E);  // EP: E rounded up to 8, 16, 32 or 64
 cudaError_t launch_dispatch(const DispatchArgs& a, int num_sms, cudaStream_t s);
 // Tensor maps of the epilogues that move their bf16 rows through shared
 // memory by TMA (64-byte swizzle, 32 x 32 boxes over [rows, columns]):
@@ -262,7 +265,7 @@ cudaError_t launch_set_words(uint32_t* dst, uint32_t w0, uint32_t w1, cudaStream
 // stats[4] = {E*sum_e f_e*P_e, CV^2(P), CV^2(counts), dropped fraction}
 cudaError_t launch_router_stats(const float* prob_mean, const int32_t* counts, const int32_t* offsets,
                                 float* stats, int T, int E, int k, cudaStream_t s);
-constexpr int kRouteTok = 64;  // tokens per router CTA
+constexpr int kRouteTok = 128;  // tokens per router CTA
 
 // One-time per-device kernel attributes (dynamic shared memory opt-in).
 cudaError_t prepare_grouped_gemm();

@@ -8,44 +8,62 @@
 // largest router scores pick the experts; their softmax probabilities weight
 // the expert outputs.
 //
-// The contraction runs on the tensor cores (warp-level mma.sync m16n8k16,
-// bf16 in, fp32 out) without losing the exactness routing needs:
+// The contraction runs on the 5th-generation tensor cores (tcgen05.mma,
+// cta_group::1, M = 128 tokens, N = 2 EP, bf16 in, fp32 in TMEM) without
+// losing the exactness routing needs:
 //  - w' (two bf16 multiplied: 16 significant bits) is split exactly into
 //    w' = hi + lo with hi, lo bf16 (8 bits each), so x*w' = x*hi + x*lo and
-//    every product the tensor core forms is exact;
-//  - each 64-element chunk is accumulated by the MMAs from zero (4 k-steps),
-//    and the chunk partials are summed in fp64; r and l = r*acc + b are
-//    formed in fp64 and each logit is rounded once to fp32.
+//    every product the tensor core forms is exact; B = [hi | lo] holds the
+//    two halves as 2 EP columns (EP = E rounded up to 8, 16, 32 or 64);
+//  - each 64-element chunk of d is accumulated by 4 MMAs from zero into its
+//    own TMEM buffer (a ring of four), and the epilogue adds every chunk's hi
+//    and lo partials into fp64 registers; r and l = r*acc + b are formed in
+//    fp64 and each logit is rounded once to fp32.
 // A near-tie between the k-th and (k+1)-th logit can therefore only flip when
 // the two fp32 logits differ by about one ulp.
 //
-// Layout: a CTA (4 warps) owns 64 tokens, a warp 16.  x streams through a ring
-// of stages, each a TMA tile [64 tokens x 64 elements] (128-byte swizzle;
-// ldmatrix reads it conflict-free) plus the chunk's B fragments of hi/lo
-// (precomputed once per call into the workspace, in the per-lane order the
-// MMA wants, and fetched with one bulk copy).  The sum of squares for r comes
-// from the same A fragments.  Logits meet in shared memory (rows padded to an
-// odd word stride, so the per-token threads read them without bank conflicts),
-// where one thread per token does the softmax and the top-k.
+// Layout: a CTA owns 128 tokens.  Warp 0 streams x through a ring of stages
+// by TMA, each [128 tokens x 64 elements] (128-byte swizzle) plus the chunk's
+// B tile [2 EP x 64] of hi/lo (precomputed once per call into the workspace,
+// K-major); warp 1 issues the MMAs; warps 2-5 (one per TMEM lane quarter, a
+// thread per token) read each chunk's partials from TMEM, add the sum of
+// squares of their token's 64 elements from the staged x tile (for r), and
+// release the stage.  After the last chunk each thread has its token's fp64
+// logit sums and sum of squares; logits meet in shared memory (rows padded to
+// an odd word stride, so per-token threads read them without bank conflicts),
+// where each thread does its token's softmax and top-k.
 #include "moe_internal.h"
 #include "ptx.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kTok = kRouteTok;                // tokens per CTA
-constexpr int kWarps = kTok / 16;              // a warp owns 16 tokens (MMA rows)
-constexpr int kThreads = kWarps * 32;
-constexpr int kChunk = 64;                     // elements of d per stage (4 k-steps)
-constexpr int kTileBytes = kTok * kChunk * 2;  // 8 KB of x per stage
+constexpr int kTok = kRouteTok;                // tokens per CTA (the MMA's M)
+constexpr int kThreads = 192;                  // producer, MMA, four epilogue warps
+constexpr int kChunk = 64;                     // elements of d per stage (4 MMAs of K = 16)
+constexpr int kTileBytes = kTok * kChunk * 2;  // 16 KB of x per stage
+constexpr int kStages = 6;
+constexpr int kBufs = 4;                       // TMEM chunk-partial buffers
 
 template <int EP>
 struct RouteCfg {
-  static constexpr int NT = EP / 8;                            // MMA n-tiles
-  static constexpr int kFragBytes = 4 * NT * 2 * 32 * 8;       // k-steps x tiles x {hi,lo} x lanes x 8 B
-  static constexpr int kStageBytes = kTileBytes + kFragBytes;  // a multiple of 1024
-  static constexpr int kRing = EP <= 16 ? 6 : (EP == 32 ? 5 : 4);
-  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kRing) * kStageBytes + 64;
+  static constexpr int N = 2 * EP;                             // MMA N: hi and lo columns
+  static constexpr int kBBytes = N * kChunk * 2;               // B tile: a multiple of 1024
+  static constexpr int kStageBytes = kTileBytes + kBBytes;
+  static constexpr uint32_t kTmemCols = kBufs * N < 32 ? 32u : static_cast<uint32_t>(kBufs * N);
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * kStageBytes + 256;
+};
+
+struct __align__(8) RouteShared {
+  uint64_t full[kStages];    // the stage's x and B tiles landed
+  uint64_t empty[kStages];   // the MMAs and the epilogue's sums of squares are done with the stage
+  uint64_t tfull[kBufs];     // a chunk's partials are in the TMEM buffer
+  uint64_t tempty[kBufs];    // the epilogue read the buffer
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  uint32_t dummy_err;
+  int is_last;
 };
 
 __device__ __forceinline__ uint32_t bf16_bits_rn(float v) {
@@ -53,37 +71,67 @@ __device__ __forceinline__ uint32_t bf16_bits_rn(float v) {
   return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&h));
 }
 
-// B fragments of hi(w') and lo(w') for every (k-step, n-tile, lane):
-// b0 = {w'[k0][n], w'[k0+1][n]}, b1 = {w'[k0+8][n], w'[k0+9][n]},
-// k0 = 16*ks + 2*(lane%4), n = 8*nt + lane/4 (zero for n >= E).
-__global__ void router_weight_kernel(const RouteArgs a, int nt_count) {
-  const int ksteps = a.d / 16;
-  const int n = ksteps * nt_count * 2 * 32;
+// B = (gamma * Wr)^T split exactly into bf16 hi (rows [0, EP)) and lo (rows
+// [EP, 2 EP)), K-major [2 EP, d]; experts n >= E are zero rows.
+__global__ void router_weight_kernel(const RouteArgs a, int ep) {
+  const int n = 2 * ep * a.d;
   const uint16_t* gam = reinterpret_cast<const uint16_t*>(a.gamma);
   const uint16_t* wr = reinterpret_cast<const uint16_t*>(a.Wr);
-  uint2* out = reinterpret_cast<uint2*>(a.wprime);
+  uint16_t* out = reinterpret_cast<uint16_t*>(a.wprime);
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
-    const int lane = i % 32;
-    const int hl = (i / 32) % 2;
-    const int nt = (i / 64) % nt_count;
-    const int ks = i / (64 * nt_count);
-    const int col = nt * 8 + lane / 4;
-    const int k0 = ks * 16 + 2 * (lane % 4);
-    uint32_t h16[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int kk = k0 + (j & 1) + (j >> 1) * 8;
-      float w = 0.f;
-      if (col < a.E) {
-        const float g = __uint_as_float(static_cast<uint32_t>(gam[kk]) << 16);
-        const float v = __uint_as_float(static_cast<uint32_t>(wr[static_cast<size_t>(kk) * a.E + col]) << 16);
-        w = g * v;  // exact
-      }
-      const uint32_t hi = bf16_bits_rn(w);
-      const float hif = __uint_as_float(hi << 16);
-      h16[j] = hl == 0 ? hi : bf16_bits_rn(w - hif);  // w - hi is exact and fits in bf16
+    const int row = i / a.d, kk = i - row * a.d;
+    const int col = row < ep ? row : row - ep;
+    float w = 0.f;
+    if (col < a.E) {
+      const float g = __uint_as_float(static_cast<uint32_t>(gam[kk]) << 16);
+      const float v = __uint_as_float(static_cast<uint32_t>(wr[static_cast<size_t>(kk) * a.E + col]) << 16);
+      w = g * v;  // exact
     }
-    out[i] = make_uint2(h16[0] | (h16[1] << 16), h16[2] | (h16[3] << 16));
+    const uint32_t hi = bf16_bits_rn(w);
+    out[i] = static_cast<uint16_t>(row < ep ? hi : bf16_bits_rn(w - __uint_as_float(hi << 16)));  // w - hi is exact
+  }
+}
+
+// 32 lanes x 16 consecutive 32-bit TMEM columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+
+// acc[e] += hi_e + lo_e (fp64) for the chunk partials in TMEM columns
+// [col, col + 2 EP) of this warp's lane quarter: hi in [col, col + EP), lo in
+// [col + EP, col + 2 EP).  Every load stays inside those 2 EP columns.
+template <int EP>
+__device__ __forceinline__ void add_chunk(uint32_t taddr, double (&acc)[EP]) {
+  if constexpr (EP == 8) {
+    uint32_t v[16];
+    tmem_ld_32x32b_x16(taddr, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      acc[e] += static_cast<double>(__uint_as_float(v[e])) + static_cast<double>(__uint_as_float(v[8 + e]));
+  } else if constexpr (EP == 16) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(taddr, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      acc[e] += static_cast<double>(__uint_as_float(v[e])) + static_cast<double>(__uint_as_float(v[16 + e]));
+  } else {  // EP = 32 or 64: 16-column loads of hi and of lo (few registers beside acc)
+#pragma unroll
+    for (int h = 0; h < EP / 16; ++h) {
+      uint32_t hv[16], lv[16];
+      tmem_ld_32x32b_x16(taddr + 16 * h, hv);
+      tmem_ld_32x32b_x16(taddr + EP + 16 * h, lv);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        acc[16 * h + e] += static_cast<double>(__uint_as_float(hv[e])) + static_cast<double>(__uint_as_float(lv[e]));
+    }
   }
 }
 
@@ -92,161 +140,161 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, float* lg, float
                                             bool keep_probs);
 
 template <int EP>
-__global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__ CUtensorMap xmap,
-                                                         const RouteArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) route_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                            const __grid_constant__ CUtensorMap wmap,
+                                                            const RouteArgs a) {
   using Cfg = RouteCfg<EP>;
-  constexpr int NT = Cfg::NT;
+  constexpr int N = Cfg::N;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + Cfg::kRing * Cfg::kStageBytes);
-  int* abort_flag = reinterpret_cast<int*>(full + Cfg::kRing);
-  uint32_t* dummy_err = reinterpret_cast<uint32_t*>(abort_flag + 1);
+  RouteShared& sh = *reinterpret_cast<RouteShared*>(ring + kStages * Cfg::kStageBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t0 = blockIdx.x * kTok;
-  uint32_t* err = a.err ? a.err : dummy_err;
   const int nchunks = a.d / kChunk;
-  const uint64_t wait_ns = wait_limit_ns(a.wait_ctl);  // the stage waits' limit (workspace header)
-  const uint8_t* frag_src = reinterpret_cast<const uint8_t*>(a.wprime);
-
-  auto issue = [&](int c, int s) {
-    uint8_t* st = ring + s * Cfg::kStageBytes;
-    mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
-    tma_load_2d(st, &xmap, &full[s], c * kChunk, t0);
-    bulk_load(st + kTileBytes, frag_src + static_cast<size_t>(c) * Cfg::kFragBytes, Cfg::kFragBytes, &full[s]);
-  };
+  const uint64_t wait_ns = wait_limit_ns(a.wait_ctl);  // the pipeline waits' limit (workspace header)
 
   if (tid == 0) {
-    for (int s = 0; s < Cfg::kRing; ++s) mbar_init(&full[s], 1);
-    *abort_flag = 0;
-    *dummy_err = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.empty[s], 1 + 4);  // MMA commit + the four epilogue warps
+    }
+    for (int b = 0; b < kBufs; ++b) {
+      mbar_init(&sh.tfull[b], 1);
+      mbar_init(&sh.tempty[b], 4);
+    }
+    mbar_init(&sh.drain, 1);
+    sh.abort_flag = 0;
+    sh.dummy_err = 0;
     fence_mbar_init();
     tma_prefetch_map(&xmap);
+    tma_prefetch_map(&wmap);
   }
+  if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
-  if (tid == 0)
-    for (int c = 0; c < Cfg::kRing && c < nchunks; ++c) issue(c, c);
+  tc_fence_after();
+  uint32_t* err = a.err ? a.err : &sh.dummy_err;
+  volatile int* abort_flag = &sh.abort_flag;
+  const uint32_t tmem_base = sh.tmem_base;
 
-  // accumulators: this lane's C elements (rows g, g+8; columns 2t, 2t+1 of each n-tile)
-  double acc[NT][4];
+  double acc[EP];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0;
-  double ss_g = 0.0, ss_g8 = 0.0;
+  for (int e = 0; e < EP; ++e) acc[e] = 0.0;
+  double ss = 0.0;
   bool ok = true;
 
-  // ldmatrix row address of this lane: matrix m = lane/8 -> rows +8*(m&1), k piece +(m>>1)
-  const int lrow = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-  const int lpiece = lane >> 4;
-
-  int stop = nchunks;  // chunks consumed
-  for (int c = 0; c < nchunks; ++c) {
-    const int s = c % Cfg::kRing;
-    const uint32_t ph = (c / Cfg::kRing) & 1u;
-    ok = mbar_wait(&full[s], ph, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns);
-    if (ok) {
-      const uint8_t* st = ring + s * Cfg::kStageBytes;
-      const uint2* frag = reinterpret_cast<const uint2*>(st + kTileBytes);
-      const uint32_t tile = smem_addr(st);
-      float chi[NT][4], clo[NT][4];
+  if (warp == 0) {
+    // ================= TMA producer
+    if (lane == 0) {
+      int c = 0;
+      for (; c < nchunks; ++c) {
+        const int s = c % kStages;
+        if (!mbar_wait(&sh.empty[s], ((c / kStages) & 1u) ^ 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns)) break;
+        uint8_t* st = ring + s * Cfg::kStageBytes;
+        mbar_arrive_expect_tx(&sh.full[s], Cfg::kStageBytes);
+        tma_load_2d(st, &xmap, &sh.full[s], c * kChunk, t0);
+        tma_load_2d(st + kTileBytes, &wmap, &sh.full[s], c * kChunk, 0);
+      }
+      // the copies still in flight land before the CTA goes on (default limit)
+      volatile int no_abort = 0;
+      for (int j = c > kStages ? c - kStages : 0; j < c; ++j)
+        mbar_wait(&sh.full[j % kStages], (j / kStages) & 1u, &no_abort, err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs);
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(kTok, N, 0u, 0u);  // A and B K-major
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c % kStages, b = c % kBufs;
+        if (!mbar_wait(&sh.full[s], (c / kStages) & 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns) ||
+            !mbar_wait(&sh.tempty[b], ((c / kBufs) & 1u) ^ 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns))
+          break;
+        tc_fence_after();
+        const uint32_t aA = smem_addr(ring + s * Cfg::kStageBytes);
+        const uint32_t aB = aA + kTileBytes;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+        for (int kk = 0; kk < kChunk / 16; ++kk)
+          umma_bf16(tmem_base + b * N, smem_desc_sw128(aA + kk * 32, 16, 1024),
+                    smem_desc_sw128(aB + kk * 32, 16, 1024), idesc, kk != 0 ? 1u : 0u);
+        umma_commit(&sh.empty[s]);
+        umma_commit(&sh.tfull[b]);
+      }
+      umma_commit(&sh.drain);
+      volatile int no_abort = 0;
+      mbar_wait(&sh.drain, 0, &no_abort, err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs);
+    }
+  } else {
+    // ================= epilogue: thread = token row (TMEM lane q*32 + lane)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c % kStages, b = c % kBufs;
+      ok = mbar_wait(&sh.full[s], (c / kStages) & 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) break;
+      // sum of squares of this token's 64 elements (128-byte swizzled row)
+      const uint8_t* xr = ring + s * Cfg::kStageBytes + row * 128;
+      float sq = 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) chi[nt][i] = clo[nt][i] = 0.f;
-      float sg = 0.f, sg8 = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const int piece = 2 * kk + lpiece;
-        uint32_t av[4];
-        ldmatrix_x4(tile + lrow * 128 + ((piece ^ (lrow & 7)) << 4), av);
+      for (int j = 0; j < 8; ++j) {
+        const uint4 v = *reinterpret_cast<const uint4*>(xr + ((j ^ (row & 7)) << 4));
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float lo = __uint_as_float(av[i] << 16), hi = __uint_as_float(av[i] & 0xFFFF0000u);
-          if (i & 1) {
-            sg8 = fmaf(lo, lo, sg8);
-            sg8 = fmaf(hi, hi, sg8);
-          } else {
-            sg = fmaf(lo, lo, sg);
-            sg = fmaf(hi, hi, sg);
-          }
-        }
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const uint2 bh = frag[((kk * NT + nt) * 2 + 0) * 32 + lane];
-          const uint2 bl = frag[((kk * NT + nt) * 2 + 1) * 32 + lane];
-          mma_bf16_16816(chi[nt], av, bh.x, bh.y);
-          mma_bf16_16816(clo[nt], av, bl.x, bl.y);
+          const float lo = __uint_as_float(w4[i] << 16), hi = __uint_as_float(w4[i] & 0xFFFF0000u);
+          sq = fmaf(lo, lo, sq);
+          sq = fmaf(hi, hi, sq);
         }
       }
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nt][i] += static_cast<double>(chi[nt][i]) + static_cast<double>(clo[nt][i]);
-      ss_g += static_cast<double>(sg);
-      ss_g8 += static_cast<double>(sg8);
+      ss += static_cast<double>(sq);
+      ok = mbar_wait(&sh.tfull[b], (c / kBufs) & 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      add_chunk<EP>(tq + b * N, acc);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&sh.tempty[b]);
+        mbar_arrive(&sh.empty[s]);
+      }
     }
-    // every warp is done with stage s; a wait that gave up anywhere stops the CTA
-    ok = __syncthreads_and(ok) != 0;
-    if (!ok) {
-      stop = c;
-      break;
-    }
-    if (tid == 0 && c + Cfg::kRing < nchunks) issue(c + Cfg::kRing, s);
   }
-  if (!ok) {
-    // chunks [stop, stop + ring) were issued but not consumed: let them land
-    // (default limit: issued copies always finish) before exiting
-    if (tid == 0) {
-      volatile int no_abort = 0;
-      for (int c = stop; c < nchunks && c < stop + Cfg::kRing; ++c)
-        mbar_wait(&full[c % Cfg::kRing], (c / Cfg::kRing) & 1u, &no_abort, err, MOE_DEVERR_TIMEOUT,
-                  kWaitTimeoutNs);
-    }
-    return;
+  ok = __syncthreads_and(ok && !*abort_flag) != 0;
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
   }
+  if (!ok) return;  // a wait gave up: the error word says so, outputs are undefined
 
-  // sum of squares of rows g and g+8 over the quad's columns
-#pragma unroll
-  for (int m = 1; m <= 2; m <<= 1) {
-    ss_g += __shfl_xor_sync(0xFFFFFFFFu, ss_g, m);
-    ss_g8 += __shfl_xor_sync(0xFFFFFFFFu, ss_g8, m);
-  }
-  const int g = lane >> 2, tq = lane & 3;
-  const int row_g = warp * 16 + g, row_g8 = row_g + 8;
-  const double inv_d = 1.0 / static_cast<double>(a.d);
-  const double r_g = 1.0 / sqrt(ss_g * inv_d + static_cast<double>(a.eps));
-  const double r_g8 = 1.0 / sqrt(ss_g8 * inv_d + static_cast<double>(a.eps));
-
-  // logits of the CTA's 64 tokens meet in shared memory (the ring is idle now)
+  // logits of the CTA's tokens meet in shared memory (the ring is idle now)
   float* lg = reinterpret_cast<float*>(ring);
   constexpr int LS = EP + 1;  // logit row stride in words: odd, so one token per bank
-  static_assert((kTok * LS + kTok) * 4 <= Cfg::kRing * Cfg::kStageBytes, "logits exceed the idle ring");
+  static_assert((kTok * LS + kTok) * 4 <= kStages * Cfg::kStageBytes, "logits exceed the idle ring");
   float* rr = lg + kTok * LS;
+  const bool keep_probs = a.prob_mean != nullptr;
+  if (warp >= 2) {
+    const int row = (warp & 3) * 32 + lane;
+    const double rv = 1.0 / sqrt(ss / static_cast<double>(a.d) + static_cast<double>(a.eps));
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = nt * 8 + 2 * tq + (i & 1);
-      const int row = (i < 2) ? row_g : row_g8;
-      const double rv = (i < 2) ? r_g : r_g8;
-      const double b = (a.bias != nullptr && e < a.E) ? static_cast<double>(a.bias[e]) : 0.0;
-      lg[row * LS + e] = e < a.E ? static_cast<float>(fma(rv, acc[nt][i], b)) : -INFINITY;
+    for (int e = 0; e < EP; ++e) {
+      const double bb = (a.bias != nullptr && e < a.E) ? static_cast<double>(a.bias[e]) : 0.0;
+      lg[row * LS + e] = e < a.E ? static_cast<float>(fma(rv, acc[e], bb)) : -INFINITY;
     }
+    rr[row] = static_cast<float>(rv);
+    const int t = t0 + row;
+    if (t < a.T) route_token<EP>(a, lg + row * LS, rr[row], t, keep_probs);
+    else if (keep_probs)
+      for (int e = 0; e < EP; ++e) lg[row * LS + e] = 0.f;  // rows past T add nothing
   }
-  if (tq == 0) {
-    rr[row_g] = static_cast<float>(r_g);
-    rr[row_g8] = static_cast<float>(r_g8);
-  }
-  __syncthreads();
-  const int t = t0 + tid;
-  if (tid < kTok && t < a.T) route_token<EP>(a, lg + tid * LS, rr[tid], t, a.prob_mean != nullptr);
-  else if (tid < kTok && a.prob_mean != nullptr)
-    for (int e = 0; e < EP; ++e) lg[tid * LS + e] = 0.f;  // rows past T add nothing
-  if (a.prob_mean == nullptr) return;
+  if (!keep_probs) return;
 
   // Router metric in the epilogue: this CTA's probability sums, then the last
   // CTA to finish sums every CTA's partials in CTA order (deterministic).
-  __shared__ int is_last;
   __syncthreads();
   if (tid < a.E) {
     float sum = 0.f;
@@ -255,9 +303,9 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const __grid_constant__
   }
   __threadfence();
   __syncthreads();
-  if (tid == 0) is_last = atomicAdd(a.ticket, 1u) == gridDim.x - 1;
+  if (tid == 0) sh.is_last = atomicAdd(a.ticket, 1u) == gridDim.x - 1;
   __syncthreads();
-  if (!is_last) return;
+  if (!sh.is_last) return;
   __threadfence();
   if (tid < a.E) {
     double sum = 0.0;
@@ -324,7 +372,7 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, float* lg, float
 }
 
 template <int EP>
-cudaError_t launch_route_t(const RouteArgs& a, const CUtensorMap& xmap, cudaStream_t s) {
+cudaError_t launch_route_t(const RouteArgs& a, const CUtensorMap& xmap, const CUtensorMap& wmap, cudaStream_t s) {
   const size_t smem = RouteCfg<EP>::kSmem;
   static bool attr_done[64] = {};
   int dev = 0;
@@ -335,10 +383,10 @@ cudaError_t launch_route_t(const RouteArgs& a, const CUtensorMap& xmap, cudaStre
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
-  const int n = (a.d / 16) * RouteCfg<EP>::NT * 64;
-  router_weight_kernel<<<(n + 255) / 256, 256, 0, s>>>(a, RouteCfg<EP>::NT);
+  const int n = 2 * EP * a.d;
+  router_weight_kernel<<<(n + 255) / 256, 256, 0, s>>>(a, EP);
   const int grid = (a.T + kTok - 1) / kTok;
-  route_kernel<EP><<<grid, kThreads, smem, s>>>(xmap, a);
+  route_kernel<EP><<<grid, kThreads, smem, s>>>(xmap, wmap, a);
   return cudaGetLastError();
 }
 
@@ -385,12 +433,16 @@ cudaError_t launch_router_stats(const float* prob_mean, const int32_t* counts, c
   return cudaGetLastError();
 }
 
-cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, cudaStream_t s) {
+int route_padded_experts(int E) { return E <= 8 ? 8 : (E <= 16 ? 16 : (E <= 32 ? 32 : 64)); }
+
+cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, const CUtensorMap& wmap, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
-  if (a.E <= 8) return launch_route_t<8>(a, xmap, s);
-  if (a.E <= 16) return launch_route_t<16>(a, xmap, s);
-  if (a.E <= 32) return launch_route_t<32>(a, xmap, s);
-  return launch_route_t<64>(a, xmap, s);
+  switch (route_padded_experts(a.E)) {
+    case 8: return launch_route_t<8>(a, xmap, wmap, s);
+    case 16: return launch_route_t<16>(a, xmap, wmap, s);
+    case 32: return launch_route_t<32>(a, xmap, wmap, s);
+    default: return launch_route_t<64>(a, xmap, wmap, s);
+  }
 }
 
 }  // namespace moe
