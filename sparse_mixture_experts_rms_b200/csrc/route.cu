@@ -39,26 +39,36 @@ namespace moe {
 namespace {
 
 constexpr int kTok = kRouteTok;                // tokens per CTA (the MMA's M)
-constexpr int kThreads = 192;                  // producer, MMA, four epilogue warps
-constexpr int kChunk = 64;                     // elements of d per stage (4 MMAs of K = 16)
-constexpr int kTileBytes = kTok * kChunk * 2;  // 16 KB of x per stage
-constexpr int kStages = 6;
-constexpr int kBufs = 4;                       // TMEM chunk-partial buffers
+constexpr int kChunk = 64;                     // elements of d per fp32 partial (4 MMAs of K = 16)
+constexpr int kTileBytes = kTok * kChunk * 2;  // 16 KB of x per chunk
+constexpr int kGroups = 2;                     // TMEM buffer groups (one stage's chunks each)
+constexpr int kMaxStages = 8;
 
 template <int EP>
 struct RouteCfg {
   static constexpr int N = 2 * EP;                             // MMA N: hi and lo columns
-  static constexpr int kBBytes = N * kChunk * 2;               // B tile: a multiple of 1024
-  static constexpr int kStageBytes = kTileBytes + kBBytes;
-  static constexpr uint32_t kTmemCols = kBufs * N < 32 ? 32u : static_cast<uint32_t>(kBufs * N);
-  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * kStageBytes + 256;
+  // epilogue warps: one per TMEM lane quarter, or two (each on half of the
+  // experts and half of the row's sum of squares) when the fp64 chunk sums of
+  // 32 or 64 experts would bound the kernel
+  static constexpr int kEpi = EP >= 32 ? 8 : 4;
+  static constexpr int kEP = EP / (kEpi / 4);                  // experts per epilogue thread
+  static constexpr int kThreads = 64 + 32 * kEpi;
+  static constexpr int kBBytes = N * kChunk * 2;               // B tile of a chunk: a multiple of 1024
+  // A stage carries several chunks (their x tiles side by side along d, so a
+  // row's 256-512 contiguous bytes are fetched together, and one MMA commit /
+  // epilogue hand-off per stage); each chunk still gets its own TMEM buffer.
+  static constexpr int kCps = EP <= 8 ? 4 : 2;                 // chunks per stage
+  static constexpr int kStageBytes = kCps * (kTileBytes + kBBytes);
+  static constexpr int kStages = (220 * 1024) / kStageBytes < kMaxStages ? (220 * 1024) / kStageBytes : kMaxStages;
+  static constexpr uint32_t kTmemCols = kGroups * kCps * N < 32 ? 32u : static_cast<uint32_t>(kGroups * kCps * N);
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * kStageBytes + 512;
 };
 
 struct __align__(8) RouteShared {
-  uint64_t full[kStages];    // the stage's x and B tiles landed
-  uint64_t empty[kStages];   // the MMAs and the epilogue's sums of squares are done with the stage
-  uint64_t tfull[kBufs];     // a chunk's partials are in the TMEM buffer
-  uint64_t tempty[kBufs];    // the epilogue read the buffer
+  uint64_t full[kMaxStages];   // the stage's x and B tiles landed
+  uint64_t empty[kMaxStages];  // the MMAs and the epilogue's sums of squares are done with the stage
+  uint64_t tfull[kGroups];     // a stage's chunk partials are in the TMEM buffer group
+  uint64_t tempty[kGroups];    // the epilogue read the group
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -102,37 +112,33 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)
       : "r"(taddr));
 }
 
-// acc[e] += hi_e + lo_e (fp64) for the chunk partials in TMEM columns
-// [col, col + 2 EP) of this warp's lane quarter: hi in [col, col + EP), lo in
-// [col + EP, col + 2 EP).  Every load stays inside those 2 EP columns.
-template <int EP>
-__device__ __forceinline__ void add_chunk(uint32_t taddr, double (&acc)[EP]) {
-  if constexpr (EP == 8) {
-    uint32_t v[16];
-    tmem_ld_32x32b_x16(taddr, v);
-    tmem_ld_wait();
+// 32 lanes x 8 consecutive 32-bit TMEM columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&v)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(taddr));
+}
+
+template <int NC>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[NC]) {
+  if constexpr (NC == 8) tmem_ld_32x32b_x8(taddr, v);
+  else if constexpr (NC == 16) tmem_ld_32x32b_x16(taddr, v);
+  else tmem_ld_32x32b_x32(taddr, v);
+}
+
+// acc[e] += hi_e + lo_e (fp64) for NE experts whose chunk partials sit in
+// TMEM columns [thi, thi + NE) (hi) and [tlo, tlo + NE) (lo) of this warp's
+// lane quarter.
+template <int NE>
+__device__ __forceinline__ void add_chunk(uint32_t thi, uint32_t tlo, double (&acc)[NE]) {
+  static_assert(NE == 8 || NE == 16 || NE == 32, "8, 16 or 32 experts per epilogue thread");
+  uint32_t h[NE], l[NE];
+  tmem_ld_cols<NE>(thi, h);
+  tmem_ld_cols<NE>(tlo, l);
+  tmem_ld_wait();
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      acc[e] += static_cast<double>(__uint_as_float(v[e])) + static_cast<double>(__uint_as_float(v[8 + e]));
-  } else if constexpr (EP == 16) {
-    uint32_t v[32];
-    tmem_ld_32x32b_x32(taddr, v);
-    tmem_ld_wait();
-#pragma unroll
-    for (int e = 0; e < 16; ++e)
-      acc[e] += static_cast<double>(__uint_as_float(v[e])) + static_cast<double>(__uint_as_float(v[16 + e]));
-  } else {  // EP = 32 or 64: 16-column loads of hi and of lo (few registers beside acc)
-#pragma unroll
-    for (int h = 0; h < EP / 16; ++h) {
-      uint32_t hv[16], lv[16];
-      tmem_ld_32x32b_x16(taddr + 16 * h, hv);
-      tmem_ld_32x32b_x16(taddr + EP + 16 * h, lv);
-      tmem_ld_wait();
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        acc[16 * h + e] += static_cast<double>(__uint_as_float(hv[e])) + static_cast<double>(__uint_as_float(lv[e]));
-    }
-  }
+  for (int e = 0; e < NE; ++e)
+    acc[e] += static_cast<double>(__uint_as_float(h[e])) + static_cast<double>(__uint_as_float(l[e]));
 }
 
 template <int EP>
@@ -140,27 +146,31 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, float* lg, float
                                             bool keep_probs);
 
 template <int EP>
-__global__ void __launch_bounds__(kThreads, 1) route_kernel(const __grid_constant__ CUtensorMap xmap,
-                                                            const __grid_constant__ CUtensorMap wmap,
-                                                            const RouteArgs a) {
+__global__ void __launch_bounds__(RouteCfg<EP>::kThreads, 1)
+    route_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap,
+                 const RouteArgs a) {
   using Cfg = RouteCfg<EP>;
   constexpr int N = Cfg::N;
+  constexpr int EPI = Cfg::kEpi;
+  constexpr int NE = Cfg::kEP;          // experts per epilogue thread
+  constexpr int NJ = 8 / (EPI / 4);     // 16-byte pieces of a row's 64 elements per thread
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  RouteShared& sh = *reinterpret_cast<RouteShared*>(ring + kStages * Cfg::kStageBytes);
+  RouteShared& sh = *reinterpret_cast<RouteShared*>(ring + Cfg::kStages * Cfg::kStageBytes);
+  static_assert(Cfg::kStages >= 2 && Cfg::kStages <= kMaxStages, "stage count");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t0 = blockIdx.x * kTok;
   const int nchunks = a.d / kChunk;
   const uint64_t wait_ns = wait_limit_ns(a.wait_ctl);  // the pipeline waits' limit (workspace header)
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < Cfg::kStages; ++s) {
       mbar_init(&sh.full[s], 1);
-      mbar_init(&sh.empty[s], 1 + 4);  // MMA commit + the four epilogue warps
+      mbar_init(&sh.empty[s], 1 + EPI);  // MMA commit + the epilogue warps
     }
-    for (int b = 0; b < kBufs; ++b) {
-      mbar_init(&sh.tfull[b], 1);
-      mbar_init(&sh.tempty[b], 4);
+    for (int g = 0; g < kGroups; ++g) {
+      mbar_init(&sh.tfull[g], 1);
+      mbar_init(&sh.tempty[g], EPI);
     }
     mbar_init(&sh.drain, 1);
     sh.abort_flag = 0;
@@ -180,88 +190,115 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(const __grid_constan
   volatile int* abort_flag = &sh.abort_flag;
   const uint32_t tmem_base = sh.tmem_base;
 
-  double acc[EP];
+  double acc[NE];
 #pragma unroll
-  for (int e = 0; e < EP; ++e) acc[e] = 0.0;
+  for (int e = 0; e < NE; ++e) acc[e] = 0.0;
   double ss = 0.0;
   bool ok = true;
+  const int q = warp & 3;                     // TMEM lane quarter of an epilogue warp
+  const int half = warp >= 2 ? (warp - 2) / 4 : 0;  // which half of the experts (8 epilogue warps)
+  const int row = q * 32 + lane;              // token row of an epilogue thread
 
+  constexpr int S = Cfg::kStages, CPS = Cfg::kCps;
+  const int nst = (nchunks + CPS - 1) / CPS;  // stages; the last one may hold fewer chunks
+  auto chunks_of = [&](int st) { return nchunks - st * CPS < CPS ? nchunks - st * CPS : CPS; };
   if (warp == 0) {
     // ================= TMA producer
     if (lane == 0) {
-      int c = 0;
-      for (; c < nchunks; ++c) {
-        const int s = c % kStages;
-        if (!mbar_wait(&sh.empty[s], ((c / kStages) & 1u) ^ 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns)) break;
-        uint8_t* st = ring + s * Cfg::kStageBytes;
-        mbar_arrive_expect_tx(&sh.full[s], Cfg::kStageBytes);
-        tma_load_2d(st, &xmap, &sh.full[s], c * kChunk, t0);
-        tma_load_2d(st + kTileBytes, &wmap, &sh.full[s], c * kChunk, 0);
+      int st = 0;
+      for (; st < nst; ++st) {
+        const int s = st % S, nc = chunks_of(st);
+        if (!mbar_wait(&sh.empty[s], ((st / S) & 1u) ^ 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns)) break;
+        uint8_t* xs = ring + s * Cfg::kStageBytes;
+        uint8_t* bs = xs + CPS * kTileBytes;
+        mbar_arrive_expect_tx(&sh.full[s], static_cast<uint32_t>(nc * (kTileBytes + Cfg::kBBytes)));
+        for (int i = 0; i < nc; ++i) {
+          const int kx = (st * CPS + i) * kChunk;
+          tma_load_2d(xs + i * kTileBytes, &xmap, &sh.full[s], kx, t0);
+          tma_load_2d(bs + i * Cfg::kBBytes, &wmap, &sh.full[s], kx, 0);
+        }
       }
       // the copies still in flight land before the CTA goes on (default limit)
       volatile int no_abort = 0;
-      for (int j = c > kStages ? c - kStages : 0; j < c; ++j)
-        mbar_wait(&sh.full[j % kStages], (j / kStages) & 1u, &no_abort, err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs);
+      for (int j = st > S ? st - S : 0; j < st; ++j)
+        mbar_wait(&sh.full[j % S], (j / S) & 1u, &no_abort, err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs);
     }
   } else if (warp == 1) {
-    // ================= MMA issuer
+    // ================= MMA issuer: chunk i of a stage goes to TMEM buffer g*CPS + i
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_bf16(kTok, N, 0u, 0u);  // A and B K-major
-      for (int c = 0; c < nchunks; ++c) {
-        const int s = c % kStages, b = c % kBufs;
-        if (!mbar_wait(&sh.full[s], (c / kStages) & 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns) ||
-            !mbar_wait(&sh.tempty[b], ((c / kBufs) & 1u) ^ 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns))
+      for (int st = 0; st < nst; ++st) {
+        const int s = st % S, g = st % kGroups, nc = chunks_of(st);
+        if (!mbar_wait(&sh.full[s], (st / S) & 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns) ||
+            !mbar_wait(&sh.tempty[g], ((st / kGroups) & 1u) ^ 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns))
           break;
         tc_fence_after();
-        const uint32_t aA = smem_addr(ring + s * Cfg::kStageBytes);
-        const uint32_t aB = aA + kTileBytes;
+        const uint32_t aX = smem_addr(ring + s * Cfg::kStageBytes);
+        const uint32_t aB = aX + CPS * kTileBytes;
+        for (int i = 0; i < nc; ++i) {
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>((g * CPS + i) * N);
 #pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk)
-          umma_bf16(tmem_base + b * N, smem_desc_sw128(aA + kk * 32, 16, 1024),
-                    smem_desc_sw128(aB + kk * 32, 16, 1024), idesc, kk != 0 ? 1u : 0u);
+          for (int kk = 0; kk < kChunk / 16; ++kk)
+            umma_bf16(d_tmem, smem_desc_sw128(aX + i * kTileBytes + kk * 32, 16, 1024),
+                      smem_desc_sw128(aB + i * Cfg::kBBytes + kk * 32, 16, 1024), idesc, kk != 0 ? 1u : 0u);
+        }
         umma_commit(&sh.empty[s]);
-        umma_commit(&sh.tfull[b]);
+        umma_commit(&sh.tfull[g]);
       }
       umma_commit(&sh.drain);
       volatile int no_abort = 0;
       mbar_wait(&sh.drain, 0, &no_abort, err, MOE_DEVERR_TIMEOUT, kWaitTimeoutNs);
     }
   } else {
-    // ================= epilogue: thread = token row (TMEM lane q*32 + lane)
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    for (int c = 0; c < nchunks; ++c) {
-      const int s = c % kStages, b = c % kBufs;
-      ok = mbar_wait(&sh.full[s], (c / kStages) & 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns);
+    // ================= epilogue: thread = token row (TMEM lane q*32 + lane);
+    // experts [half*NE, half*NE + NE) and pieces [half*NJ, half*NJ + NJ) of each chunk's row
+    const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + half * NE;
+    for (int st = 0; st < nst; ++st) {
+      const int s = st % S, g = st % kGroups, nc = chunks_of(st);
+      ok = mbar_wait(&sh.full[s], (st / S) & 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) break;
-      // sum of squares of this token's 64 elements (128-byte swizzled row)
-      const uint8_t* xr = ring + s * Cfg::kStageBytes + row * 128;
-      float sq = 0.f;
+      // sum of squares of this thread's pieces of its token's elements
+      // (128-byte swizzled rows), one independent accumulator per piece
+      float sq[CPS * NJ];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint4 v = *reinterpret_cast<const uint4*>(xr + ((j ^ (row & 7)) << 4));
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      for (int i = 0; i < CPS; ++i) {
+        const uint8_t* xr = ring + s * Cfg::kStageBytes + i * kTileBytes + row * 128;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float lo = __uint_as_float(w4[i] << 16), hi = __uint_as_float(w4[i] & 0xFFFF0000u);
-          sq = fmaf(lo, lo, sq);
-          sq = fmaf(hi, hi, sq);
+        for (int j = 0; j < NJ; ++j) {
+          float acc_j = 0.f;
+          if (i < nc) {
+            const int jj = half * NJ + j;
+            const uint4 v = *reinterpret_cast<const uint4*>(xr + ((jj ^ (row & 7)) << 4));
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float lo = __uint_as_float(w4[u] << 16), hi = __uint_as_float(w4[u] & 0xFFFF0000u);
+              acc_j = fmaf(lo, lo, acc_j);
+              acc_j = fmaf(hi, hi, acc_j);
+            }
+          }
+          sq[i * NJ + j] = acc_j;
         }
       }
-      ss += static_cast<double>(sq);
-      ok = mbar_wait(&sh.tfull[b], (c / kBufs) & 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns);
+      ok = mbar_wait(&sh.tfull[g], (st / kGroups) & 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) break;
       tc_fence_after();
-      add_chunk<EP>(tq + b * N, acc);
+      for (int i = 0; i < nc; ++i) {
+        const uint32_t tb = tq + static_cast<uint32_t>((g * CPS + i) * N);
+        add_chunk<NE>(tb, tb + EP, acc);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&sh.tempty[b]);
+        mbar_arrive(&sh.tempty[g]);
         mbar_arrive(&sh.empty[s]);
       }
+      float sqs = 0.f;
+#pragma unroll
+      for (int j = 0; j < CPS * NJ; ++j) sqs += sq[j];
+      ss += static_cast<double>(sqs);
     }
   }
   ok = __syncthreads_and(ok && !*abort_flag) != 0;
@@ -274,20 +311,27 @@ __global__ void __launch_bounds__(kThreads, 1) route_kernel(const __grid_constan
   // logits of the CTA's tokens meet in shared memory (the ring is idle now)
   float* lg = reinterpret_cast<float*>(ring);
   constexpr int LS = EP + 1;  // logit row stride in words: odd, so one token per bank
-  static_assert((kTok * LS + kTok) * 4 <= kStages * Cfg::kStageBytes, "logits exceed the idle ring");
-  float* rr = lg + kTok * LS;
+  static_assert((kTok * LS + 1 + 4 * kTok) * 4 <= Cfg::kStages * Cfg::kStageBytes, "logits exceed the idle ring");
+  double* ssp = reinterpret_cast<double*>(lg + kTok * LS + (kTok * LS) % 2);  // [2][kTok] partial sums of squares
   const bool keep_probs = a.prob_mean != nullptr;
+  if (warp >= 2) ssp[half * kTok + row] = ss;
+  __syncthreads();
   if (warp >= 2) {
-    const int row = (warp & 3) * 32 + lane;
-    const double rv = 1.0 / sqrt(ss / static_cast<double>(a.d) + static_cast<double>(a.eps));
+    const double sst = EPI == 8 ? ssp[row] + ssp[kTok + row] : ssp[row];
+    const double rv = 1.0 / sqrt(sst / static_cast<double>(a.d) + static_cast<double>(a.eps));
 #pragma unroll
-    for (int e = 0; e < EP; ++e) {
-      const double bb = (a.bias != nullptr && e < a.E) ? static_cast<double>(a.bias[e]) : 0.0;
-      lg[row * LS + e] = e < a.E ? static_cast<float>(fma(rv, acc[e], bb)) : -INFINITY;
+    for (int e = 0; e < NE; ++e) {
+      const int ex = half * NE + e;
+      const double bb = (a.bias != nullptr && ex < a.E) ? static_cast<double>(a.bias[ex]) : 0.0;
+      lg[row * LS + ex] = ex < a.E ? static_cast<float>(fma(rv, acc[e], bb)) : -INFINITY;
     }
-    rr[row] = static_cast<float>(rv);
+  }
+  __syncthreads();
+  if (warp >= 2 && half == 0) {
+    const double sst = EPI == 8 ? ssp[row] + ssp[kTok + row] : ssp[row];
+    const float rv = static_cast<float>(1.0 / sqrt(sst / static_cast<double>(a.d) + static_cast<double>(a.eps)));
     const int t = t0 + row;
-    if (t < a.T) route_token<EP>(a, lg + row * LS, rr[row], t, keep_probs);
+    if (t < a.T) route_token<EP>(a, lg + row * LS, rv, t, keep_probs);
     else if (keep_probs)
       for (int e = 0; e < EP; ++e) lg[row * LS + e] = 0.f;  // rows past T add nothing
   }
@@ -386,7 +430,7 @@ cudaError_t launch_route_t(const RouteArgs& a, const CUtensorMap& xmap, const CU
   const int n = 2 * EP * a.d;
   router_weight_kernel<<<(n + 255) / 256, 256, 0, s>>>(a, EP);
   const int grid = (a.T + kTok - 1) / kTok;
-  route_kernel<EP><<<grid, kThreads, smem, s>>>(xmap, wmap, a);
+  route_kernel<EP><<<grid, RouteCfg<EP>::kThreads, smem, s>>>(xmap, wmap, a);
   return cudaGetLastError();
 }
 
