@@ -69,9 +69,12 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v
 }
 
 // Wait for the phase of `bar` with the given parity to complete, giving up
-// after `timeout_ns` or as soon as *abort is set.  The clock is checked on the
-// first retry and then every 64 polls, so a wait that does not complete at
-// once under a limit of a few nanoseconds gives up.  On a timeout it sets
+// after `timeout_ns` or as soon as *abort is set.  The clock and the abort
+// flag are checked every 64 polls -- and, under a limit below 1 ms (a test of
+// this path), also on the first retry, so that a wait that does not complete
+// at once under a limit of a few nanoseconds gives up.  (Checking on the first
+// retry always was measured to cost the MMA issue loop: it delays the poll
+// that sees a stage land.)  On a timeout it sets
 // *abort (and, when `peer_abort` is a shared::cluster address, the same flag
 // of the other CTA of the pair) and ORs `err_bit` into *err.  Returns false
 // if it gave up.  With `cluster` set, the wait acquires at cluster scope (for
@@ -82,9 +85,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   auto poll = [&]() { return cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
   if (poll()) return true;
   const uint64_t t0 = global_timer_ns();
+  const uint32_t first = timeout_ns < 1000000ull ? 1u : 0u;  // the poll index (mod 64) that checks
   for (uint32_t n = 1;; ++n) {
     if (poll()) return true;
-    if ((n & 63u) == 1u) {
+    if ((n & 63u) == first) {
       if (*abort) return false;
       if (global_timer_ns() - t0 > timeout_ns) {
         *abort = 1;
