@@ -113,9 +113,9 @@ MOE_API int64_t moe_max_kept(const moe_config_t* cfg);
  * activations H and the per-assignment expert outputs). */
 MOE_API size_t moe_workspace_size(const moe_config_t* cfg);
 
-/* Zero the workspace header (the device error word, the expert GEMMs' tile
- * counter, the wait limit).  Call once after allocating a workspace, before
- * its first use.  Asynchronous on `stream`. */
+/* Zero the workspace header (the device error word and the wait limit, which
+ * then means the default).  Call once after allocating a workspace, before its
+ * first use.  Asynchronous on `stream`. */
 MOE_API moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, copy the device error word to *code and clear it.

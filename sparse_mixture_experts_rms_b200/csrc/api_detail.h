@@ -30,7 +30,6 @@ struct Layout {
 };
 
 constexpr int kTrainRowAlign = 64;  // row-segment padding of the training layout
-constexpr int64_t BM_PAIR = 256;    // rows of a grouped-GEMM pair tile
 constexpr int kMxRowAlign = 128;    // MX path: a CTA's 128 rows are one scale block
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -80,10 +79,6 @@ moe_status_t run_dispatch(const moe_config_t& c, const Layout& L, void* ws, cons
                           uint8_t* xsf = nullptr, moe_bf16_t* zero_out = nullptr);
 void fill_gemm_common(GemmArgs& g, const moe_config_t& c, const Layout& L, void* ws,
                       const int32_t* perm, const int32_t* offsets);
-// Whether a grouped GEMM launch draws its tiles dynamically: a long reduction
-// (K >= 4096) and many tiles per pair (estimated from the buffer sizes; the
-// exact count is known only on the device).
-int dynamic_tiles(int64_t K, int64_t tiles_estimate, int grid);
 moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x_perm,
                     const float* r, const int32_t* perm, const int32_t* offsets,
                     const moe_bf16_t* W1, const moe_bf16_t* W3, int sms, cudaStream_t s,

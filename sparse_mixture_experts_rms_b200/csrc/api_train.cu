@@ -77,7 +77,6 @@ moe_status_t run_backward(const moe_config_t& c, const Layout& L, void* ws, cons
     fill_gemm_common(g, c, L, ws, perm, offsets);
     g.mode = kGemmBwdH;
     g.bn = bn_h;
-    g.dynamic = dynamic_tiles(d, (static_cast<int64_t>(rows) / BM_PAIR + 1) * std::max<int64_t>(1, F / (c.E * bn_h)), grid);
     g.scale = b.r;
     g.ld_out = L.ldh;
     g.in_u = at<__nv_bfloat16>(ws, L.U);
@@ -100,7 +99,6 @@ moe_status_t run_backward(const moe_config_t& c, const Layout& L, void* ws, cons
     fill_gemm_common(g, c, L, ws, perm, offsets);
     g.mode = kGemmBwdX;
     g.bn = bn_d;
-    g.dynamic = dynamic_tiles(2 * static_cast<int64_t>(ldh), (static_cast<int64_t>(rows) / BM_PAIR + 1) * (d / bn_d), grid);
     g.out_f0 = at<float>(ws, L.dXp);
     g.ld_f = c.d_model;
     EpiMaps em{};
@@ -115,8 +113,6 @@ moe_status_t run_backward(const moe_config_t& c, const Layout& L, void* ws, cons
     fill_gemm_common(g, c, L, ws, perm, offsets);
     g.mode = kGemmWgradX;
     g.bn = 256;
-    g.dynamic = dynamic_tiles(static_cast<int64_t>(rows) / c.E,
-                              c.E * ((d + BM_PAIR - 1) / BM_PAIR) * std::max<int64_t>(1, 2 * F / (c.E * 256)), grid);
     g.out_f0 = dW1;
     g.out_f1 = dW3;
     g.ld_f = static_cast<int>(F);
@@ -132,8 +128,6 @@ moe_status_t run_backward(const moe_config_t& c, const Layout& L, void* ws, cons
     fill_gemm_common(g, c, L, ws, perm, offsets);
     g.mode = kGemmWgradH;
     g.bn = bn_d;
-    g.dynamic = dynamic_tiles(static_cast<int64_t>(rows) / c.E,
-                              c.E * std::max<int64_t>(1, F / (c.E * BM_PAIR)) * (d / bn_d), grid);
     g.out_f0 = dW2;
     g.ld_f = c.d_model;
     EpiMaps em{};

@@ -44,18 +44,7 @@
 // Tiles: expert e contributes ceil(M_e/256) * (N_e/BN) pair tiles, listed on
 // the device from the row offsets (no host sync) in raster groups of M tiles
 // whose A bytes fit a 48 MB L2 budget (M fastest inside a group).  Persistent
-// pairs take tiles from the list in order.  With a long reduction (and many
-// tiles per pair) they take them dynamically (`dynamic`): the leader's
-// producer draws the next index from a counter in the workspace header
-// (zeroed in stream order before each launch) and hands it through a small
-// ring in shared memory to its own MMA and epilogue warps and to the peer
-// CTA, so the tiles in flight stay a contiguous window of the raster (pairs
-// that stall on memory take fewer tiles instead of drifting apart, which
-// would spread the operand panels in use beyond what L2 holds: measured on
-// the Mixtral-shaped up GEMM, DRAM traffic 4.8 -> 3.2 GB against 3.1 GB
-// algorithmic, 3-8 % faster).  With short reductions the hand-off costs more
-// per tile than drift does (measured 5-14 % slower), so pair p then takes
-// tiles p, p + pairs, ... .
+// pairs stride through the list.
 //
 // Warp roles (192 threads per CTA): warp 0 = TMA producer, warp 1 = MMA issuer
 // (leader only) and TMEM owner, warps 2..5 = epilogue (TMEM -> registers ->
@@ -107,7 +96,6 @@ constexpr int kTmemCols = 512;
 constexpr int kAccCols = 256;                 // columns per accumulator buffer
 constexpr int kAtomBytes = BK * 64 * 2;       // one 64(mn) x 64(k) MN-major box: 8 KB
 constexpr long long kL2GroupBudget = 48ll << 20;  // A bytes of one raster group
-constexpr int kTileRing = 8;                   // tile indices handed through shared memory
 // Epilogue staging: per epilogue warp four 32-row x 32-column bf16 boxes
 // (2 KB each, 64-byte swizzle) through which up, down and bwd_h move their
 // rows by TMA
@@ -122,9 +110,6 @@ struct __align__(8) GemmShared {
   uint64_t drain;
   uint64_t ebar[kEpiWarps][2];  // bwd_h: an epilogue warp's U, V box pair landed
   PairDrain pd;                 // the producers' end-of-pipeline handshake
-  uint64_t tq_full[kTileRing];  // each CTA: the slot holds the pair's next tile index
-  uint64_t tq_empty[kTileRing]; // leader: every consumer in the pair has read the slot
-  int tq[kTileRing];            // tile indices in the order the pair processes them (-1: no more)
   uint32_t tmem_base;
   int abort_flag;
   int bad_segment;
@@ -132,6 +117,7 @@ struct __align__(8) GemmShared {
   int tile_start[kMaxExperts + 1];
   int m_tiles[kMaxExperts];
   int n_tiles[kMaxExperts];
+  int k_blocks[kMaxExperts];
   int group_m[kMaxExperts];  // raster block: group_m x group_n tiles (see decode_tile)
   int group_n[kMaxExperts];
   int seg[kMaxExperts + 1];
@@ -193,54 +179,6 @@ __device__ __forceinline__ void store_row_f32(float* dst, const uint32_t (&u)[32
                                __uint_as_float(u[4 * j + 2]), __uint_as_float(u[4 * j + 3]));
 }
 
-// The next tile index of the pair, read by a consumer (the leader's MMA
-// thread and epilogue warps, the peer's producer and epilogue warps) from
-// slot n % kTileRing, which it then releases on the leader.
-__device__ __forceinline__ bool next_tile(GemmShared& sh, uint32_t n, uint32_t rank, uint32_t tq_empty_leader0,
-                                          int* tile, volatile int* abort, uint32_t* err, uint64_t wait_ns,
-                                          uint32_t peer_abort) {
-  const uint32_t slot = n % kTileRing;
-  // the leader's slots are filled by its own producer (CTA scope); the peer's by a remote store
-  if (!mbar_wait(&sh.tq_full[slot], (n / kTileRing) & 1u, abort, err, MOE_DEVERR_TIMEOUT, wait_ns, rank != 0,
-                 peer_abort))
-    return false;
-  *tile = *reinterpret_cast<volatile int*>(&sh.tq[slot]);
-  if (rank == 0)
-    mbar_arrive(&sh.tq_empty[slot]);
-  else
-    mbar_arrive_cluster(tq_empty_leader0 + slot * 8u);
-  return true;
-}
-
-// The leader's producer publishes the pair's n-th tile `t` (-1 when the list
-// is exhausted) in both CTAs' slot n % kTileRing.
-__device__ __forceinline__ bool publish_tile(GemmShared& sh, uint32_t n, int t, volatile int* abort, uint32_t* err,
-                                             uint64_t wait_ns, uint32_t peer_abort) {
-  const uint32_t slot = n % kTileRing;
-  if (!mbar_wait(&sh.tq_empty[slot], ((n / kTileRing) & 1u) ^ 1u, abort, err, MOE_DEVERR_TIMEOUT, wait_ns, true,
-                 peer_abort))
-    return false;
-  sh.tq[slot] = t;
-  st_cluster_u32(map_to_cta(smem_addr(&sh.tq[slot]), 1), static_cast<uint32_t>(t));
-  mbar_arrive(&sh.tq_full[slot]);                                        // this CTA's consumers
-  mbar_arrive_cluster(map_to_cta(smem_addr(&sh.tq_full[slot]), 1));      // the peer's (release: its copy first)
-  return true;
-}
-
-// Tile n of pair p under the static schedule, or -1 past the end.
-__device__ __forceinline__ int static_tile(int pair, int npairs, uint32_t n, int total) {
-  const long long t = static_cast<long long>(pair) + static_cast<long long>(n) * npairs;
-  return t < total ? static_cast<int>(t) : -1;
-}
-
-// The next tile of the list, or -1 when it is exhausted.  (Dealing the list
-// into eight interleaved queues with their own counters was measured slower
-// on every workload: one counter's contention is not what costs.)
-__device__ __forceinline__ int draw_tile(int* ctr, int total) {
-  const int t = atomicAdd(ctr, 1);
-  return t < total ? t : -1;
-}
-
 template <int MODE>
 struct Traits {
   static constexpr bool a_mn = (MODE == kGemmWgradX || MODE == kGemmWgradH);
@@ -265,14 +203,6 @@ __device__ __forceinline__ void geometry(int rows, int f, int d, int bn, int& me
   } else {  // kGemmWgradH
     mext = f; nt = d / bn; kb = rows / BK;
   }
-}
-
-// K blocks of expert e's tiles.
-template <int MODE>
-__device__ __forceinline__ int kblocks_of(const GemmArgs& a, const GemmShared& sh, int e) {
-  int mext, nt, kb;
-  geometry<MODE>(sh.seg[e + 1] - sh.seg[e], a.ffn.off[e + 1] - a.ffn.off[e], a.d, a.bn, mext, nt, kb);
-  return kb;
 }
 
 struct Maps {
@@ -601,7 +531,7 @@ __device__ __forceinline__ void epilogue_wgrad(const GemmArgs& a, const GemmShar
   const int f = a.ffn.off[c.e + 1] - o_e;
   const int m0 = c.mt * BM + static_cast<int>(rank) * BM_CTA + q * 32;
   const int m = m0 + lane;
-  const bool zero = kblocks_of<MODE>(a, sh, c.e) == 0;
+  const bool zero = sh.k_blocks[c.e] == 0;
   const int m_end = MODE == kGemmWgradX ? a.d : f;
   const bool valid = m < m_end;
   const bool staged = a.staged != 0 && m0 + 32 <= m_end;
@@ -671,10 +601,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
       mbar_init(&sh.ebar[w][1], 1);
     }
     pair_drain_init(sh.pd);
-    for (int i = 0; i < kTileRing; ++i) {
-      mbar_init(&sh.tq_full[i], 1);
-      mbar_init(&sh.tq_empty[i], 2 + 2 * EPI);  // leader MMA + peer producer + both CTAs' epilogue warps
-    }
     sh.abort_flag = 0;
     sh.bad_segment = 0;
     fence_mbar_init();
@@ -718,6 +644,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
     }
     sh.m_tiles[tid] = mtc;
     sh.n_tiles[tid] = ntc;
+    sh.k_blocks[tid] = kb;
     sh.group_m[tid] = gm;
     sh.group_n[tid] = gn;
     sh.tile_start[tid + 1] = (mt > 0 && nt > 0) ? mt * nt : 0;  // count for now
@@ -742,7 +669,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
   // main-loop waits: the workspace's limit; a wait that gives up also stops the other CTA
   const uint64_t wait_ns = wait_limit_ns(a.wait_ctl);
   const uint32_t peer_abort = map_to_cta(smem_addr(&sh.abort_flag), rank ^ 1u);
-  const uint32_t tq_empty_leader0 = map_to_cta(smem_addr(&sh.tq_empty[0]), 0);
 
   if (warp == 0) {
     // ================= TMA producer (one lane per CTA)
@@ -751,44 +677,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
       const uint32_t tx_pair = 2u * (kABytes + static_cast<uint32_t>(a.bn / 2) * BK * 2u);
       uint32_t it = 0;
       bool ok = true;
-      // The leader draws the next index a few K blocks before the current tile
-      // ends and publishes it two K blocks before, so the counter's round trip
-      // and the hand-off to the peer overlap loads still being issued; the
-      // pair holds the drawn tile only briefly (drawing a whole tile ahead was
-      // measured slower: it unbalances the last wave).
-      constexpr int kDrawAhead = 4, kPublishAhead = 2;
-      const bool dyn = a.dynamic != 0;
-      int cur = -1;
-      if (dyn && rank == 0) {
-        cur = draw_tile(a.tile_ctr, total);
-        ok = publish_tile(sh, 0, cur, abort_flag, a.err, wait_ns, peer_abort);
-      }
-      for (uint32_t n = 0; ok; ++n) {
-        int tile = dyn ? cur : static_tile(pair, npairs, n, total);
-        if (dyn && rank != 0 &&
-            !next_tile(sh, n, rank, tq_empty_leader0, &tile, abort_flag, a.err, wait_ns, peer_abort)) {
-          ok = false;
-          break;
-        }
-        if (tile < 0) break;
+      for (int tile = pair; ok && tile < total; tile += npairs) {
         const TileCoord c = decode_tile(sh, E, tile);
         const int o_e = a.ffn.off[c.e];
         const int f = a.ffn.off[c.e + 1] - o_e;
-        const int kblocks = kblocks_of<MODE>(a, sh, c.e);
-        const int kdraw = kblocks > kDrawAhead ? kblocks - kDrawAhead : 0;
-        const int kpub = kblocks - kPublishAhead > kdraw ? kblocks - kPublishAhead : kdraw;
-        int pending = -1;
-        bool published = false;
+        const int kblocks = sh.k_blocks[c.e];
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          if (dyn && rank == 0 && kb == kdraw) pending = draw_tile(a.tile_ctr, total);
-          if (dyn && rank == 0 && kb == kpub) {
-            cur = pending;
-            published = true;
-            if (!publish_tile(sh, n + 1, cur, abort_flag, a.err, wait_ns, peer_abort)) {
-              ok = false;
-              break;
-            }
-          }
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1u;
           if (!mbar_wait(&sh.empty[s], ph ^ 1u, abort_flag, a.err, MOE_DEVERR_TIMEOUT, wait_ns, false,
@@ -801,10 +695,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
           if (rank == 0) mbar_arrive_expect_tx(&sh.full[s], tx_pair);
           issue_loads<MODE>(maps, c, kb, sA, sA + kABytes, bar, sh.seg[c.e], o_e, f, rank, a.bn);
         }
-        if (dyn && ok && rank == 0 && !published) {  // a tile without K blocks (an expert with no rows)
-          cur = draw_tile(a.tile_ctr, total);
-          ok = publish_tile(sh, n + 1, cur, abort_flag, a.err, wait_ns, peer_abort);
-        }
       }
       // no copy into either CTA is in flight when it exits, whatever stopped the loop
       pair_producer_drain<kStages>(sh.pd, sh.full, it, rank, tx_pair / 2u, a.err);
@@ -815,15 +705,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
       const uint32_t idesc = umma_idesc_bf16(BM, a.bn, Traits<MODE>::b_mn ? 1u : 0u, Traits<MODE>::a_mn ? 1u : 0u);
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (; ok; ++tcount) {
-        int tile = static_tile(pair, npairs, tcount, total);
-        if (a.dynamic && !next_tile(sh, tcount, 0, tq_empty_leader0, &tile, abort_flag, a.err, wait_ns, peer_abort)) {
-          ok = false;
-          break;
-        }
-        if (tile < 0) break;
+      for (int tile = pair; ok && tile < total; tile += npairs, ++tcount) {
         const TileCoord c = decode_tile(sh, E, tile);
-        const int kblocks = kblocks_of<MODE>(a, sh, c.e);
+        const int kblocks = sh.k_blocks[c.e];
         const uint32_t buf = tcount & 1u;
         const uint32_t aph = (tcount >> 1) & 1u;
         // both CTAs' epilogues release the buffer (the peer's arrival is remote)
@@ -877,15 +761,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
     }
     const uint32_t tempty_leader0 = map_to_cta(smem_addr(&sh.tempty[0]), 0);
     uint32_t tcount = 0, eit = 0;
-    for (;; ++tcount) {
-      int tile = static_tile(pair, npairs, tcount, total), got = 1;
-      if (a.dynamic) {
-        if (lane == 0)
-          got = next_tile(sh, tcount, rank, tq_empty_leader0, &tile, abort_flag, a.err, wait_ns, peer_abort) ? 1 : 0;
-        got = __shfl_sync(0xFFFFFFFFu, got, 0);
-        tile = __shfl_sync(0xFFFFFFFFu, tile, 0);
-      }
-      if (!got || tile < 0) break;
+    for (int tile = pair; tile < total; tile += npairs, ++tcount) {
       const TileCoord c = decode_tile(sh, E, tile);
       const uint32_t buf = tcount & 1u;
       const uint32_t aph = (tcount >> 1) & 1u;
@@ -966,14 +842,6 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA0, con
   static const EpiMaps kNoMaps{};
   const EpiMaps& em = em_opt != nullptr ? *em_opt : kNoMaps;
   if (a.epi8 && a.mode != kGemmUp && a.mode != kGemmDown) return cudaErrorInvalidValue;
-  if (a.tile_ctr == nullptr) return cudaErrorInvalidValue;
-  // the tile list is drawn from the start.  (Having the last CTA of each launch
-  // rewind the counter instead was measured ~10 us slower per launch: every
-  // CTA's exit then waits on one contended atomic.)
-  if (a.dynamic) {
-    cudaError_t e0 = cudaMemsetAsync(a.tile_ctr, 0, sizeof(int), s);
-    if (e0 != cudaSuccess) return e0;
-  }
   GemmArgs ga = a;
   ga.staged = em_opt != nullptr ? 1 : 0;
   switch (a.mode) {

@@ -351,12 +351,7 @@ void fill_gemm_common(GemmArgs& g, const moe_config_t& c, const Layout& L, void*
   g.perm = perm;
   g.err = at<uint32_t>(ws, L.err);
   g.wait_ctl = at<uint32_t>(ws, kWaitCtlOffset);
-  g.tile_ctr = at<int>(ws, kTileCtrOffset);
   for (int e = 0; e <= c.E; ++e) g.ffn.off[e] = c.ffn_offsets[e];
-}
-
-int dynamic_tiles(int64_t K, int64_t tiles_estimate, int grid) {
-  return (K >= 4096 && tiles_estimate >= 16ll * (grid / 2)) ? 1 : 0;
 }
 
 // GEMM 1: x_perm [rows, d] x (W1 | W3) [d, F] -> SwiGLU -> H [rows, ldh] (workspace)
@@ -384,8 +379,6 @@ moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_
   // short reduction: a tile's MMAs take about as long as its epilogue, so run 8 epilogue
   // warps (the training up keeps 4: its three output boxes per chunk need a warp's 8 KB)
   g.epi8 = (c.d_model <= kEpi8MaxK && U == nullptr) ? 1 : 0;
-  const int grid = gemm_grid_of_current_device();
-  g.dynamic = dynamic_tiles(c.d_model, (L.max_kept / BM_PAIR + 1) * std::max<int64_t>(1, F / (c.E * kBlockN)), grid);
   const uint64_t ldh = static_cast<uint64_t>(L.ldh);
   EpiMaps em{};
   if (!make_map(&em.m[0], g.out, ldh, rows, ldh, 32, 32, true) ||
@@ -393,7 +386,7 @@ moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_
                         !make_map(&em.m[2], V, ldh, rows, ldh, 32, 32, true))))
     return MOE_ERR_CUDA;
   (void)sms;
-  return cuda_status(launch_grouped_gemm(g, mA, mA, mB0, mB1, grid, s, &em));
+  return cuda_status(launch_grouped_gemm(g, mA, mA, mB0, mB1, gemm_grid_of_current_device(), s, &em));
 }
 
 // GEMM 2: H [rows, f_e] (workspace) x W2 [F, d] -> y [rows, d], gate in the epilogue;
@@ -419,7 +412,6 @@ moe_status_t run_down(const moe_config_t& c, const Layout& L, void* ws, const fl
   g.ld_out = c.d_model;
   g.out_yu = reinterpret_cast<__nv_bfloat16*>(yu);
   g.epi8 = L.ldh <= kEpi8MaxK ? 1 : 0;  // the down GEMM reduces over the expert width
-  g.dynamic = dynamic_tiles(L.ldh, (L.max_kept / BM_PAIR + 1) * (c.d_model / g.bn), gemm_grid_of_current_device());
   (void)sms;
   if (to_token && c.k == 1 && yu == nullptr) {  // scattered rows: stored row by row
     g.to_token = 1;

@@ -19,12 +19,11 @@ constexpr int kDispatchTile = 1024;     // assignments per dispatch CTA
 constexpr uint64_t kWaitTimeoutNs = 4000000000ull;  // bounded pipeline waits: 4 s (default)
 
 // Workspace header (256 bytes at offset 0 of every workspace): word 0 = the
-// device error word, word 1 = a CTA ticket, word 4 = the grouped GEMMs' tile
-// counter (zeroed before each launch), words 2-3 = the wait-limit control: the tag kWaitCtlTag and a limit in ns for the pipeline waits of
+// device error word, word 1 = a CTA ticket, words 2-3 = the wait-limit
+// control: the tag kWaitCtlTag and a limit in ns for the pipeline waits of
 // the kernels that run on this workspace (moe_set_wait_limit).  Any other
 // tag, or a zero limit, means the default kWaitTimeoutNs.
 constexpr size_t kWaitCtlOffset = 8;
-constexpr size_t kTileCtrOffset = 16;  // word 4: the grouped GEMMs' tile counter
 constexpr uint32_t kWaitCtlTag = 0x544D494Cu;
 __device__ __forceinline__ uint64_t wait_limit_ns(const uint32_t* ctl) {
   if (ctl != nullptr) {
@@ -177,8 +176,6 @@ struct GemmArgs {
   int ld_f;
   uint32_t* err;
   const uint32_t* wait_ctl;  // wait-limit control of the workspace header
-  int* tile_ctr;            // next tile of the list (workspace header word; zeroed before each launch)
-  int dynamic;              // 1: pairs draw tiles from tile_ctr; 0: pair p takes p, p + pairs, ...
   ExpertTable ffn;
   int to_token;             // down, k = 1: row p goes to row perm[p] (its token) of out [T, d]
   int staged;               // set by the launcher: epilogue tensor maps were given
