@@ -72,9 +72,7 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v
 // after `timeout_ns` or as soon as *abort is set.  The clock and the abort
 // flag are checked every 64 polls -- and, under a limit below 1 ms (a test of
 // this path), also on the first retry, so that a wait that does not complete
-// at once under a limit of a few nanoseconds gives up.  (Checking on the first
-// retry always was measured to cost the MMA issue loop: it delays the poll
-// that sees a stage land.)  On a timeout it sets
+// at once under a limit of a few nanoseconds gives up.  On a timeout it sets
 // *abort (and, when `peer_abort` is a shared::cluster address, the same flag
 // of the other CTA of the pair) and ORs `err_bit` into *err.  Returns false
 // if it gave up.  With `cluster` set, the wait acquires at cluster scope (for
