@@ -44,8 +44,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (dram__bytes_read.sum + dram__bytes_write.sum, 1-pass metrics).  Reported
 # only while the kernel sources still hash to `digest`; after any change it
 # is null until re-measured.
-MEASURED_TRAFFIC = {"workload": "mixtral", "T": 16384, "digest": "b4abbd4f955304ae",
-                    "bytes": 2.2958e9 + 0.9299e9}   # dram read + write of the up launch
+MEASURED_TRAFFIC = {"workload": "mixtral", "T": 16384, "digest": "26676d48ab70fd46",
+                    "bytes": 4.7353e9 + 0.9312e9}   # dram read + write of the up launch
 
 
 def kernel_digest() -> str:
@@ -469,6 +469,11 @@ def run_ours(args, rank, world, local):
     stages = ["route", "dispatch", "gemm_up", "gemm_down", "combine"]
 
     def staged(evs):
+        # queued behind a ~1 ms device-side spin, so the host has enqueued all
+        # five calls before the first event fires: the events time the kernels
+        # back to back, not the host's enqueue of each call
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(2_000_000)
         evs[0].record(stream)
         moe.moe_route(c, x, gamma, Wr, bias, st["idx"], st["gate"], st["r"], None, ws, stream=stream)
         evs[1].record(stream)
@@ -686,6 +691,9 @@ def mx_leg(moe, cfg, w, x, gamma, Wr, bias, W1, W3, W2, stream, steps, F_alg, sa
            "layer_frac_of_fp8_peak": F_alg / (ms * 1e-3) / 1e12 / fp8_peak,
            "peak_note": f"fp8 peak = 2 x {peaks['source']} sustained bf16 ({fp8_peak:.0f} TFLOP/s)",
            "dtype": "mxfp8 expert GEMMs (E4M3, E8M0 per 32), bf16 router/out", "steps": n,
+           "accuracy": ("output 7.6e-2 .. 7.8e-2 normwise per token from the exact (fp64) layer: the "
+                        "format's own error, above the bf16 path's 2e-2 bar; parity is checked against "
+                        "the MX oracle (same quantisation), within 2.4e-3"),
            "device_error": moe.moe_get_device_error(ws, stream=stream, raise_on_error=False)}
     del wq, ws
     torch.cuda.empty_cache()
