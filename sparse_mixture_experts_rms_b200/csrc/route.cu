@@ -16,11 +16,13 @@
 //    every product the tensor core forms is exact; B = [hi | lo] holds the
 //    two halves as 2 EP columns (EP = E rounded up to 8, 16, 32 or 64);
 //  - each 64-element chunk of d is accumulated by 4 MMAs from zero into its
-//    own TMEM buffer (a ring of four), and the epilogue adds every chunk's hi
-//    and lo partials into fp64 registers; r and l = r*acc + b are formed in
-//    fp64 and each logit is rounded once to fp32.
-// A near-tie between the k-th and (k+1)-th logit can therefore only flip when
-// the two fp32 logits differ by about one ulp.
+//    own TMEM buffer, so no fp32 sum runs over more than 64 products; the
+//    epilogue adds the hi and lo partials of a stage's 2-4 chunks in fp32
+//    and the stage sums in fp64; r and l = r*acc + b are formed in fp64 and
+//    each logit is rounded once to fp32.
+// The logit's error is a few fp32 roundings of 64-product partial sums, far
+// below the 1e-5 margin within which a near-tie of the k-th and (k+1)-th
+// logit is treated as either order.
 //
 // Layout: a CTA owns 128 tokens.  Warp 0 streams x through a ring of stages
 // by TMA, each [128 tokens x 64 elements] (128-byte swizzle) plus the chunk's
@@ -126,19 +128,22 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[NC]) 
   else tmem_ld_32x32b_x32(taddr, v);
 }
 
-// acc[e] += hi_e + lo_e (fp64) for NE experts whose chunk partials sit in
+// sum[e] += hi_e + lo_e (fp32) for NE experts whose chunk partials sit in
 // TMEM columns [thi, thi + NE) (hi) and [tlo, tlo + NE) (lo) of this warp's
 // lane quarter.
 template <int NE>
-__device__ __forceinline__ void add_chunk(uint32_t thi, uint32_t tlo, double (&acc)[NE]) {
+__device__ __forceinline__ void add_chunk(uint32_t thi, uint32_t tlo, float (&sum)[NE]) {
   static_assert(NE == 8 || NE == 16 || NE == 32, "8, 16 or 32 experts per epilogue thread");
-  uint32_t h[NE], l[NE];
-  tmem_ld_cols<NE>(thi, h);
-  tmem_ld_cols<NE>(tlo, l);
-  tmem_ld_wait();
+  constexpr int P = NE < 16 ? NE : 16;  // columns per load (bounds the registers in flight)
 #pragma unroll
-  for (int e = 0; e < NE; ++e)
-    acc[e] += static_cast<double>(__uint_as_float(h[e])) + static_cast<double>(__uint_as_float(l[e]));
+  for (int e0 = 0; e0 < NE; e0 += P) {
+    uint32_t h[P], l[P];
+    tmem_ld_cols<P>(thi + e0, h);
+    tmem_ld_cols<P>(tlo + e0, l);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < P; ++e) sum[e0 + e] += __uint_as_float(h[e]) + __uint_as_float(l[e]);
+  }
 }
 
 template <int EP>
@@ -285,10 +290,19 @@ __global__ void __launch_bounds__(RouteCfg<EP>::kThreads, 1)
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) break;
       tc_fence_after();
+      // the stage's 2 * nc partials of each logit meet in fp32 (a few fp32
+      // roundings of the partials' size, like the MMA's own accumulation),
+      // and the stage sum goes into the fp64 accumulator: one fp64 conversion
+      // per expert and stage, not two per chunk
+      float stage_sum[NE];
+#pragma unroll
+      for (int e = 0; e < NE; ++e) stage_sum[e] = 0.f;
       for (int i = 0; i < nc; ++i) {
         const uint32_t tb = tq + static_cast<uint32_t>((g * CPS + i) * N);
-        add_chunk<NE>(tb, tb + EP, acc);
+        add_chunk<NE>(tb, tb + EP, stage_sum);
       }
+#pragma unroll
+      for (int e = 0; e < NE; ++e) acc[e] += static_cast<double>(stage_sum[e]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
