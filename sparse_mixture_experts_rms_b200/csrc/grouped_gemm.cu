@@ -307,6 +307,26 @@ __device__ __forceinline__ void box_slot_store(const EpiMaps& em, uint8_t* slot,
   }
 }
 
+// A row-tile epilogue thread's assignment (perm entry of its row, -1 past the
+// expert's rows or at padding) and scale (up: r of the token; down: the
+// gate), read before the thread waits for the tile's accumulator so that the
+// two dependent loads overlap the tile's MMAs.
+struct RowPre {
+  int asg;
+  float scale;
+};
+
+template <int MODE>
+__device__ __forceinline__ RowPre row_pre(const GemmArgs& a, const GemmShared& sh, const TileCoord& c, int q,
+                                          int lane, uint32_t rank) {
+  const int p = sh.seg[c.e] + c.mt * BM + static_cast<int>(rank) * BM_CTA + q * 32 + lane;
+  const int asg = p < sh.seg[c.e + 1] ? a.perm[p] : -1;
+  float scale = 0.f;
+  if (MODE == kGemmUp && asg >= 0) scale = a.scale[asg / a.k];
+  if (MODE == kGemmDown && asg >= 0) scale = a.scale[asg];
+  return RowPre{asg, scale};
+}
+
 // Row-tile epilogues (up, down, bwd_x); one thread per accumulator row
 // (TMEM lane), 32-column chunks.  The outputs leave through shared memory by
 // TMA when the warp's 32 rows all belong to the expert (`staged`); otherwise
@@ -316,18 +336,18 @@ template <int MODE>
 __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShared& sh, const EpiMaps& em,
                                               const TileCoord& c, uint32_t taddr, int q, int lane,
                                               uint32_t rank, uint8_t* boxes, int bpw, uint32_t& n, int c_lo,
-                                              int c_hi) {
+                                              int c_hi, const RowPre& pre) {
   const int p0 = sh.seg[c.e] + c.mt * BM + static_cast<int>(rank) * BM_CTA + q * 32;
   const int p = p0 + lane;
   const bool valid = p < sh.seg[c.e + 1];
   const int nbox_max = MODE == kGemmUp ? (a.out_u != nullptr ? 3 : 1) : (MODE == kGemmDown && a.out_yu != nullptr ? 2 : 1);
   // rows sent to their tokens (down, k = 1) are not contiguous: no boxes
   const bool staged = a.staged != 0 && a.to_token == 0 && nbox_max <= bpw && p0 + 32 <= sh.seg[c.e + 1];
-  const int asg = valid ? a.perm[p] : -1;
+  const int asg = pre.asg;
   const bool pad = valid && asg < 0;
   const size_t prow = static_cast<size_t>(valid ? p : 0);
   if (MODE == kGemmUp) {
-    const float scale = asg >= 0 ? a.scale[asg / a.k] : 0.f;
+    const float scale = pre.scale;
     const size_t off = prow * a.ld_out + c.nt * kBlockN;
     const bool keep_uv = a.out_u != nullptr;
     const int nbox = keep_uv ? 3 : 1;
@@ -367,7 +387,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
       if (staged) box_slot_store(em, slot, nbox, c.nt * kBlockN + cc, p0, lane);
     }
   } else if (MODE == kGemmDown) {
-    const float scale = asg >= 0 ? a.scale[asg] : 0.f;
+    const float scale = pre.scale;
     const size_t orow = a.to_token ? static_cast<size_t>(asg >= 0 ? asg : 0) : prow;
     const size_t off = orow * a.ld_out + c.nt * a.bn;
     const bool keep_yu = a.out_yu != nullptr;
@@ -765,6 +785,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
       const TileCoord c = decode_tile(sh, E, tile);
       const uint32_t buf = tcount & 1u;
       const uint32_t aph = (tcount >> 1) & 1u;
+      RowPre pre{-1, 0.f};
+      if (Traits<MODE>::row_tiles && MODE != kGemmBwdH) pre = row_pre<MODE>(a, sh, c, q, lane, rank);
       bool ok = true;
       if (lane == 0)
         ok = mbar_wait(&sh.tfull[buf], aph, abort_flag, a.err, MOE_DEVERR_TIMEOUT, wait_ns, false, peer_abort);
@@ -776,7 +798,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
         ok = epilogue_dsh(a, sh, em, c, taddr, q, lane, rank, my_boxes, sh.ebar[w], eit, abort_flag, wait_ns,
                           peer_abort);
       else if (Traits<MODE>::row_tiles)
-        epilogue_rows<MODE>(a, sh, em, c, taddr, q, lane, rank, my_boxes, bpw, eit, c_lo, c_hi);
+        epilogue_rows<MODE>(a, sh, em, c, taddr, q, lane, rank, my_boxes, bpw, eit, c_lo, c_hi, pre);
       else
         epilogue_wgrad<MODE>(a, sh, em, c, taddr, q, lane, rank, my_boxes, eit);
       tc_fence_before();
