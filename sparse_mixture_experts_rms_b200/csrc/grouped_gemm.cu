@@ -392,12 +392,9 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
     const size_t off = orow * a.ld_out + c.nt * a.bn;
     const bool keep_yu = a.out_yu != nullptr;
     const int nbox = keep_yu ? 2 : 1;
-#pragma unroll 1
-    for (int cc = c_lo; cc < c_hi; cc += 32) {
-      uint32_t u[32];
-      tmem_ld_32x32b_x32(taddr + cc, u);
-      tmem_ld_wait();
-      if (!valid || (a.to_token && asg < 0)) continue;  // never taken when staged
+    // one 32-column chunk: gate scale, bf16 pack, out through the staged boxes or row stores
+    auto chunk = [&](const uint32_t (&u)[32], int cc) {
+      if (!valid || (a.to_token && asg < 0)) return;  // never taken when staged
       uint32_t o[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j)
@@ -417,6 +414,20 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& a, const GemmShare
         else store_row_bf16(a.out_yu + off + cc, o);
       }
       if (staged) box_slot_store(em, slot, nbox, c.nt * a.bn + cc, p0, lane);
+    };
+    // the next chunk's TMEM load is in flight while this one is scaled,
+    // packed, fenced and stored (two 32-column register sets)
+    uint32_t ua[32], ub[32];
+    tmem_ld_32x32b_x32(taddr + c_lo, ua);
+#pragma unroll 1
+    for (int cc = c_lo; cc < c_hi; cc += 64) {
+      tmem_ld_wait();  // ua
+      if (cc + 32 < c_hi) tmem_ld_32x32b_x32(taddr + cc + 32, ub);
+      chunk(ua, cc);
+      if (cc + 32 >= c_hi) break;
+      tmem_ld_wait();  // ub
+      if (cc + 64 < c_hi) tmem_ld_32x32b_x32(taddr + cc + 64, ua);
+      chunk(ub, cc + 32);
     }
   } else {  // kGemmBwdX: fp32 rows, staged as 32 x 32 fp32 boxes (128-byte swizzle, two per warp)
     float* dst = a.out_f0 + prow * a.ld_f + c.nt * a.bn;
