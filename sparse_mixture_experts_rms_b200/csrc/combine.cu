@@ -8,11 +8,13 @@
 // accumulated in fp32 in slot order j = 0..k-1 (no atomics: one warp owns a
 // token row).  A token whose slots were all dropped gets a zero row.
 #include "moe_internal.h"
+#include "ptx.cuh"
 
 namespace moe {
 namespace {
 
 __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
+  griddep_wait();  // y and inv_perm come from the kernels before
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
   const int chunks = a.d / 8;
@@ -69,8 +71,7 @@ cudaError_t launch_combine(const CombineArgs& a, int num_sms, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
   int grid = (a.T + 7) / 8;
   grid = grid < num_sms * 8 ? grid : num_sms * 8;
-  combine_kernel<<<grid, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, s, a);
 }
 
 }  // namespace moe

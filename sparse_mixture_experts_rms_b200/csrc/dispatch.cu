@@ -99,6 +99,7 @@ __device__ bool look_back(const ScanView& v, int b, int lane, uint64_t wait_ns, 
 
 // One cooperative launch over a persistent grid; CTA c handles tiles c, c + G, ...
 __global__ void __launch_bounds__(kDispThreads) dispatch_kernel(const DispatchArgs a, int ntiles) {
+  griddep_launch_dependents();  // the permute may launch; it waits for this grid to finish
   __shared__ int hist[kMaxExperts];      // this tile's counts
   __shared__ int excl[kMaxExperts];      // assignments to e in the tiles before this one
   __shared__ int offs[kMaxExperts + 1];  // row-segment offsets (kept rows + padding)
@@ -253,6 +254,8 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_kernel(const DispatchAr
 // x_perm[p] = bf16(x[perm[p]/k] * gamma) for p < offsets[E]; zero rows where
 // perm[p] = -1 (padding).
 __global__ void __launch_bounds__(256) permute_rows_kernel(const DispatchArgs a) {
+  griddep_wait();                 // perm and offsets come from dispatch_kernel
+  griddep_launch_dependents();    // the up GEMM may launch and set up meanwhile
   const int n_kept = min(a.offsets[a.E], a.max_kept);
   const int lane = threadIdx.x & 31;
   const int warps = (gridDim.x * blockDim.x) >> 5;
@@ -380,7 +383,7 @@ cudaError_t launch_dispatch(const DispatchArgs& a, int num_sms, cudaStream_t s) 
     if (a.x8 != nullptr)
       permute_rows_mx_kernel<<<grid, 256, 0, s>>>(a);
     else
-      permute_rows_kernel<<<grid, 256, 0, s>>>(a);
+      return launch_pdl(permute_rows_kernel, dim3(grid), dim3(256), 0, s, a);
   }
   return cudaGetLastError();
 }

@@ -648,6 +648,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
     tmem_alloc_pair(&sh.tmem_base, kTmemCols);
     tmem_relinquish_pair();
   }
+  // barriers, TMEM and descriptors are set up while the kernel before drains;
+  // the row offsets and every operand come from the kernels before
+  griddep_wait();
   if (tid < E + 1) sh.seg[tid] = a.offsets[tid];
   __syncthreads();
   if (tid < E) {
@@ -822,6 +825,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
   }
 
   // ---- teardown: neither CTA leaves while its pair may still touch its memory
+  griddep_launch_dependents();  // the next kernel may launch and set up meanwhile
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
@@ -877,35 +881,36 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA0, con
   if (a.epi8 && a.mode != kGemmUp && a.mode != kGemmDown) return cudaErrorInvalidValue;
   GemmArgs ga = a;
   ga.staged = em_opt != nullptr ? 1 : 0;
+  cudaError_t e = cudaSuccess;
   switch (a.mode) {
     case kGemmUp:
       if (ga.epi8)
-        grouped_gemm_kernel<kGemmUp, 8><<<grid, threads_of(8), kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+        e = launch_pdl(grouped_gemm_kernel<kGemmUp, 8>, dim3(grid), dim3(threads_of(8)), kSmemBytes, s, mapA0, mapA1, mapB0, mapB1, ga, em);
       else
-        grouped_gemm_kernel<kGemmUp, 4><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+        e = launch_pdl(grouped_gemm_kernel<kGemmUp, 4>, dim3(grid), dim3(kThreads), kSmemBytes, s, mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmDown:
       if (ga.epi8)
-        grouped_gemm_kernel<kGemmDown, 8><<<grid, threads_of(8), kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+        e = launch_pdl(grouped_gemm_kernel<kGemmDown, 8>, dim3(grid), dim3(threads_of(8)), kSmemBytes, s, mapA0, mapA1, mapB0, mapB1, ga, em);
       else
-        grouped_gemm_kernel<kGemmDown, 4><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+        e = launch_pdl(grouped_gemm_kernel<kGemmDown, 4>, dim3(grid), dim3(kThreads), kSmemBytes, s, mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmBwdH:
-      grouped_gemm_kernel<kGemmBwdH, 4><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+      e = launch_pdl(grouped_gemm_kernel<kGemmBwdH, 4>, dim3(grid), dim3(kThreads), kSmemBytes, s, mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmBwdX:
-      grouped_gemm_kernel<kGemmBwdX, 4><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+      e = launch_pdl(grouped_gemm_kernel<kGemmBwdX, 4>, dim3(grid), dim3(kThreads), kSmemBytes, s, mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmWgradX:
-      grouped_gemm_kernel<kGemmWgradX, 4><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+      e = launch_pdl(grouped_gemm_kernel<kGemmWgradX, 4>, dim3(grid), dim3(kThreads), kSmemBytes, s, mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     case kGemmWgradH:
-      grouped_gemm_kernel<kGemmWgradH, 4><<<grid, kThreads, kSmemBytes, s>>>(mapA0, mapA1, mapB0, mapB1, ga, em);
+      e = launch_pdl(grouped_gemm_kernel<kGemmWgradH, 4>, dim3(grid), dim3(kThreads), kSmemBytes, s, mapA0, mapA1, mapB0, mapB1, ga, em);
       break;
     default:
       return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace moe

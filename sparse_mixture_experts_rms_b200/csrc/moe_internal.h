@@ -10,6 +10,8 @@
 
 #include "moe.h"
 
+#include <utility>
+
 namespace moe {
 
 constexpr int kMaxExperts = 64;
@@ -273,5 +275,25 @@ cudaError_t prepare_grouped_gemm();
 // the number of co-resident 2-CTA clusters times 2.
 int grouped_gemm_max_grid(int num_sms);
 size_t grouped_gemm_smem_bytes();
+
+// Launch with programmatic stream serialization: the kernel's CTAs may start
+// (and run their prologue up to griddep_wait, which every such kernel calls
+// before touching global memory another kernel uses) while the previous
+// kernel of the stream drains.  Used between the layer's consecutive kernels.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 }  // namespace moe

@@ -105,6 +105,19 @@ __device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) 
                : "memory");
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Wait until the kernel this one was launched after (with programmatic stream
+// serialization) has completed and its memory is visible; returns at once
+// for a kernel launched the ordinary way.  Every thread that reads or writes
+// global memory another kernel of the stream uses calls it first.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next kernel of the stream, if launched programmatically, begin
+// launching (its CTAs then run up to their griddep_wait).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

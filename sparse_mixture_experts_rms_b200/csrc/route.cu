@@ -86,6 +86,7 @@ __device__ __forceinline__ uint32_t bf16_bits_rn(float v) {
 // B = (gamma * Wr)^T split exactly into bf16 hi (rows [0, EP)) and lo (rows
 // [EP, 2 EP)), K-major [2 EP, d]; experts n >= E are zero rows.
 __global__ void router_weight_kernel(const RouteArgs a, int ep) {
+  griddep_launch_dependents();  // the router may launch and set up meanwhile
   const int n = 2 * ep * a.d;
   const uint16_t* gam = reinterpret_cast<const uint16_t*>(a.gamma);
   const uint16_t* wr = reinterpret_cast<const uint16_t*>(a.Wr);
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(RouteCfg<EP>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();  // the split router weights come from router_weight_kernel
   uint32_t* err = a.err ? a.err : &sh.dummy_err;
   volatile int* abort_flag = &sh.abort_flag;
   const uint32_t tmem_base = sh.tmem_base;
@@ -444,8 +446,7 @@ cudaError_t launch_route_t(const RouteArgs& a, const CUtensorMap& xmap, const CU
   const int n = 2 * EP * a.d;
   router_weight_kernel<<<(n + 255) / 256, 256, 0, s>>>(a, EP);
   const int grid = (a.T + kTok - 1) / kTok;
-  route_kernel<EP><<<grid, RouteCfg<EP>::kThreads, smem, s>>>(xmap, wmap, a);
-  return cudaGetLastError();
+  return launch_pdl(route_kernel<EP>, dim3(grid), dim3(RouteCfg<EP>::kThreads), smem, s, xmap, wmap, a);
 }
 
 // Load-balance metrics from the router's prob_mean and the dispatch counts:
