@@ -76,7 +76,7 @@ moe_status_t run_dispatch(const moe_config_t& c, const Layout& L, void* ws, cons
                           const moe_bf16_t* x, const moe_bf16_t* gamma, int32_t* counts,
                           int32_t* offsets, int32_t* perm, int32_t* inv_perm, moe_bf16_t* x_perm,
                           int sms, cudaStream_t s, int row_align = 1, uint8_t* x8 = nullptr,
-                          uint8_t* xsf = nullptr, moe_bf16_t* zero_out = nullptr);
+                          uint8_t* xsf = nullptr);
 void fill_gemm_common(GemmArgs& g, const moe_config_t& c, const Layout& L, void* ws,
                       const int32_t* perm, const int32_t* offsets);
 moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x_perm,

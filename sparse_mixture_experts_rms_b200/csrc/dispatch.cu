@@ -226,18 +226,6 @@ __global__ void __launch_bounds__(kDispThreads) dispatch_kernel(const DispatchAr
         }
       }
       if (dropped) a.inv_perm[asg] = -1;
-      // k = 1 with an output to clear: a dropped token's row of out is zero
-      if (a.zero_out != nullptr) {
-        unsigned todo = __ballot_sync(0xFFFFFFFFu, dropped);
-        const int chunks = a.d / 8;
-        while (todo) {
-          const int src = __ffs(todo) - 1;
-          todo &= todo - 1u;
-          const int t = base + i + warp * 32 + src;  // k = 1: the assignment is the token
-          uint4* row = reinterpret_cast<uint4*>(a.zero_out + static_cast<size_t>(t) * a.d);
-          for (int c = lane; c < chunks; c += 32) row[c] = make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
       __syncthreads();
       if (tid < E) {
         int s2 = 0;

@@ -78,7 +78,6 @@ struct DispatchArgs {
                             // padded to that multiple (perm = -1, zero rows there)
   uint8_t* x8;              // MX mode (x_perm == null): E4M3 codes [max_kept, d]
   uint8_t* xsf;             // MX mode: E8M0 scale blocks of x8 (see mx_sf_offset)
-  __nv_bfloat16* zero_out;  // k = 1 only, may be null: rows of dropped tokens set to zero [T, d]
   const uint32_t* wait_ctl; // wait-limit control of the workspace header, may be null
 };
 
