@@ -263,6 +263,13 @@ MOE_API moe_status_t moe_combine(const moe_config_t* cfg, const moe_bf16_t* y, c
 
 /* The whole layer: route -> dispatch -> experts -> combine, on one stream,
  * with no host synchronisation (the kept counts never leave the device).
+ * With k = 1 there is no combine: the second GEMM writes each kept row
+ * straight to its token's row of out (a sum of one term, MoE glossary "Top-k
+ * Gating"), after a memset of out has cleared the rows of tokens a capacity
+ * limit dropped ("Expert Capacity"); the result is bit-identical to the
+ * combine.  The layer's kernels after the first are launched with
+ * programmatic stream serialization (each waits for the one before it before
+ * touching memory), so they order like ordinary launches on `stream`.
  *   out [T, d] bf16 out.  expert_idx/gate/r/counts/prob_mean: optional copies
  *   of the routing results (NULL to skip), shapes as in moe_route /
  *   moe_dispatch; stats [4]: optional router metrics (moe_router_stats). */
