@@ -279,6 +279,25 @@ MOE_API moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x,
                            int32_t* expert_idx, float* gate, float* r, int32_t* counts,
                            float* prob_mean, float* stats, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_layer_fwd with the row gather fused into GEMM 1's A-operand load (CODA
+ * thread: r travels with the dispatched token into the first expert linear;
+ * OmniMoE, section 2.2: tasks grouped by expert into a grouped GEMM).  No
+ * permuted copy of x is made: the router also writes xg = bf16(x * gamma) in
+ * token order into the workspace, and GEMM 1's producer gathers each A tile
+ * from it, row p = token perm[p] / k, with four-row TMA gathers
+ * (tile::gather4) -- rows bit-identical to moe_dispatch's x_perm, so out is
+ * bit-identical to moe_layer_fwd.  It saves the permuted copy's write and
+ * read (2 * T*k * d * 2 bytes per call) but on B200 runs slower than
+ * moe_layer_fwd: each four-row gather costs the SM's copy engine about as
+ * much as a whole 128-row tile load, which leaves GEMM 1 load-bound.  Same
+ * arguments, workspace and errors as moe_layer_fwd. */
+MOE_API moe_status_t moe_layer_fwd_gather(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
+                                          const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
+                                          const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out,
+                                          int32_t* expert_idx, float* gate, float* r, int32_t* counts,
+                                          float* prob_mean, float* stats, void* ws, size_t ws_bytes,
+                                          void* stream);
+
 /* ---- the layer on HOST buffers: copies in and out pipelined with the compute
  *
  * moe_layer_fwd with x and out in host memory (pinned memory, e.g. from

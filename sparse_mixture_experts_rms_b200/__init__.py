@@ -41,7 +41,7 @@ EXPORTED = ["moe_status_string", "moe_capacity", "moe_max_kept", "moe_workspace_
             "moe_workspace_init", "moe_get_device_error", "moe_set_wait_limit", "moe_route", "moe_dispatch",
             "moe_dispatch_noalloc",
             "moe_experts_fwd", "moe_experts_up", "moe_experts_down", "moe_combine",
-            "moe_layer_fwd", "moe_router_stats", "moe_train_workspace_size", "moe_train_rows",
+            "moe_layer_fwd", "moe_layer_fwd_gather", "moe_router_stats", "moe_train_workspace_size", "moe_train_rows",
             "moe_train_saved", "moe_layer_fwd_train", "moe_layer_bwd",
             "moe_host_workspace_size", "moe_host_chunks", "moe_layer_fwd_host",
             "moe_mx_weights_size", "moe_quantize_weights_mx", "moe_mx_workspace_size", "moe_mx_rows",
@@ -124,6 +124,8 @@ def _lib():
         lib.moe_combine.argtypes = [cfgp, P, P, P, P]
         lib.moe_layer_fwd.restype = ctypes.c_int
         lib.moe_layer_fwd.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.moe_layer_fwd_gather.restype = ctypes.c_int
+        lib.moe_layer_fwd_gather.argtypes = lib.moe_layer_fwd.argtypes
         lib.moe_mx_weights_size.restype = SZ
         lib.moe_mx_weights_size.argtypes = [cfgp]
         lib.moe_quantize_weights_mx.restype = ctypes.c_int
@@ -408,10 +410,13 @@ def moe_combine(cfg: MoEConfig, y, inv_perm, out, stream=None) -> None:
 
 def moe_layer_fwd(cfg: MoEConfig, x, gamma, Wr, bias, W1, W3, W2, out, ws: torch.Tensor,
                   expert_idx=None, gate=None, r=None, counts=None, prob_mean=None, stats=None,
-                  stream=None) -> None:
+                  stream=None, gather: bool = False) -> None:
+    """The layer; with `gather`, through moe_layer_fwd_gather (the row gather in
+    GEMM 1's A load instead of a permuted copy of x)."""
     T, d, E, k, F = cfg.T, cfg.d_model, cfg.E, cfg.k, cfg.F
     bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
-    st = _lib().moe_layer_fwd(
+    name = "moe_layer_fwd_gather" if gather else "moe_layer_fwd"
+    st = getattr(_lib(), name)(
         ctypes.byref(cfg.c()), _ptr(x, "x", bf, (T, d)), _ptr(gamma, "gamma", bf, (d,)),
         _ptr(Wr, "Wr", bf, (d, E)), _ptr(bias, "bias", f32, (E,)), _ptr(W1, "W1", bf, (d, F)),
         _ptr(W3, "W3", bf, (d, F)), _ptr(W2, "W2", bf, (F, d)), _ptr(out, "out", bf, (T, d)),
@@ -419,7 +424,7 @@ def moe_layer_fwd(cfg: MoEConfig, x, gamma, Wr, bias, W1, W3, W2, out, ws: torch
         _ptr(r, "r", f32, (T,)), _ptr(counts, "counts", i32, (E,)),
         _ptr(prob_mean, "prob_mean", f32, (E,)), _ptr(stats, "stats", f32, (4,)),
         _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream))
-    _check(st, "moe_layer_fwd")
+    _check(st, name)
 
 
 # ------------------------------------------------------------------ MXFP8 expert GEMMs

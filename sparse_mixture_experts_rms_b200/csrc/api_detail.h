@@ -71,7 +71,8 @@ bool make_map_sfp(CUtensorMap* m, const void* base, uint64_t nregions);
 // The layer's stages on one stream (cfg validated, pointers checked).
 moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf16_t* gamma,
                        const moe_bf16_t* Wr, const float* bias, int32_t* idx, float* gate, float* r,
-                       float* logits, float* prob_mean, const Layout& L, void* ws, cudaStream_t s);
+                       float* logits, float* prob_mean, const Layout& L, void* ws, cudaStream_t s,
+                       moe_bf16_t* xg = nullptr);
 moe_status_t run_dispatch(const moe_config_t& c, const Layout& L, void* ws, const int32_t* idx,
                           const moe_bf16_t* x, const moe_bf16_t* gamma, int32_t* counts,
                           int32_t* offsets, int32_t* perm, int32_t* inv_perm, moe_bf16_t* x_perm,
@@ -82,7 +83,7 @@ void fill_gemm_common(GemmArgs& g, const moe_config_t& c, const Layout& L, void*
 moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x_perm,
                     const float* r, const int32_t* perm, const int32_t* offsets,
                     const moe_bf16_t* W1, const moe_bf16_t* W3, int sms, cudaStream_t s,
-                    moe_bf16_t* U = nullptr, moe_bf16_t* V = nullptr);
+                    moe_bf16_t* U = nullptr, moe_bf16_t* V = nullptr, bool gather = false);
 moe_status_t run_down(const moe_config_t& c, const Layout& L, void* ws, const float* gate,
                       const int32_t* perm, const int32_t* offsets, const moe_bf16_t* W2,
                       moe_bf16_t* y, int sms, cudaStream_t s, moe_bf16_t* yu = nullptr,
@@ -97,7 +98,7 @@ moe_status_t run_layer(const moe_config_t& c, const Layout& L, void* ws, const m
                        const moe_bf16_t* gamma, const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
                        const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out, int32_t* expert_idx,
                        float* gate, float* r, int32_t* counts, float* prob_mean, float* stats, int sms,
-                       cudaStream_t s);
+                       cudaStream_t s, bool gather = false);
 
 }  // namespace api
 }  // namespace moe

@@ -601,7 +601,7 @@ __device__ __forceinline__ void epilogue_wgrad(const GemmArgs& a, const GemmShar
   }
 }
 
-template <int MODE, int EPI>
+template <int MODE, int EPI, int AG = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                         const __grid_constant__ CUtensorMap mapB0, const __grid_constant__ CUtensorMap mapB1,
@@ -704,7 +704,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
   const uint64_t wait_ns = wait_limit_ns(a.wait_ctl);
   const uint32_t peer_abort = map_to_cta(smem_addr(&sh.abort_flag), rank ^ 1u);
 
-  if (warp == 0) {
+  static_assert(MODE == kGemmUp || !AG, "the row gather feeds the up GEMM only");
+  if (AG && warp == 0) {
+    // ================= TMA producer, row gather (the whole warp): A rows are
+    // the tokens' rows of xg = x * gamma [T, d] (mapA0, one-row box), row p
+    // of the tile being token perm[p] / k.  Lane l gathers the CTA's rows
+    // 4l .. 4l+3 with one four-row gather per K block; lane 0 waits for the
+    // stage, arms the leader's barrier and loads the stage's B.
+    const uint32_t full_leader0 = map_to_cta(smem_addr(&sh.full[0]), 0);
+    const uint32_t tx_pair = 2u * (kABytes + static_cast<uint32_t>(a.bn / 2) * BK * 2u);
+    const int kept = sh.seg[E];
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = pair; ok && tile < total; tile += npairs) {
+      const TileCoord c = decode_tile(sh, E, tile);
+      const int o_e = a.ffn.off[c.e];
+      const int kblocks = sh.k_blocks[c.e];
+      // rows past the last kept row (their results are discarded) read token 0
+      const int p0 = sh.seg[c.e] + c.mt * BM + static_cast<int>(rank) * BM_CTA + 4 * lane;
+      int tok[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int asg = p0 + j < kept ? a.perm[p0 + j] : -1;
+        tok[j] = asg >= 0 ? asg / a.k : 0;
+      }
+      for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1u;
+        int got = 1;
+        if (lane == 0)
+          got = mbar_wait(&sh.empty[s], ph ^ 1u, abort_flag, a.err, MOE_DEVERR_TIMEOUT, wait_ns, false, peer_abort)
+                    ? 1 : 0;
+        if (!__shfl_sync(0xFFFFFFFFu, got, 0)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sA = smem + s * kStageBytes;
+        const uint32_t bar = full_leader0 + static_cast<uint32_t>(s) * 8u;
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive_expect_tx(&sh.full[s], tx_pair);
+          // leader: 128 columns of W1; peer: the same 128 columns of W3 (MN-major)
+          const CUtensorMap* mB = rank == 0 ? maps.b0 : maps.b1;
+          const int n0 = o_e + c.nt * kBlockN;
+          tma_load_2d_pair(sA + kABytes, mB, bar, n0, kb * BK);
+          tma_load_2d_pair(sA + kABytes + kAtomBytes, mB, bar, n0 + 64, kb * BK);
+        }
+        tma_gather4_pair(sA + lane * 4 * 128, maps.a0, bar, kb * BK, tok[0], tok[1], tok[2], tok[3]);
+      }
+    }
+    // no copy into either CTA is in flight when it exits, whatever stopped the loop
+    if (lane == 0) pair_producer_drain<kStages>(sh.pd, sh.full, it, rank, tx_pair / 2u, a.err);
+  } else if (warp == 0) {
     // ================= TMA producer (one lane per CTA)
     if (lane == 0) {
       const uint32_t full_leader0 = map_to_cta(smem_addr(&sh.full[0]), 0);
@@ -832,9 +882,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(EPI), 1)
   if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
 }
 
-template <int MODE, int EPI = 4>
+template <int MODE, int EPI = 4, int AG = 0>
 cudaError_t set_smem_attr() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<MODE, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(grouped_gemm_kernel<MODE, EPI, AG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(kSmemBytes));
 }
 
@@ -851,6 +901,8 @@ cudaError_t prepare_grouped_gemm() {
   if (e == cudaSuccess) e = set_smem_attr<kGemmWgradH>();
   if (e == cudaSuccess) e = set_smem_attr<kGemmUp, 8>();
   if (e == cudaSuccess) e = set_smem_attr<kGemmDown, 8>();
+  if (e == cudaSuccess) e = set_smem_attr<kGemmUp, 4, 1>();
+  if (e == cudaSuccess) e = set_smem_attr<kGemmUp, 8, 1>();
   return e;
 }
 
@@ -879,12 +931,17 @@ cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& mapA0, con
   static const EpiMaps kNoMaps{};
   const EpiMaps& em = em_opt != nullptr ? *em_opt : kNoMaps;
   if (a.epi8 && a.mode != kGemmUp && a.mode != kGemmDown) return cudaErrorInvalidValue;
+  if (a.gather && a.mode != kGemmUp) return cudaErrorInvalidValue;
   GemmArgs ga = a;
   ga.staged = em_opt != nullptr ? 1 : 0;
   cudaError_t e = cudaSuccess;
   switch (a.mode) {
     case kGemmUp:
-      if (ga.epi8)
+      if (ga.gather && ga.epi8)
+        e = launch_pdl(grouped_gemm_kernel<kGemmUp, 8, 1>, dim3(grid), dim3(threads_of(8)), kSmemBytes, s, mapA0, mapA1, mapB0, mapB1, ga, em);
+      else if (ga.gather)
+        e = launch_pdl(grouped_gemm_kernel<kGemmUp, 4, 1>, dim3(grid), dim3(kThreads), kSmemBytes, s, mapA0, mapA1, mapB0, mapB1, ga, em);
+      else if (ga.epi8)
         e = launch_pdl(grouped_gemm_kernel<kGemmUp, 8>, dim3(grid), dim3(threads_of(8)), kSmemBytes, s, mapA0, mapA1, mapB0, mapB1, ga, em);
       else
         e = launch_pdl(grouped_gemm_kernel<kGemmUp, 4>, dim3(grid), dim3(kThreads), kSmemBytes, s, mapA0, mapA1, mapB0, mapB1, ga, em);

@@ -104,7 +104,8 @@ Layout layout_of(const moe_config_t& c, bool train, bool mx) {
     L.h8 = take(mk * static_cast<size_t>(fmax));
     L.hsf = take((mk / 128) * (static_cast<size_t>(fmax) / 128) * 512);
   } else {
-    L.x_perm = take(mk * c.d_model * 2);
+    // x_perm, or the gathering layer's xg [T, d] (token order) in the same buffer
+    L.x_perm = take(std::max<size_t>(mk, static_cast<size_t>(c.T)) * c.d_model * 2);
     L.H = take(mk * static_cast<size_t>(fmax) * 2);
   }
   L.y = take(mk * c.d_model * 2);
@@ -267,7 +268,8 @@ moe_status_t cuda_status(cudaError_t e) {
 
 moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf16_t* gamma,
                        const moe_bf16_t* Wr, const float* bias, int32_t* idx, float* gate, float* r,
-                       float* logits, float* prob_mean, const Layout& L, void* ws, cudaStream_t s) {
+                       float* logits, float* prob_mean, const Layout& L, void* ws, cudaStream_t s,
+                       moe_bf16_t* xg) {
   if (c.T == 0) return MOE_OK;
   RouteArgs a{};
   a.wprime = at<__nv_bfloat16>(ws, L.rw);
@@ -294,14 +296,15 @@ moe_status_t run_route(const moe_config_t& c, const moe_bf16_t* x, const moe_bf1
   a.k = c.k;
   a.eps = c.eps;
   a.renormalize = c.renormalize ? 1 : 0;
-  CUtensorMap xmap, wmap;
-  // x [T, d]: tiles of 128 tokens x 64 elements; the router's hi/lo B [2 EP, d]: 2 EP x 64
+  CUtensorMap xmap, wmap, xgmap;
+  // x [T, d]: tiles of 128 tokens x 64 elements; the router's hi/lo B [2 EP, d]: 2 EP x 64;
+  // xg [T, d] (optional): 32-token boxes, one per epilogue lane quarter
   const uint32_t ep2 = static_cast<uint32_t>(2 * route_padded_experts(c.E));
-  if (!make_map(&xmap, x, static_cast<uint64_t>(c.d_model), static_cast<uint64_t>(c.T),
-                static_cast<uint64_t>(c.d_model), 64, kRouteTok) ||
-      !make_map(&wmap, a.wprime, static_cast<uint64_t>(c.d_model), ep2, static_cast<uint64_t>(c.d_model), 64, ep2))
+  const uint64_t d = static_cast<uint64_t>(c.d_model), T = static_cast<uint64_t>(c.T);
+  if (!make_map(&xmap, x, d, T, d, 64, kRouteTok) || !make_map(&wmap, a.wprime, d, ep2, d, 64, ep2) ||
+      (xg != nullptr && !make_map(&xgmap, xg, d, T, d, 64, 32)))
     return MOE_ERR_CUDA;
-  return cuda_status(launch_route(a, xmap, wmap, s));
+  return cuda_status(launch_route(a, xmap, wmap, xg != nullptr ? &xgmap : nullptr, s));
 }
 
 moe_status_t run_dispatch(const moe_config_t& c, const Layout& L, void* ws, const int32_t* idx,
@@ -357,7 +360,7 @@ void fill_gemm_common(GemmArgs& g, const moe_config_t& c, const Layout& L, void*
 moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_bf16_t* x_perm,
                     const float* r, const int32_t* perm, const int32_t* offsets,
                     const moe_bf16_t* W1, const moe_bf16_t* W3, int sms, cudaStream_t s,
-                    moe_bf16_t* U, moe_bf16_t* V) {
+                    moe_bf16_t* U, moe_bf16_t* V, bool gather) {
   if (L.max_kept == 0) return MOE_OK;
   const uint64_t rows = static_cast<uint64_t>(L.max_kept);
   const uint64_t d = static_cast<uint64_t>(c.d_model);
@@ -365,10 +368,14 @@ moe_status_t run_up(const moe_config_t& c, const Layout& L, void* ws, const moe_
   GemmArgs g{};
   fill_gemm_common(g, c, L, ws, perm, offsets);
   CUtensorMap mA, mB0, mB1;
-  if (!make_map(&mA, x_perm, d, rows, d, 64, 128) || !make_map(&mB0, W1, F, d, F, 64, 64) ||
+  // A: x_perm [rows, d] in 128-row boxes, or (gather) xg [T, d] in one-row boxes, row p = token perm[p] / k
+  const bool a_ok = gather ? make_map(&mA, x_perm, d, static_cast<uint64_t>(c.T), d, 64, 1)
+                           : make_map(&mA, x_perm, d, rows, d, 64, 128);
+  if (!a_ok || !make_map(&mB0, W1, F, d, F, 64, 64) ||
       !make_map(&mB1, W3, F, d, F, 64, 64))
     return MOE_ERR_CUDA;
   g.mode = kGemmUp;
+  g.gather = gather ? 1 : 0;
   g.bn = 2 * kBlockN;
   g.scale = r;
   g.out = at<__nv_bfloat16>(ws, L.H);
@@ -480,7 +487,7 @@ moe_status_t run_layer(const moe_config_t& c, const Layout& L, void* ws, const m
                        const moe_bf16_t* gamma, const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
                        const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out, int32_t* expert_idx,
                        float* gate, float* r, int32_t* counts, float* prob_mean, float* stats, int sms,
-                       cudaStream_t s) {
+                       cudaStream_t s, bool gather) {
   moe_status_t st;
   int32_t* idx_ = expert_idx ? expert_idx : at<int32_t>(ws, L.idx);
   float* gate_ = gate ? gate : at<float>(ws, L.gate);
@@ -502,10 +509,17 @@ moe_status_t run_layer(const moe_config_t& c, const Layout& L, void* ws, const m
     cudaError_t e = cudaMemsetAsync(out, 0, static_cast<size_t>(c.T) * c.d_model * sizeof(moe_bf16_t), s);
     if (e != cudaSuccess) return cuda_status(e);
   }
-  if ((st = run_route(c, x, gamma, Wr, bias, idx_, gate_, r_, nullptr, pm, L, ws, s)) != MOE_OK) return st;
-  if ((st = run_dispatch(c, L, ws, idx_, x, gamma, counts_, offsets, perm, inv_perm, x_perm, sms, s)) != MOE_OK)
+  // gather: the router also writes xg = bf16(x * gamma) in token order (into
+  // the x_perm buffer, which holds T rows), no permuted copy is made, and the
+  // up GEMM gathers its A rows from xg by perm as it loads them
+  if ((st = run_route(c, x, gamma, Wr, bias, idx_, gate_, r_, nullptr, pm, L, ws, s, gather ? x_perm : nullptr)) !=
+      MOE_OK)
     return st;
-  if ((st = run_up(c, L, ws, x_perm, r_, perm, offsets, W1, W3, sms, s)) != MOE_OK) return st;
+  if ((st = run_dispatch(c, L, ws, idx_, x, gamma, counts_, offsets, perm, inv_perm, gather ? nullptr : x_perm, sms,
+                         s)) != MOE_OK)
+    return st;
+  if ((st = run_up(c, L, ws, x_perm, r_, perm, offsets, W1, W3, sms, s, nullptr, nullptr, gather)) != MOE_OK)
+    return st;
   if ((st = run_down(c, L, ws, gate_, perm, offsets, W2, direct ? out : y, sms, s, nullptr, direct)) != MOE_OK)
     return st;
   if (!direct && (st = run_combine(c, y, inv_perm, out, sms, s)) != MOE_OK) return st;
@@ -519,6 +533,37 @@ moe_status_t run_layer(const moe_config_t& c, const Layout& L, void* ws, const m
 
 using namespace moe;
 using namespace moe::api;
+
+namespace {
+// moe_layer_fwd and moe_layer_fwd_gather: argument checks, then the layer.
+moe_status_t layer_fwd_entry(bool gather, const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
+                             const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1, const moe_bf16_t* W3,
+                             const moe_bf16_t* W2, moe_bf16_t* out, int32_t* expert_idx, float* gate, float* r,
+                             int32_t* counts, float* prob_mean, float* stats, void* ws, size_t ws_bytes,
+                             void* stream) {
+  moe_status_t st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) {  // no tokens: only the optional counts are written (zeros)
+    if (counts == nullptr) return MOE_OK;
+    if (!aligned(counts, 4)) return MOE_ERR_ALIGNMENT;
+    int sms;
+    if ((st = device_ready(&sms)) != MOE_OK) return st;
+    return cuda_status(cudaMemsetAsync(counts, 0, cfg->E * sizeof(int32_t), static_cast<cudaStream_t>(stream)));
+  }
+  if (!aligned(prob_mean, 4) || !aligned(stats, 4)) return MOE_ERR_ALIGNMENT;
+  if (!x || !gamma || !Wr || !W1 || !W3 || !W2 || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) ||
+      !aligned(W1, 16) || !aligned(W3, 16) || !aligned(W2, 16) || !aligned(out, 16) ||
+      !aligned(expert_idx, 4) || !aligned(gate, 4) || !aligned(r, 4) || !aligned(counts, 4))
+    return MOE_ERR_ALIGNMENT;
+  Layout L;
+  if ((st = check_ws(*cfg, ws, ws_bytes, &L)) != MOE_OK) return st;
+  int sms;
+  if ((st = device_ready(&sms)) != MOE_OK) return st;
+  return run_layer(*cfg, L, ws, x, gamma, Wr, bias, W1, W3, W2, out, expert_idx, gate, r, counts, prob_mean,
+                   stats, sms, static_cast<cudaStream_t>(stream), gather);
+}
+}  // namespace
 
 extern "C" {
 
@@ -763,27 +808,17 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_bf16_t* x, const m
                            const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out,
                            int32_t* expert_idx, float* gate, float* r, int32_t* counts,
                            float* prob_mean, float* stats, void* ws, size_t ws_bytes, void* stream) {
-  moe_status_t st = validate(cfg);
-  if (st != MOE_OK) return st;
-  if (cfg->T == 0) {  // no tokens: only the optional counts are written (zeros)
-    if (counts == nullptr) return MOE_OK;
-    if (!aligned(counts, 4)) return MOE_ERR_ALIGNMENT;
-    int sms;
-    if ((st = device_ready(&sms)) != MOE_OK) return st;
-    return cuda_status(cudaMemsetAsync(counts, 0, cfg->E * sizeof(int32_t), static_cast<cudaStream_t>(stream)));
-  }
-  if (!aligned(prob_mean, 4) || !aligned(stats, 4)) return MOE_ERR_ALIGNMENT;
-  if (!x || !gamma || !Wr || !W1 || !W3 || !W2 || !out) return MOE_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(gamma, 16) || !aligned(Wr, 2) || !aligned(bias, 4) ||
-      !aligned(W1, 16) || !aligned(W3, 16) || !aligned(W2, 16) || !aligned(out, 16) ||
-      !aligned(expert_idx, 4) || !aligned(gate, 4) || !aligned(r, 4) || !aligned(counts, 4))
-    return MOE_ERR_ALIGNMENT;
-  Layout L;
-  if ((st = check_ws(*cfg, ws, ws_bytes, &L)) != MOE_OK) return st;
-  int sms;
-  if ((st = device_ready(&sms)) != MOE_OK) return st;
-  return run_layer(*cfg, L, ws, x, gamma, Wr, bias, W1, W3, W2, out, expert_idx, gate, r, counts, prob_mean,
-                   stats, sms, static_cast<cudaStream_t>(stream));
+  return layer_fwd_entry(false, cfg, x, gamma, Wr, bias, W1, W3, W2, out, expert_idx, gate, r, counts, prob_mean,
+                         stats, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_layer_fwd_gather(const moe_config_t* cfg, const moe_bf16_t* x, const moe_bf16_t* gamma,
+                                  const moe_bf16_t* Wr, const float* bias, const moe_bf16_t* W1,
+                                  const moe_bf16_t* W3, const moe_bf16_t* W2, moe_bf16_t* out,
+                                  int32_t* expert_idx, float* gate, float* r, int32_t* counts,
+                                  float* prob_mean, float* stats, void* ws, size_t ws_bytes, void* stream) {
+  return layer_fwd_entry(true, cfg, x, gamma, Wr, bias, W1, W3, W2, out, expert_idx, gate, r, counts, prob_mean,
+                         stats, ws, ws_bytes, stream);
 }
 
 moe_status_t moe_router_stats(const moe_config_t* cfg, const float* prob_mean, const int32_t* counts,

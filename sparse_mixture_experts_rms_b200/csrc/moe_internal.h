@@ -181,6 +181,7 @@ struct GemmArgs {
   int to_token;             // down, k = 1: row p goes to row perm[p] (its token) of out [T, d]
   int staged;               // set by the launcher: epilogue tensor maps were given
   int epi8;                 // up / down: 8 epilogue warps (short reductions)
+  int gather;               // up: A rows gathered from xg [T, d] (mapA0, one-row box) by perm[p] / k
 };
 
 struct CombineArgs {
@@ -239,7 +240,10 @@ constexpr int kEpi8MaxK = 1024;
 // Launchers (return the launch error, if any).
 // xmap: x [T, d], boxes of 64 x 128 tokens; wmap: the [2 EP, d] hi/lo scratch,
 // boxes of 64 x 2 EP (both 128-byte swizzled).
-cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, const CUtensorMap& wmap, cudaStream_t s);
+// With `xgmap` (may be null; box 64 x 32, 128-byte swizzle over a [T, d] bf16
+// buffer) the router also writes xg = bf16(x * gamma) in token order.
+cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, const CUtensorMap& wmap,
+                         const CUtensorMap* xgmap, cudaStream_t s);
 int route_padded_experts(int E);  // EP: E rounded up to 8, 16, 32 or 64
 cudaError_t launch_dispatch(const DispatchArgs& a, int num_sms, cudaStream_t s);
 // Tensor maps of the epilogues that move their bf16 rows through shared

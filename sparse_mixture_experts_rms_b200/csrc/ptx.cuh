@@ -207,6 +207,20 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// Row gather of a 2-CTA pair: rows r0..r3 (outer coordinates) of a 2-D map
+// whose box is one row high, columns from c0 (box-wide), land as four
+// consecutive box rows at `dst` in this CTA (swizzled by their shared-memory
+// address, like the rows of a tiled box there), completing on the mbarrier at
+// `bar_cluster` (the pair leader's).
+__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int32_t c0, int32_t r0, int32_t r1, int32_t r2, int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
 // Untiled bulk copy global -> this CTA's shared memory (16-byte aligned
 // addresses, size a multiple of 16), completing on `bar` with complete_tx.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

@@ -72,6 +72,7 @@ struct __align__(8) RouteShared {
   uint64_t tfull[kGroups];     // a stage's chunk partials are in the TMEM buffer group
   uint64_t tempty[kGroups];    // the epilogue read the group
   uint64_t drain;
+  uint64_t xg_ready[4];        // with xg and 8 epilogue warps: both warps of a lane quarter rewrote their pieces
   uint32_t tmem_base;
   int abort_flag;
   uint32_t dummy_err;
@@ -151,10 +152,10 @@ template <int EP>
 __device__ __forceinline__ void route_token(const RouteArgs& a, float* lg, float rtok, int t,
                                             bool keep_probs);
 
-template <int EP>
+template <int EP, bool XG>
 __global__ void __launch_bounds__(RouteCfg<EP>::kThreads, 1)
     route_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap wmap,
-                 const RouteArgs a) {
+                 const __grid_constant__ CUtensorMap xgmap, const RouteArgs a) {
   using Cfg = RouteCfg<EP>;
   constexpr int N = Cfg::N;
   constexpr int EPI = Cfg::kEpi;
@@ -179,11 +180,13 @@ __global__ void __launch_bounds__(RouteCfg<EP>::kThreads, 1)
       mbar_init(&sh.tempty[g], EPI);
     }
     mbar_init(&sh.drain, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&sh.xg_ready[i], 2);
     sh.abort_flag = 0;
     sh.dummy_err = 0;
     fence_mbar_init();
     tma_prefetch_map(&xmap);
     tma_prefetch_map(&wmap);
+    if (XG) tma_prefetch_map(&xgmap);
   }
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, Cfg::kTmemCols);
@@ -307,15 +310,66 @@ __global__ void __launch_bounds__(RouteCfg<EP>::kThreads, 1)
       for (int e = 0; e < NE; ++e) acc[e] += static_cast<double>(stage_sum[e]);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sh.tempty[g]);
-        mbar_arrive(&sh.empty[s]);
+      if (lane == 0) mbar_arrive(&sh.tempty[g]);
+      if constexpr (XG) {
+        // The stage's MMAs are complete (tfull), so its x tiles may change:
+        // this thread's pieces become bf16(x * gamma) in place, and one warp
+        // of the lane quarter stores the quarter's 32 rows of every chunk to
+        // xg by TMA before the stage goes back to the producer.
+        uint8_t* xs = ring + s * Cfg::kStageBytes;
+        const uint4* g4 = reinterpret_cast<const uint4*>(a.gamma);
+        for (int i = 0; i < nc; ++i) {
+          uint8_t* xr = xs + i * kTileBytes + row * 128;
+          const int kx8 = (st * CPS + i) * (kChunk / 8);
+#pragma unroll
+          for (int j = 0; j < NJ; ++j) {
+            const int jj = half * NJ + j;
+            uint4* pv = reinterpret_cast<uint4*>(xr + ((jj ^ (row & 7)) << 4));
+            const uint4 v = *pv, gv = __ldg(g4 + kx8 + jj);
+            const uint32_t xw[4] = {v.x, v.y, v.z, v.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float lo = __uint_as_float(xw[u] << 16) * __uint_as_float(gw[u] << 16);
+              const float hi = __uint_as_float(xw[u] & 0xFFFF0000u) * __uint_as_float(gw[u] & 0xFFFF0000u);
+              const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+              o[u] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            *pv = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        bool stored = true;
+        if (EPI == 8) {
+          // the other warp of the quarter holds the rest of each row
+          if (lane == 0) mbar_arrive(&sh.xg_ready[q]);
+          if (half == 0) {
+            int got = 1;
+            if (lane == 0)
+              got = mbar_wait(&sh.xg_ready[q], st & 1u, abort_flag, err, MOE_DEVERR_TIMEOUT, wait_ns) ? 1 : 0;
+            stored = __shfl_sync(0xFFFFFFFFu, got, 0) != 0;
+          }
+        }
+        if (stored && half == 0 && lane == 0 && t0 + q * 32 < a.T) {
+          for (int i = 0; i < nc; ++i)
+            tma_store_2d(&xgmap, xs + i * kTileBytes + q * 32 * 128, (st * CPS + i) * kChunk, t0 + q * 32);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+        __syncwarp();
+        if (!stored) {
+          ok = false;
+          break;
+        }
       }
+      if (lane == 0) mbar_arrive(&sh.empty[s]);
       float sqs = 0.f;
 #pragma unroll
       for (int j = 0; j < CPS * NJ; ++j) sqs += sq[j];
       ss += static_cast<double>(sqs);
     }
+    if (XG && half == 0 && lane == 0) bulk_wait_group0();  // xg written before the kernel ends
   }
   ok = __syncthreads_and(ok && !*abort_flag) != 0;
   if (warp == 1) {
@@ -431,14 +485,15 @@ __device__ __forceinline__ void route_token(const RouteArgs& a, float* lg, float
   }
 }
 
-template <int EP>
-cudaError_t launch_route_t(const RouteArgs& a, const CUtensorMap& xmap, const CUtensorMap& wmap, cudaStream_t s) {
+template <int EP, bool XG>
+cudaError_t launch_route_t(const RouteArgs& a, const CUtensorMap& xmap, const CUtensorMap& wmap,
+                           const CUtensorMap& xgmap, cudaStream_t s) {
   const size_t smem = RouteCfg<EP>::kSmem;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(route_kernel<EP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(route_kernel<EP, XG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
@@ -446,7 +501,7 @@ cudaError_t launch_route_t(const RouteArgs& a, const CUtensorMap& xmap, const CU
   const int n = 2 * EP * a.d;
   router_weight_kernel<<<(n + 255) / 256, 256, 0, s>>>(a, EP);
   const int grid = (a.T + kTok - 1) / kTok;
-  return launch_pdl(route_kernel<EP>, dim3(grid), dim3(RouteCfg<EP>::kThreads), smem, s, xmap, wmap, a);
+  return launch_pdl(route_kernel<EP, XG>, dim3(grid), dim3(RouteCfg<EP>::kThreads), smem, s, xmap, wmap, xgmap, a);
 }
 
 // Load-balance metrics from the router's prob_mean and the dispatch counts:
@@ -494,13 +549,22 @@ cudaError_t launch_router_stats(const float* prob_mean, const int32_t* counts, c
 
 int route_padded_experts(int E) { return E <= 8 ? 8 : (E <= 16 ? 16 : (E <= 32 ? 32 : 64)); }
 
-cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, const CUtensorMap& wmap, cudaStream_t s) {
+cudaError_t launch_route(const RouteArgs& a, const CUtensorMap& xmap, const CUtensorMap& wmap,
+                         const CUtensorMap* xgmap, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
+  if (xgmap != nullptr) {
+    switch (route_padded_experts(a.E)) {
+      case 8: return launch_route_t<8, true>(a, xmap, wmap, *xgmap, s);
+      case 16: return launch_route_t<16, true>(a, xmap, wmap, *xgmap, s);
+      case 32: return launch_route_t<32, true>(a, xmap, wmap, *xgmap, s);
+      default: return launch_route_t<64, true>(a, xmap, wmap, *xgmap, s);
+    }
+  }
   switch (route_padded_experts(a.E)) {
-    case 8: return launch_route_t<8>(a, xmap, wmap, s);
-    case 16: return launch_route_t<16>(a, xmap, wmap, s);
-    case 32: return launch_route_t<32>(a, xmap, wmap, s);
-    default: return launch_route_t<64>(a, xmap, wmap, s);
+    case 8: return launch_route_t<8, false>(a, xmap, wmap, xmap, s);
+    case 16: return launch_route_t<16, false>(a, xmap, wmap, xmap, s);
+    case 32: return launch_route_t<32, false>(a, xmap, wmap, xmap, s);
+    default: return launch_route_t<64, false>(a, xmap, wmap, xmap, s);
   }
 }
 
