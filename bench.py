@@ -80,6 +80,8 @@ def parse_args():
                     help="skip the MXFP8 leg (the layer with block-scaled E4M3 expert GEMMs)")
     ap.add_argument("--no-train", action="store_true",
                     help="skip the training leg (forward with saved state + backward)")
+    ap.add_argument("--no-gather", action="store_true",
+                    help="skip the leg timing moe_layer_fwd_gather (the row gather in the up GEMM's A load)")
     ap.add_argument("--no-others", action="store_true",
                     help="skip the other workload configurations (tiny, switch_capacity, variable_size, "
                          "fine_grained) timed after the main line")
@@ -283,6 +285,39 @@ def dispatch_scale_leg(moe, steps: int = 20):
     res["device_error"] = moe.moe_get_device_error(ws, raise_on_error=False)
     res["counts_sum_ok"] = int(o["counts"].sum().item()) == T * k
     del ws, o, idx, x
+    torch.cuda.empty_cache()
+    return res
+
+
+def gather_leg(moe, cfg, w, x, gamma, Wr, bias, W1, W3, W2, out_ref, stream, ms_layer, barrier, world):
+    """moe_layer_fwd_gather on the main workload: 5 steps after 3 warm-ups,
+    CUDA events on the launching stream, max over ranks; its output against
+    the main line's last output (the same inputs) bit for bit."""
+    import torch
+    ws = moe.alloc_workspace(cfg)
+    out = torch.empty_like(out_ref)
+    step = lambda: moe.moe_layer_fwd(cfg, x, gamma, Wr, bias, W1, W3, W2, out, ws, stream=stream, gather=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+    stream.synchronize()
+    n = 5
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    stream.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda") / n
+    res = {"call": "moe_layer_fwd_gather", "ms_per_step": ms, "tokens_per_s": world * w.T / (ms * 1e-3),
+           "vs_layer": ms / ms_layer, "bit_identical_to_layer": bool(torch.equal(out, out_ref)), "steps": n,
+           "device_error": moe.moe_get_device_error(ws, stream=stream, raise_on_error=False),
+           "note": "row gather fused into the up GEMM's A load (tile::gather4); slower on B200: "
+                   "each four-row gather costs the copy engine about as much as a 128-row tile load"}
+    del ws
     torch.cuda.empty_cache()
     return res
 
@@ -577,6 +612,13 @@ def run_ours(args, rank, world, local):
         train = train_leg(moe, cfg, w, x, gamma, Wr, bias, W1, W3, W2, stream, args.steps, nf, sampler,
                           barrier, world)
 
+    # ---- the same layer through moe_layer_fwd_gather (no permuted copy of x;
+    # the up GEMM gathers its A rows by TMA): timed like the main line, its
+    # output compared bit for bit with the main line's
+    gather = None
+    if not args.no_gather:
+        gather = gather_leg(moe, cfg, w, x, gamma, Wr, bias, W1, W3, W2, out, stream, ms_step, barrier, world)
+
     # ---- the other workload configurations, each timed alone after the main line
     others = None
     if not args.no_others and args.tokens == 0:
@@ -645,6 +687,8 @@ def run_ours(args, rank, world, local):
         result["train"] = train
     if mx is not None:
         result["mx"] = mx
+    if gather is not None:
+        result["gather"] = gather
     if others is not None:
         result["other_workloads"] = others
     if dscale is not None:
