@@ -109,8 +109,9 @@ MOE_API int64_t moe_max_kept(const moe_config_t* cfg);
 /* Bytes of workspace every entry point below needs for `cfg` (0 if cfg is
  * invalid).  One workspace of this size serves all calls; it holds the device
  * error word, the dispatch scratch and, for moe_layer_fwd, every
- * intermediate (routing, permutation, permuted activations, the SwiGLU
- * activations H and the per-assignment expert outputs). */
+ * intermediate (routing, permutation, permuted activations -- or, for
+ * moe_layer_fwd_gather, x * gamma in token order in the same buffer -- the
+ * SwiGLU activations H and the per-assignment expert outputs). */
 MOE_API size_t moe_workspace_size(const moe_config_t* cfg);
 
 /* Zero the workspace header (the device error word and the wait limit, which
