@@ -95,37 +95,40 @@ def test_too_many_experts_unsupported(lib):
     assert moe.moe_workspace_size(c) == 0
 
 
-def _call_layer(lib, cfg, ptrs, ws_ptr, ws_bytes):
+def _call_layer(lib, cfg, ptrs, ws_ptr, ws_bytes, entry="moe_layer_fwd"):
     P = ctypes.c_void_p
-    return lib.moe_layer_fwd(ctypes.byref(cfg.c()), *[P(p) for p in ptrs], P(0), P(0), P(0), P(0),
-                             P(0), P(0), P(ws_ptr), ws_bytes, P(0))
+    return getattr(lib, entry)(ctypes.byref(cfg.c()), *[P(p) for p in ptrs], P(0), P(0), P(0), P(0),
+                               P(0), P(0), P(ws_ptr), ws_bytes, P(0))
 
 
-def test_layer_argument_errors_before_any_device_work(lib):
+@pytest.mark.parametrize("entry", ["moe_layer_fwd", "moe_layer_fwd_gather"])
+def test_layer_argument_errors_before_any_device_work(lib, entry):
+    _call = lambda *a: _call_layer(*a, entry=entry)
     c = _cfg(mw.WORKLOADS["tiny"])
     good = [4096 * (i + 1) for i in range(8)]   # fake, aligned, never dereferenced
     wsz = moe.moe_workspace_size(c)
     # null tensor
     bad = list(good); bad[0] = 0
-    assert _call_layer(lib, c, bad, 1 << 20, wsz) == moe.MOE_ERR_INVALID_ARG
+    assert _call(lib, c, bad, 1 << 20, wsz) == moe.MOE_ERR_INVALID_ARG
     # misaligned bf16 matrix
     bad = list(good); bad[4] += 8
-    assert _call_layer(lib, c, bad, 1 << 20, wsz) == moe.MOE_ERR_ALIGNMENT
+    assert _call(lib, c, bad, 1 << 20, wsz) == moe.MOE_ERR_ALIGNMENT
     # workspace too small / missing / misaligned
-    assert _call_layer(lib, c, good, 1 << 20, wsz - 1) == moe.MOE_ERR_WORKSPACE
-    assert _call_layer(lib, c, good, 0, wsz) == moe.MOE_ERR_WORKSPACE
-    assert _call_layer(lib, c, good, (1 << 20) + 16, wsz) == moe.MOE_ERR_ALIGNMENT
+    assert _call(lib, c, good, 1 << 20, wsz - 1) == moe.MOE_ERR_WORKSPACE
+    assert _call(lib, c, good, 0, wsz) == moe.MOE_ERR_WORKSPACE
+    assert _call(lib, c, good, (1 << 20) + 16, wsz) == moe.MOE_ERR_ALIGNMENT
     # k > E
     ck = _cfg(mw.WORKLOADS["tiny"], k=9)
-    assert _call_layer(lib, ck, good, 1 << 20, wsz) == moe.MOE_ERR_INVALID_ARG
+    assert _call(lib, ck, good, 1 << 20, wsz) == moe.MOE_ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
-def test_valid_call_without_device_reports_no_device(lib):
+@pytest.mark.parametrize("entry", ["moe_layer_fwd", "moe_layer_fwd_gather"])
+def test_valid_call_without_device_reports_no_device(lib, entry):
     c = _cfg(mw.WORKLOADS["tiny"])
     good = [4096 * (i + 1) for i in range(8)]
     wsz = moe.moe_workspace_size(c)
-    assert _call_layer(lib, c, good, 1 << 20, wsz) == moe.MOE_ERR_NO_DEVICE
+    assert _call_layer(lib, c, good, 1 << 20, wsz, entry=entry) == moe.MOE_ERR_NO_DEVICE
 
 
 def test_wait_limit_rejects_bad_workspace_before_device_work(lib):
