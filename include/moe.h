@@ -106,6 +106,18 @@ MOE_API int64_t moe_capacity(const moe_config_t* cfg);
 /* Maximum number of kept assignments: T*k when dropless, else min(T*k, E*C). */
 MOE_API int64_t moe_max_kept(const moe_config_t* cfg);
 
+/* Expert column offsets for moe_config_t.ffn_offsets from a variable-size
+ * expert list of n_groups (count, size) pairs (nanoMOE notes, "Expert Size
+ * Computation" and "Offset Calculation"): each size is rounded up to a
+ * multiple of 128 and repeated count times, in list order, and the offsets
+ * are the running sums of those widths, starting at 0.  Host only, no
+ * device work.  Writes E + 1 entries to offsets (E = the sum of the counts,
+ * which must be at most max_experts) and returns E; returns -1 and writes
+ * nothing on a null pointer, n_groups < 0, a count < 0, a size < 1, E >
+ * max_experts or a total width above 2^31 - 1. */
+MOE_API int32_t moe_expert_offsets(const int32_t* counts, const int32_t* sizes, int32_t n_groups,
+                                   int32_t* offsets, int32_t max_experts);
+
 /* Bytes of workspace every entry point below needs for `cfg` (0 if cfg is
  * invalid).  One workspace of this size serves all calls; it holds the device
  * error word, the dispatch scratch and, for moe_layer_fwd, every

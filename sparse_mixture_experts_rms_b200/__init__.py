@@ -37,7 +37,7 @@ MOE_DEVERR_EXPERT_ID = 0x1
 MOE_DEVERR_TIMEOUT = 0x2
 MOE_DEVERR_TILE_TABLE = 0x4
 
-EXPORTED = ["moe_status_string", "moe_capacity", "moe_max_kept", "moe_workspace_size",
+EXPORTED = ["moe_status_string", "moe_capacity", "moe_max_kept", "moe_expert_offsets", "moe_workspace_size",
             "moe_workspace_init", "moe_get_device_error", "moe_set_wait_limit", "moe_route", "moe_dispatch",
             "moe_dispatch_noalloc",
             "moe_experts_fwd", "moe_experts_up", "moe_experts_down", "moe_combine",
@@ -96,6 +96,8 @@ def _lib():
         lib.moe_status_string.argtypes = [ctypes.c_int]
         lib.moe_capacity.restype = ctypes.c_int64
         lib.moe_capacity.argtypes = [cfgp]
+        lib.moe_expert_offsets.restype = ctypes.c_int32
+        lib.moe_expert_offsets.argtypes = [P, P, ctypes.c_int32, P, ctypes.c_int32]
         lib.moe_max_kept.restype = ctypes.c_int64
         lib.moe_max_kept.argtypes = [cfgp]
         lib.moe_workspace_size.restype = SZ
@@ -165,19 +167,19 @@ def _status_text(status: int) -> str:
         return f"status {status}"
 
 
-def ffn_offsets_from_sizes(expert_sizes: Sequence[Tuple[int, int]], block: int = 128) -> List[int]:
-    """Cumulative expert column offsets [E+1] from ``[(count, size), ...]``.
-
-    Each size is rounded up to a multiple of ``block`` and repeated ``count``
-    times; offsets are running sums of the widths (nanoMOE variable-size
-    experts notes, "Expert Size Computation" / "Offset Calculation").
-    """
-    offs = [0]
-    for count, size in expert_sizes:
-        w = -(-int(size) // block) * block
-        for _ in range(int(count)):
-            offs.append(offs[-1] + w)
-    return offs
+def ffn_offsets_from_sizes(expert_sizes: Sequence[Tuple[int, int]], max_experts: int = 64) -> List[int]:
+    """Cumulative expert column offsets [E+1] from ``[(count, size), ...]``,
+    computed by the library (moe_expert_offsets: sizes rounded up to 128,
+    repeated count times, running sums)."""
+    n = len(expert_sizes)
+    counts = (ctypes.c_int32 * max(n, 1))(*[int(c) for c, _ in expert_sizes])
+    sizes = (ctypes.c_int32 * max(n, 1))(*[int(s) for _, s in expert_sizes])
+    offs = (ctypes.c_int32 * (max_experts + 1))()
+    E = _lib().moe_expert_offsets(counts, sizes, n, offs, max_experts)
+    if E < 0:
+        raise ValueError(f"invalid expert sizes {list(expert_sizes)} (counts >= 0, sizes >= 1, "
+                         f"at most {max_experts} experts)")
+    return [int(offs[i]) for i in range(E + 1)]
 
 
 @dataclass

@@ -591,6 +591,26 @@ int64_t moe_max_kept(const moe_config_t* cfg) {
   return max_kept_of(*cfg);
 }
 
+int32_t moe_expert_offsets(const int32_t* counts, const int32_t* sizes, int32_t n_groups, int32_t* offsets,
+                           int32_t max_experts) {
+  if (counts == nullptr || sizes == nullptr || offsets == nullptr || n_groups < 0 || max_experts < 0) return -1;
+  int64_t E = 0, total = 0;
+  for (int32_t g = 0; g < n_groups; ++g) {
+    if (counts[g] < 0 || sizes[g] < 1) return -1;
+    const int64_t width = (static_cast<int64_t>(sizes[g]) + kBlockN - 1) / kBlockN * kBlockN;
+    E += counts[g];
+    total += width * counts[g];
+    if (E > max_experts || total > INT32_MAX) return -1;
+  }
+  int32_t e = 0;
+  offsets[0] = 0;
+  for (int32_t g = 0; g < n_groups; ++g) {
+    const int32_t width = static_cast<int32_t>((static_cast<int64_t>(sizes[g]) + kBlockN - 1) / kBlockN * kBlockN);
+    for (int32_t c = 0; c < counts[g]; ++c, ++e) offsets[e + 1] = offsets[e] + width;
+  }
+  return e;
+}
+
 size_t moe_workspace_size(const moe_config_t* cfg) {
   if (validate(cfg) != MOE_OK) return 0;
   return layout_of(*cfg).total;

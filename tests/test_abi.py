@@ -257,3 +257,30 @@ def test_mx_weights_layout(lib, name):
         assert off >= end and off % 256 == 0, part
         end = off + sizes[part]
     assert total - end >= 4 * 3 * d * F // 32
+
+
+def test_expert_offsets_printed_example(golden_dir):
+    """moe_expert_offsets against the nanoMOE notes' printed widths and offsets."""
+    import json
+    import os
+    with open(os.path.join(golden_dir, "nanomoe_variable_experts.json")) as f:
+        g = json.load(f)
+    assert moe.ffn_offsets_from_sizes([tuple(p) for p in g["expert_sizes"]]) == g["expert_offsets"]
+
+
+@pytest.mark.parametrize("sizes", [((8, 14336),), ((16, 4096),), ((64, 512),), ((1, 1), (2, 127), (0, 9), (3, 129)),
+                                   ((1, 2048), (7, 1024))])
+def test_expert_offsets_follow_the_rounding_rule(sizes):
+    widths = [-(-s // 128) * 128 for c, s in sizes for _ in range(c)]
+    assert moe.ffn_offsets_from_sizes(sizes) == [0] + list(np.cumsum(widths).astype(int))
+
+
+@pytest.mark.parametrize("bad", [((65, 128),), ((1, 0),), ((-1, 128),), ((2, 2 ** 30),)])
+def test_expert_offsets_reject_bad_lists(lib, bad):
+    n = len(bad)
+    counts = (ctypes.c_int32 * n)(*[c for c, _ in bad])
+    sizes = (ctypes.c_int32 * n)(*[s for _, s in bad])
+    offs = (ctypes.c_int32 * 65)(*([-7] * 65))
+    assert lib.moe_expert_offsets(counts, sizes, n, offs, 64) == -1
+    assert offs[0] == -7  # nothing written
+    assert lib.moe_expert_offsets(None, sizes, n, offs, 64) == -1
